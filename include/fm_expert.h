@@ -1,0 +1,202 @@
+/*
+ * fm_expert.h -- C ABI of the B200 (sm_100a) flow-matching action-expert
+ * denoise loop.
+ *
+ * What the library computes (the pages print no formula; every convention
+ * below is this library's reading, stated where it is used):
+ *
+ *   "LingBot-VLA on Thor (sm_110)", §1 Architecture / shapes: a 36-layer
+ *   flow-matching action expert, action chunk [1, 50, 75], denoise step count
+ *   10 / 25 / 50.  §2 Build: fused AdaRMSNorm, SwiGLU tail, QKV + RoPE.
+ *   §3 FlashAttention-4: grouped-query denoise attention.  §6 Notes: all
+ *   buffers pre-allocated, the loop captured in a CUDA graph, shapes fixed
+ *   per graph.
+ *   "LingBot-VLA v2 Examples", Configuration / CUDA Graph: the 36-layer
+ *   prefix KV cache is built per request and reused by all denoise steps; a
+ *   new instruction reuses the same denoise graph (here: fm_set_prefix never
+ *   forces a recapture).
+ *
+ * One velocity evaluation v(x, t) for a chunk x [T, A] (T = chunk_len):
+ *   m      = SiLU(sinusoid256(t) W1^T) W2^T, cut per layer into
+ *            (s_a, b_a, g_a, s_f, b_f, g_f) and a final (s_o, b_o)
+ *   h      = x W_in^T
+ *   per layer l:
+ *     y    = h (mean(h^2) + eps)^-1/2 (1 + s_a) + b_a
+ *     q,k,v= y Wq^T, y Wk^T, y Wv^T; rotate-half RoPE on q, k at P .. P+T-1
+ *     o    = softmax(q K^T / sqrt(hd)) V over [prefix K/V ; chunk k/v],
+ *            query head h reading KV head h / (H_q / H_kv), no mask
+ *     h   += g_a * (o Wo^T)
+ *     y    = AdaRMSNorm(h; s_f, b_f)
+ *     h   += g_f * ((SiLU(y Wg^T) * (y Wu^T)) Wd^T)
+ *   v      = AdaRMSNorm(h; s_o, b_o) W_out^T (+ out_bias)
+ * and fm_denoise integrates x <- x + dt v(x, t_k), t_k = 1 - k/n, dt = -1/n.
+ *
+ * Conventions of every entry point:
+ *   * Matrices are row-major W[out, in]; bf16 values are passed as their
+ *     16-bit patterns (uint16_t).  Activations handed in or out are fp32.
+ *   * Pointers marked "host or device" are classified with
+ *     cudaPointerGetAttributes; host memory may be pageable or pinned.
+ *   * `stream` is a cudaStream_t (NULL = legacy default stream).  Calls on
+ *     device buffers are stream-ordered and asynchronous; a call that writes
+ *     to a host buffer synchronises `stream` before it returns.
+ *   * A handle is not thread-safe: use it from one host thread (and one
+ *     stream at a time).  Different handles are independent.
+ *   * On error the call returns a non-zero fm_status, leaves outputs
+ *     unspecified, and fm_last_error(handle) describes the failure.  A device
+ *     wait that exceeds its bound is reported as FM_ERR_TIMEOUT by the next
+ *     call that synchronises (fm_sync, or any call writing host memory).
+ */
+#ifndef FM_EXPERT_H
+#define FM_EXPERT_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define FM_ABI_VERSION 1
+
+typedef enum fm_status {
+  FM_OK = 0,
+  FM_ERR_INVALID_ARG = 1,   /* null pointer, bad shape, size beyond capacity   */
+  FM_ERR_NOT_READY = 2,     /* fm_set_prefix has not been called for this batch */
+  FM_ERR_OOM = 3,           /* device allocation failed                         */
+  FM_ERR_CUDA = 4,          /* a CUDA call failed (text in fm_last_error)       */
+  FM_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up               */
+  FM_ERR_UNSUPPORTED = 6    /* shape or device this build cannot run            */
+} fm_status;
+
+typedef enum fm_wtype {
+  FM_W_BF16 = 0,            /* per-layer linears kept in bf16                   */
+  FM_W_FP8_E4M3 = 1         /* per-layer linears quantised to E4M3, one fp32
+                               scale per output row (s = absmax / 448)          */
+} fm_wtype;
+
+/* Model shape and capacities.  Requirements (checked by fm_expert_create):
+ * d_model, d_ff and n_q_heads*head_dim multiples of 64; head_dim even and
+ * <= 128; n_q_heads a multiple of n_kv_heads; chunk_len <= 50 rows per
+ * request fit one 64-row tile; action_dim <= 128; max_steps <= 64. */
+typedef struct fm_config {
+  int n_layers;      /* L: transformer layers of the expert (36)              */
+  int d_model;       /* d: residual width (1024)                              */
+  int n_q_heads;     /* H_q (16)                                              */
+  int n_kv_heads;    /* H_kv (2)                                              */
+  int head_dim;      /* hd (128)                                              */
+  int d_ff;          /* F: SwiGLU width (4096)                                */
+  int action_dim;    /* A: action dimension (75; 55 for the v2 chunk)         */
+  int chunk_len;     /* T: action horizon (50)                                */
+  int max_prefix;    /* capacity for P, the prefix length                     */
+  int max_batch;     /* capacity for B, requests per call                     */
+  int max_steps;     /* capacity for n, Euler steps per call                  */
+  float rms_eps;     /* AdaRMSNorm epsilon (1e-6)                             */
+  float rope_base;   /* RoPE base (1e4)                                       */
+  int wtype;         /* fm_wtype                                              */
+} fm_config;
+
+/* Per-layer weights, bf16 bits, [out, in], host or device. */
+typedef struct fm_layer_weights {
+  const uint16_t *wq;      /* [H_q*hd, d]   query projection                 */
+  const uint16_t *wk;      /* [H_kv*hd, d]  key projection                   */
+  const uint16_t *wv;      /* [H_kv*hd, d]  value projection                 */
+  const uint16_t *wo;      /* [d, H_q*hd]   attention output projection      */
+  const uint16_t *w_gate;  /* [F, d]        SwiGLU gate                      */
+  const uint16_t *w_up;    /* [F, d]        SwiGLU up                        */
+  const uint16_t *w_down;  /* [d, F]        SwiGLU down                      */
+} fm_layer_weights;
+
+typedef struct fm_weights {
+  const uint16_t *time_w1;   /* [d, 256]           time MLP, first linear    */
+  const uint16_t *time_w2;   /* [L*6*d + 2*d, d]   time MLP, second linear   */
+  const uint16_t *in_proj;   /* [d, A]             action in-projection      */
+  const uint16_t *out_proj;  /* [A, d]             action out-projection     */
+  const float *out_bias;     /* [A] fp32 or NULL: constant added to v (a test
+                                hook to build a constant velocity field)     */
+  const fm_layer_weights *layers;   /* [L], host memory                      */
+} fm_weights;
+
+typedef struct fm_expert fm_expert;
+
+/* Create a handle on `device`.  COPIES every weight into a library-owned,
+ * kernel-ready arena (and, for FM_W_FP8_E4M3, quantises the per-layer
+ * linears itself); the caller may free its copies when the call returns.
+ * Allocates every buffer the loop needs for the capacities in `cfg`.
+ * Returns FM_ERR_INVALID_ARG for a bad config, FM_ERR_UNSUPPORTED for a
+ * device that is not sm_100, FM_ERR_OOM when the arena does not fit. */
+fm_status fm_expert_create(const fm_config *cfg, const fm_weights *w, int device,
+                           fm_expert **out);
+
+/* Load the cached prefix K/V of `batch` requests, P = prefix_len rows each:
+ * k[l], v[l] point to bf16 bits [batch, P, H_kv, hd] (host or device), one
+ * pointer per layer; K is taken as already rotated.  The data is copied into
+ * the handle's fixed-capacity cache; P and the RoPE positions P .. P+T-1 are
+ * stored on the device, so graphs captured earlier stay valid ("LingBot-VLA
+ * v2 Examples", CUDA Graph: new instructions reuse the denoise graph).
+ * Requires 0 <= prefix_len <= max_prefix and 1 <= batch <= max_batch. */
+fm_status fm_set_prefix(fm_expert *h, const uint16_t *const *k, const uint16_t *const *v,
+                        int batch, int prefix_len, void *stream);
+
+/* Denoise `batch` chunks: x0 and out are fp32 [batch, T, A], host or device
+ * (independently); out may alias x0.  Runs the time MLP once, then `steps`
+ * Euler steps from t = 1 to t = 0 ("LingBot-VLA on Thor (sm_110)", §1: the
+ * denoise step count is configurable, 10 / 25 / 50).  The first call for a
+ * given (batch, steps) captures a CUDA graph; later calls replay it.
+ * batch must equal the batch of the last fm_set_prefix (else
+ * FM_ERR_NOT_READY); 1 <= steps <= max_steps. */
+fm_status fm_denoise(fm_expert *h, const float *x0, int batch, int steps, float *out,
+                     void *stream);
+
+/* Test hook: one velocity evaluation v(x, t_k) with t_k = 1 - step_index/steps,
+ * without the Euler update.  x, v_out: fp32 [batch, T, A], host or device. */
+fm_status fm_velocity(fm_expert *h, const float *x, int batch, int step_index, int steps,
+                      float *v_out, void *stream);
+
+/* Test hook: the modulation rows m_k for t_k = 1 - k/steps, k < steps, as
+ * fp32 [steps, L*6*d + 2*d] into m_out (host or device). */
+fm_status fm_time_modulation(fm_expert *h, int steps, float *m_out, void *stream);
+
+/* Test hook: per-layer intermediates of one velocity evaluation for request 0
+ * (batch must be 1).  Writes, into host memory `trace` of fm_trace_bytes()
+ * bytes, for each layer l in order (T = chunk_len):
+ *   h_in  fp32 [T, d]           residual stream entering the layer
+ *   q     fp32 [T, H_q*hd]      query after RoPE (bf16 values, widened)
+ *   k     fp32 [T, H_kv*hd]     chunk key after RoPE (bf16 values)
+ *   v     fp32 [T, H_kv*hd]     chunk value (bf16 values)
+ *   o     fp32 [T, H_q*hd]      attention output (bf16 values)
+ *   h_mid fp32 [T, d]           after the attention residual
+ *   u     fp32 [T, F]           SwiGLU product (bf16 values)
+ *   h_out fp32 [T, d]           after the FFN residual
+ * then v fp32 [T, A].  Synchronises `stream`. */
+size_t fm_trace_bytes(const fm_expert *h);
+fm_status fm_trace_velocity(fm_expert *h, const float *x, int step_index, int steps,
+                            float *trace, void *stream);
+
+/* Test hook: the E4M3 codes [out, in] and fp32 row scales [out] the handle
+ * holds for per-layer linear `which` (0 wq, 1 wk, 2 wv, 3 wo, 4 w_gate,
+ * 5 w_up, 6 w_down) of `layer`; host buffers.  FM_ERR_INVALID_ARG for a bf16
+ * handle. */
+fm_status fm_get_fp8_weights(fm_expert *h, int layer, int which, uint8_t *codes,
+                             float *scale);
+
+/* Wait for `stream`, then report (and clear) any device-side timeout. */
+fm_status fm_sync(fm_expert *h, void *stream);
+
+/* Launch geometry the handle chose: CTAs per cluster, clusters, CTAs. */
+fm_status fm_get_geometry(const fm_expert *h, int *cluster_size, int *n_clusters,
+                          int *n_ctas);
+
+/* Release the handle and every device buffer it owns; NULL is a no-op.
+ * Returns the number of device bytes released. */
+size_t fm_expert_destroy(fm_expert *h);
+
+/* Text of the last error on this handle ("" if none); NULL handle: the last
+ * error of a failed fm_expert_create on this thread. */
+const char *fm_last_error(const fm_expert *h);
+const char *fm_status_string(fm_status s);
+int fm_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* FM_EXPERT_H */

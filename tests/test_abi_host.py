@@ -1,0 +1,89 @@
+"""Host-side checks of the C ABI (no GPU needed): the library loads, exports
+every entry point the header declares, and rejects bad arguments before it
+touches a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from vla_flow_matching_denoise_b200 import binding, synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = []
+    inc = os.path.join(ROOT, "include")
+    for f in os.listdir(inc):
+        if f.endswith(".h"):
+            src = open(os.path.join(inc, f)).read()
+            src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+            names += re.findall(r"\b(fm_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_header_declares_the_binding_exports():
+    assert set(_declared()) == set(binding.EXPORTS)
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings_and_version(lib):
+    assert lib.fm_abi_version() == 1
+    assert lib.fm_status_string(0) == b"FM_OK"
+    assert lib.fm_status_string(5) == b"FM_ERR_TIMEOUT"
+
+
+def test_null_handles_are_safe(lib):
+    assert lib.fm_expert_destroy(None) == 0
+    assert lib.fm_trace_bytes(None) == 0
+    assert lib.fm_sync(None, None) == 1
+    assert lib.fm_denoise(None, None, 1, 10, None, None) == 1
+
+
+def _cfg(**kw):
+    c = binding.make_config(synth.WORKLOADS["tiny"])
+    for k, v in kw.items():
+        setattr(c, k, v)
+    return c
+
+
+@pytest.mark.parametrize("field,value,status", [
+    ("d_model", 100, 1),          # not a multiple of 64
+    ("head_dim", 96, 6),          # unsupported head width
+    ("n_q_heads", 3, 1),          # not a multiple of n_kv_heads
+    ("chunk_len", 64, 6),         # more than one 50-row tile
+    ("max_steps", 65, 1),         # modulation rows per tile
+    ("rms_eps", 0.0, 1),
+    ("wtype", 7, 1),
+    ("max_batch", 0, 1),
+])
+def test_create_rejects_bad_config_before_touching_the_device(lib, field, value, status):
+    cfg = _cfg(**{field: value})
+    h = ctypes.c_void_p()
+    w = binding.FmWeights()
+    st = lib.fm_expert_create(ctypes.byref(cfg), ctypes.byref(w), 0, ctypes.byref(h))
+    assert st == status, lib.fm_last_error(None)
+    assert not h.value
+    assert lib.fm_last_error(None)
+
+
+def test_create_rejects_null_weights(lib):
+    cfg = _cfg()
+    h = ctypes.c_void_p()
+    assert lib.fm_expert_create(ctypes.byref(cfg), None, 0, ctypes.byref(h)) == 1
+    assert lib.fm_expert_create(ctypes.byref(cfg), ctypes.byref(binding.FmWeights()), 0,
+                                ctypes.byref(h)) == 1
+
+
+def test_binding_raises_when_library_missing(tmp_path):
+    with pytest.raises(FileNotFoundError):
+        binding._lib = None
+        try:
+            binding.load(str(tmp_path / "nope.so"))
+        finally:
+            binding._lib = None

@@ -1,0 +1,239 @@
+"""Python binding of the C ABI in include/fm_expert.h (argument marshalling only).
+
+Every step of the denoise loop runs in the CUDA kernels of libfm_expert.so;
+this module only turns numpy arrays (host memory) and torch CUDA tensors
+(device memory) into pointers and back.  It raises when the shared library
+is missing: there is no other implementation to fall back to.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, List, Optional, Sequence
+
+import numpy as np
+
+from .synth import LAYER_KEYS, ExpertShape
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libfm_expert.so")
+
+FM_W_BF16 = 0
+FM_W_FP8_E4M3 = 1
+
+STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_NOT_READY", 3: "FM_ERR_OOM",
+          4: "FM_ERR_CUDA", 5: "FM_ERR_TIMEOUT", 6: "FM_ERR_UNSUPPORTED"}
+
+# Every symbol include/fm_expert.h declares.
+EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity", "fm_time_modulation",
+           "fm_trace_bytes", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
+           "fm_get_geometry", "fm_expert_destroy", "fm_last_error", "fm_status_string",
+           "fm_abi_version")
+
+
+class FmConfig(ctypes.Structure):
+    _fields_ = [("n_layers", ctypes.c_int), ("d_model", ctypes.c_int), ("n_q_heads", ctypes.c_int),
+                ("n_kv_heads", ctypes.c_int), ("head_dim", ctypes.c_int), ("d_ff", ctypes.c_int),
+                ("action_dim", ctypes.c_int), ("chunk_len", ctypes.c_int),
+                ("max_prefix", ctypes.c_int), ("max_batch", ctypes.c_int),
+                ("max_steps", ctypes.c_int), ("rms_eps", ctypes.c_float),
+                ("rope_base", ctypes.c_float), ("wtype", ctypes.c_int)]
+
+
+_P16 = ctypes.POINTER(ctypes.c_uint16)
+
+
+class FmLayerWeights(ctypes.Structure):
+    _fields_ = [(k, ctypes.c_void_p) for k in LAYER_KEYS]
+
+
+class FmWeights(ctypes.Structure):
+    _fields_ = [("time_w1", ctypes.c_void_p), ("time_w2", ctypes.c_void_p),
+                ("in_proj", ctypes.c_void_p), ("out_proj", ctypes.c_void_p),
+                ("out_bias", ctypes.c_void_p), ("layers", ctypes.POINTER(FmLayerWeights))]
+
+
+class FmError(RuntimeError):
+    def __init__(self, call: str, status: int, text: str):
+        super().__init__(f"{call} -> {STATUS.get(status, status)}: {text}")
+        self.status = status
+
+
+_lib: Optional[ctypes.CDLL] = None
+
+
+def load(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load the C-ABI library (built by vla_flow_matching_denoise_b200.build)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise FileNotFoundError(f"{path} is missing: run `python -m vla_flow_matching_denoise_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, ip, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+    lib.fm_expert_create.argtypes = [ctypes.POINTER(FmConfig), ctypes.POINTER(FmWeights), ip,
+                                     ctypes.POINTER(vp)]
+    lib.fm_set_prefix.argtypes = [vp, ctypes.POINTER(vp), ctypes.POINTER(vp), ip, ip, vp]
+    lib.fm_denoise.argtypes = [vp, vp, ip, ip, vp, vp]
+    lib.fm_velocity.argtypes = [vp, vp, ip, ip, ip, vp, vp]
+    lib.fm_time_modulation.argtypes = [vp, ip, vp, vp]
+    lib.fm_trace_bytes.argtypes = [vp]
+    lib.fm_trace_bytes.restype = sz
+    lib.fm_trace_velocity.argtypes = [vp, vp, ip, ip, vp, vp]
+    lib.fm_get_fp8_weights.argtypes = [vp, ip, ip, vp, vp]
+    lib.fm_sync.argtypes = [vp, vp]
+    lib.fm_get_geometry.argtypes = [vp, ctypes.POINTER(ip), ctypes.POINTER(ip), ctypes.POINTER(ip)]
+    lib.fm_expert_destroy.argtypes = [vp]
+    lib.fm_expert_destroy.restype = sz
+    lib.fm_last_error.argtypes = [vp]
+    lib.fm_last_error.restype = ctypes.c_char_p
+    lib.fm_status_string.argtypes = [ip]
+    lib.fm_status_string.restype = ctypes.c_char_p
+    lib.fm_abi_version.restype = ip
+    for name in ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity",
+                 "fm_time_modulation", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
+                 "fm_get_geometry"):
+        getattr(lib, name).restype = ip
+    _lib = lib
+    return lib
+
+
+def _ptr(a) -> Optional[int]:
+    """Address of a numpy array (host) or a torch tensor (host or device)."""
+    if a is None:
+        return None
+    if isinstance(a, np.ndarray):
+        if not a.flags["C_CONTIGUOUS"]:
+            raise ValueError("array must be C-contiguous")
+        return a.ctypes.data
+    if hasattr(a, "data_ptr"):
+        if not a.is_contiguous():
+            raise ValueError("tensor must be contiguous")
+        return a.data_ptr()
+    raise TypeError(f"unsupported buffer type {type(a)}")
+
+
+def _stream(stream) -> Optional[int]:
+    if stream is None:
+        try:
+            import torch
+            if torch.cuda.is_available():
+                return torch.cuda.current_stream().cuda_stream
+        except Exception:
+            pass
+        return None
+    return stream if isinstance(stream, int) else stream.cuda_stream
+
+
+def make_config(shape: ExpertShape, max_prefix: Optional[int] = None, max_batch: Optional[int] = None,
+                max_steps: int = 64) -> FmConfig:
+    return FmConfig(shape.n_layers, shape.d_model, shape.n_q_heads, shape.n_kv_heads, shape.head_dim,
+                    shape.d_ff, shape.action_dim, shape.chunk_len,
+                    shape.prefix_len if max_prefix is None else max_prefix,
+                    shape.batch if max_batch is None else max_batch, max_steps,
+                    shape.rms_eps, shape.rope_base, FM_W_FP8_E4M3 if shape.fp8 else FM_W_BF16)
+
+
+class Expert:
+    """One fm_expert handle: weights copied in at construction."""
+
+    def __init__(self, shape: ExpertShape, weights: Dict, device: int = 0,
+                 max_prefix: Optional[int] = None, max_batch: Optional[int] = None,
+                 max_steps: int = 64, out_bias: Optional[np.ndarray] = None):
+        self.lib = load()
+        self.shape = shape
+        self.cfg = make_config(shape, max_prefix, max_batch, max_steps)
+        layers = (FmLayerWeights * shape.n_layers)()
+        for i, lw in enumerate(weights["layers"]):
+            for k in LAYER_KEYS:
+                setattr(layers[i], k, _ptr(lw[k]))
+        bias = None if out_bias is None else np.ascontiguousarray(out_bias, dtype=np.float32)
+        w = FmWeights(_ptr(weights["time_w1"]), _ptr(weights["time_w2"]), _ptr(weights["in_proj"]),
+                      _ptr(weights["out_proj"]), _ptr(bias), layers)
+        h = ctypes.c_void_p()
+        st = self.lib.fm_expert_create(ctypes.byref(self.cfg), ctypes.byref(w), device, ctypes.byref(h))
+        if st != 0:
+            raise FmError("fm_expert_create", st, self.lib.fm_last_error(None).decode())
+        self.h = h
+
+    # ------------------------------------------------------------------ helpers
+    def _check(self, call: str, st: int):
+        if st != 0:
+            raise FmError(call, st, self.lib.fm_last_error(self.h).decode())
+
+    def close(self) -> int:
+        if getattr(self, "h", None):
+            n = self.lib.fm_expert_destroy(self.h)
+            self.h = None
+            return n
+        return 0
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def geometry(self):
+        a, b, c = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+        self._check("fm_get_geometry", self.lib.fm_get_geometry(self.h, ctypes.byref(a), ctypes.byref(b),
+                                                                ctypes.byref(c)))
+        return a.value, b.value, c.value
+
+    # ------------------------------------------------------------------ calls
+    def set_prefix(self, k: Sequence, v: Sequence, batch: int, prefix_len: int, stream=None):
+        L = self.shape.n_layers
+        kp = (ctypes.c_void_p * L)(*[_ptr(x) for x in k])
+        vp = (ctypes.c_void_p * L)(*[_ptr(x) for x in v])
+        self._check("fm_set_prefix", self.lib.fm_set_prefix(self.h, kp, vp, batch, prefix_len, _stream(stream)))
+
+    def denoise(self, x0, steps: int, out=None, stream=None):
+        """x0: fp32 [B, T, A] numpy (host) or torch (device).  Returns `out`."""
+        if out is None:
+            out = np.empty_like(x0) if isinstance(x0, np.ndarray) else x0.new_empty(x0.shape)
+        B = x0.shape[0]
+        self._check("fm_denoise", self.lib.fm_denoise(self.h, _ptr(x0), B, steps, _ptr(out), _stream(stream)))
+        return out
+
+    def velocity(self, x, step_index: int, steps: int, out=None, stream=None):
+        if out is None:
+            out = np.empty_like(x) if isinstance(x, np.ndarray) else x.new_empty(x.shape)
+        self._check("fm_velocity", self.lib.fm_velocity(self.h, _ptr(x), x.shape[0], step_index, steps,
+                                                         _ptr(out), _stream(stream)))
+        return out
+
+    def time_modulation(self, steps: int, stream=None) -> np.ndarray:
+        n_mod = self.shape.n_mod
+        out = np.empty((steps, n_mod), dtype=np.float32)
+        self._check("fm_time_modulation", self.lib.fm_time_modulation(self.h, steps, _ptr(out), _stream(stream)))
+        return out
+
+    def trace_velocity(self, x: np.ndarray, step_index: int, steps: int, stream=None) -> List[Dict]:
+        s = self.shape
+        n = self.lib.fm_trace_bytes(self.h) // 4
+        buf = np.empty(n, dtype=np.float32)
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        self._check("fm_trace_velocity", self.lib.fm_trace_velocity(self.h, _ptr(x), step_index, steps,
+                                                                     _ptr(buf), _stream(stream)))
+        T, d, F = s.chunk_len, s.d_model, s.d_ff
+        qn, kn = s.n_q_heads * s.head_dim, s.n_kv_heads * s.head_dim
+        out, o = [], 0
+        for _ in range(s.n_layers):
+            rec = {}
+            for name, w in (("h_in", d), ("q", qn), ("k", kn), ("v", kn), ("o", qn), ("h_mid", d),
+                            ("u", F), ("h_out", d)):
+                rec[name] = buf[o:o + T * w].reshape(T, w)
+                o += T * w
+            out.append(rec)
+        out.append({"v": buf[o:o + T * s.action_dim].reshape(T, s.action_dim)})
+        return out
+
+    def get_fp8_weights(self, layer: int, which: int, rows: int, cols: int):
+        codes = np.empty((rows, cols), dtype=np.uint8)
+        scale = np.empty(rows, dtype=np.float32)
+        self._check("fm_get_fp8_weights", self.lib.fm_get_fp8_weights(self.h, layer, which, _ptr(codes),
+                                                                       _ptr(scale)))
+        return codes, scale
+
+    def sync(self, stream=None):
+        self._check("fm_sync", self.lib.fm_sync(self.h, _stream(stream)))

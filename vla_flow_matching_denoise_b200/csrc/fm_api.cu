@@ -1,0 +1,915 @@
+// Host engine behind include/fm_expert.h: argument checks, the work plan,
+// weight packing into the kernel-ready arena, buffers, the prefix cache, the
+// per-(batch, steps) CUDA-graph cache and the test hooks.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <map>
+#include <string>
+#include <utility>
+#include <vector>
+
+#include "../../include/fm_expert.h"
+#include "fm_internal.h"
+#include "fm_launch.h"
+
+using namespace fm;
+
+namespace {
+
+thread_local std::string g_create_error;
+
+struct DevBuf {
+  void* p = nullptr;
+  size_t n = 0;
+};
+
+}  // namespace
+
+struct fm_expert {
+  fm_config cfg{};
+  int device = 0;
+  int n_sms = 0;
+  int n_clusters = 0;
+  int n_ctas = 0;
+  int n_mod = 0;
+  GemmPlan plan[4]{};
+  int uc = 0;
+  std::string err;
+  std::vector<DevBuf> bufs;
+  size_t bytes = 0;
+  cudaStream_t cap_stream = nullptr;
+  // weights
+  uint8_t* arena = nullptr;
+  uint64_t layer_bytes = 0;
+  uint32_t* span_off = nullptr;
+  uint8_t* w2_packed = nullptr;
+  uint16_t* w1 = nullptr;
+  uint16_t* w_in = nullptr;
+  uint16_t* w_out = nullptr;
+  float* out_bias = nullptr;
+  // fp8 copies kept for fm_get_fp8_weights
+  std::vector<uint8_t*> fp8_codes;   // [L*7]
+  std::vector<float*> fp8_scale;     // [L*7]
+  // buffers
+  float* mod = nullptr;
+  uint16_t* h1_act = nullptr;
+  float* rope = nullptr;
+  int* P_dev = nullptr;
+  float* x = nullptr;      // [B_cap, T, A]
+  float* vbuf = nullptr;   // [B_cap, T, A]
+  float* h_a = nullptr;
+  float* h_b = nullptr;
+  uint16_t* z_a = nullptr;
+  uint16_t* z_f = nullptr;
+  uint16_t* o_act = nullptr;
+  uint16_t* u_act = nullptr;
+  float* sumsq_a = nullptr;
+  float* sumsq_f = nullptr;
+  uint16_t* qbuf = nullptr;
+  uint16_t* kcache = nullptr;
+  uint16_t* vcache = nullptr;
+  uint32_t* bar_count = nullptr;
+  uint32_t* err_word = nullptr;
+  int S_max = 0;
+  int prefix_batch = 0;   // batch of the last fm_set_prefix (0 = none)
+  int prefix_len = 0;
+  std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
+  std::map<std::pair<int, int>, cudaGraph_t> graph_defs;
+};
+
+namespace {
+
+fm_status set_err(fm_expert* h, fm_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  if (h) h->err = buf;
+  else g_create_error = buf;
+  return s;
+}
+
+#define CK(call)                                                                          \
+  do {                                                                                    \
+    cudaError_t e_ = (call);                                                              \
+    if (e_ != cudaSuccess)                                                                \
+      return set_err(h, e_ == cudaErrorMemoryAllocation ? FM_ERR_OOM : FM_ERR_CUDA,       \
+                     "%s: %s (%s:%d)", #call, cudaGetErrorString(e_), __FILE__, __LINE__); \
+  } while (0)
+
+template <class T>
+fm_status dalloc(fm_expert* h, T** out, size_t bytes) {
+  void* p = nullptr;
+  cudaError_t e = cudaMalloc(&p, bytes ? bytes : 16);
+  if (e != cudaSuccess)
+    return set_err(h, FM_ERR_OOM, "cudaMalloc(%zu bytes): %s", bytes, cudaGetErrorString(e));
+  e = cudaMemset(p, 0, bytes ? bytes : 16);
+  if (e != cudaSuccess) return set_err(h, FM_ERR_CUDA, "cudaMemset: %s", cudaGetErrorString(e));
+  h->bufs.push_back({p, bytes});
+  h->bytes += bytes;
+  *out = static_cast<T*>(p);
+  return FM_OK;
+}
+#define DALLOC(ptr, bytes)                        \
+  do {                                            \
+    fm_status s_ = dalloc(h, &(ptr), (bytes));    \
+    if (s_ != FM_OK) return s_;                   \
+  } while (0)
+
+int round_up(int x, int m) { return (x + m - 1) / m * m; }
+
+// Plans one linear over `nc` clusters (see GemmPlan).  `own_mult` is the
+// granularity of the columns a CTA owns after the reduction.
+bool plan_gemm(GemmPlan& g, int N, int K, int nc, int pref_ks, int own_mult) {
+  g.N = N;
+  g.K = K;
+  int ks = pref_ks;
+  while (ks > 1 && ((K / 64) % ks != 0)) ks /= 2;
+  if (K % 64 != 0) return false;
+  g.KS = ks;
+  g.NS = kClusterSize / ks;
+  const int per = (N + nc * g.NS - 1) / (nc * g.NS);
+  g.Ng = round_up(std::max(per, 1), std::max(16, ks * own_mult));
+  if (g.Ng > 256) return false;
+  g.own = g.Ng / ks;
+  g.kslice = K / ks;
+  g.nchunk = g.kslice / 64;
+  g.chunk_bytes = (uint32_t)g.Ng * 128u;
+  g.busy_clusters = std::min(nc, (N + g.NS * g.Ng - 1) / (g.NS * g.Ng));
+  if ((size_t)g.nchunk * 8192 > (size_t)kWorkBytes) return false;
+  if ((size_t)(kBiasRow + 1) * g.Ng * 4 > (size_t)kWorkBytes) return false;
+  return true;
+}
+
+// Source row (in the concatenated matrix of gemm g) of packed channel q of the
+// n-group (cluster c, group ng); -1 for padding.
+int source_row(const fm_expert* h, int g, int c, int ng, int q) {
+  const fm_config& cf = h->cfg;
+  const GemmPlan& gp = h->plan[g];
+  const int pc = (c * gp.NS + ng) * gp.Ng + q;
+  if (g == G_QKV) {
+    const int qn = cf.n_q_heads * cf.head_dim, kn = cf.n_kv_heads * cf.head_dim;
+    if (pc >= gp.N) return -1;
+    if (pc < qn + kn) {
+      // rotate-half partners (i, i + hd/2) are packed next to each other
+      const int base = pc < qn ? 0 : qn;
+      const int nn = pc - base;
+      const int head = nn / cf.head_dim, w = nn % cf.head_dim;
+      const int i = w >> 1;
+      return base + head * cf.head_dim + i + (w & 1) * (cf.head_dim / 2);
+    }
+    return pc;
+  }
+  if (g == G_GU) {
+    const int ks = q / gp.own, rr = q % gp.own, uown = gp.own / 2;
+    const int u = (c * gp.NS + ng) * h->uc + ks * uown + (rr % uown);
+    if (u >= cf.d_ff) return -1;
+    return rr < uown ? u : cf.d_ff + u;
+  }
+  return pc < gp.N ? pc : -1;
+}
+
+fm_status build_plan(fm_expert* h) {
+  const fm_config& c = h->cfg;
+  const int nc = h->n_clusters;
+  const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+  if (!plan_gemm(h->plan[G_QKV], qkv, c.d_model, nc, 8, 2) ||
+      !plan_gemm(h->plan[G_O], c.d_model, c.n_q_heads * c.head_dim, nc, 8, 8) ||
+      !plan_gemm(h->plan[G_GU], 2 * c.d_ff, c.d_model, nc, 4, 16) ||
+      !plan_gemm(h->plan[G_DOWN], c.d_model, c.d_ff, nc, 8, 8))
+    return set_err(h, FM_ERR_UNSUPPORTED, "no work plan for this shape on %d clusters", nc);
+  h->uc = h->plan[G_GU].Ng / 2;
+  return FM_OK;
+}
+
+fm_status upload_rows(fm_expert* h, uint16_t* dst, const uint16_t* src, size_t elems, const char* what) {
+  if (!src) return set_err(h, FM_ERR_INVALID_ARG, "weight %s is NULL", what);
+  CK(cudaMemcpy(dst, src, elems * 2, cudaMemcpyDefault));
+  return FM_OK;
+}
+
+fm_status pack_weights(fm_expert* h, const fm_weights* w) {
+  const fm_config& c = h->cfg;
+  const int d = c.d_model, F = c.d_ff, qn = c.n_q_heads * c.head_dim,
+            kn = c.n_kv_heads * c.head_dim;
+  // Per-layer packing jobs (identical for every layer) and CTA spans.
+  std::vector<PackChunk> jobs;
+  std::vector<int32_t> rows;
+  std::vector<uint32_t> span(h->n_ctas + 1, 0);
+  uint64_t off = 0;
+  for (int cta = 0; cta < h->n_ctas; ++cta) {
+    span[cta] = (uint32_t)off;
+    const int cl = cta / kClusterSize, rank = cta % kClusterSize;
+    for (int g = 0; g < 4; ++g) {
+      const GemmPlan& gp = h->plan[g];
+      if (cl >= gp.busy_clusters) continue;
+      const int ng = rank / gp.KS, ks = rank % gp.KS;
+      const uint32_t roff = (uint32_t)rows.size();
+      for (int q = 0; q < gp.Ng; ++q) rows.push_back(source_row(h, g, cl, ng, q));
+      for (int i = 0; i < gp.nchunk; ++i) {
+        PackChunk pc{};
+        pc.dst_off = off;
+        pc.rowidx_off = roff;
+        pc.nrows = (uint16_t)gp.Ng;
+        pc.mat = (uint8_t)g;
+        pc.kb = (uint32_t)(ks * gp.nchunk + i);
+        jobs.push_back(pc);
+        off += gp.chunk_bytes;
+      }
+    }
+  }
+  span[h->n_ctas] = (uint32_t)off;
+  h->layer_bytes = off;
+  if (off > 0xFFFFFFFFull) return set_err(h, FM_ERR_UNSUPPORTED, "layer span too large");
+
+  PackChunk* d_jobs = nullptr;
+  int32_t* d_rows = nullptr;
+  uint16_t** d_mats = nullptr;
+  int* d_matk = nullptr;
+  DALLOC(h->arena, (size_t)c.n_layers * off);
+  DALLOC(h->span_off, span.size() * 4);
+  CK(cudaMemcpy(h->span_off, span.data(), span.size() * 4, cudaMemcpyHostToDevice));
+  // temporary buffers (freed at the end)
+  void* tmp[6] = {};
+  const size_t sz_qkv = (size_t)(qn + 2 * kn) * d, sz_o = (size_t)d * qn, sz_gu = (size_t)2 * F * d,
+               sz_dn = (size_t)d * F;
+  cudaError_t e = cudaSuccess;
+  e = cudaMalloc(&tmp[0], sz_qkv * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&tmp[1], sz_o * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&tmp[2], sz_gu * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&tmp[3], sz_dn * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&tmp[4], jobs.size() * sizeof(PackChunk) + rows.size() * 4 + 64);
+  if (e == cudaSuccess) e = cudaMalloc(&tmp[5], 4 * sizeof(void*) + 4 * sizeof(int));
+  fm_status st = FM_OK;
+  if (e != cudaSuccess) {
+    st = set_err(h, FM_ERR_OOM, "packing buffers: %s", cudaGetErrorString(e));
+  } else {
+    d_jobs = static_cast<PackChunk*>(tmp[4]);
+    d_rows = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(tmp[4]) + jobs.size() * sizeof(PackChunk));
+    d_mats = static_cast<uint16_t**>(tmp[5]);
+    d_matk = reinterpret_cast<int*>(static_cast<uint8_t*>(tmp[5]) + 4 * sizeof(void*));
+    uint16_t* mats[4] = {static_cast<uint16_t*>(tmp[0]), static_cast<uint16_t*>(tmp[1]),
+                         static_cast<uint16_t*>(tmp[2]), static_cast<uint16_t*>(tmp[3])};
+    const int matk[4] = {d, qn, d, F};
+    e = cudaMemcpy(d_jobs, jobs.data(), jobs.size() * sizeof(PackChunk), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(d_rows, rows.data(), rows.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(d_mats, mats, sizeof(mats), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(d_matk, matk, sizeof(matk), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) st = set_err(h, FM_ERR_CUDA, "pack tables: %s", cudaGetErrorString(e));
+    for (int l = 0; l < c.n_layers && st == FM_OK; ++l) {
+      const fm_layer_weights& lw = w->layers[l];
+      if (!lw.wq || !lw.wk || !lw.wv || !lw.wo || !lw.w_gate || !lw.w_up || !lw.w_down) {
+        st = set_err(h, FM_ERR_INVALID_ARG, "layer %d has a NULL weight", l);
+        break;
+      }
+      e = cudaMemcpy(mats[0], lw.wq, (size_t)qn * d * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess) e = cudaMemcpy(mats[0] + (size_t)qn * d, lw.wk, (size_t)kn * d * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess) e = cudaMemcpy(mats[0] + (size_t)(qn + kn) * d, lw.wv, (size_t)kn * d * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess) e = cudaMemcpy(mats[1], lw.wo, sz_o * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess) e = cudaMemcpy(mats[2], lw.w_gate, (size_t)F * d * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess) e = cudaMemcpy(mats[2] + (size_t)F * d, lw.w_up, (size_t)F * d * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess) e = cudaMemcpy(mats[3], lw.w_down, sz_dn * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess)
+        e = launch_pack(d_jobs, (int)jobs.size(), d_rows, d_mats, d_matk, h->arena + (size_t)l * off, 0);
+      if (e == cudaSuccess) e = cudaDeviceSynchronize();
+      if (e != cudaSuccess) st = set_err(h, FM_ERR_CUDA, "packing layer %d: %s", l, cudaGetErrorString(e));
+    }
+  }
+  for (void* p : tmp)
+    if (p) cudaFree(p);
+  if (st != FM_OK) return st;
+
+  // Time MLP: W1 plain bf16, W2 packed in tiles of 128 rows x 64 columns.
+  DALLOC(h->w1, (size_t)d * kTimeDim * 2);
+  st = upload_rows(h, h->w1, w->time_w1, (size_t)d * kTimeDim, "time_w1");
+  if (st != FM_OK) return st;
+  const int n_mod = h->n_mod;
+  const int ntiles = (n_mod + 127) / 128, nkb = d / 64;
+  DALLOC(h->w2_packed, (size_t)ntiles * nkb * 16384);
+  {
+    std::vector<PackChunk> tj;
+    std::vector<int32_t> tr((size_t)ntiles * 128);
+    for (int t = 0; t < ntiles; ++t) {
+      for (int q = 0; q < 128; ++q) tr[(size_t)t * 128 + q] = (t * 128 + q < n_mod) ? t * 128 + q : -1;
+      for (int kb = 0; kb < nkb; ++kb) {
+        PackChunk pc{};
+        pc.dst_off = ((uint64_t)t * nkb + kb) * 16384;
+        pc.rowidx_off = (uint32_t)t * 128;
+        pc.nrows = 128;
+        pc.mat = 0;
+        pc.kb = (uint32_t)kb;
+        tj.push_back(pc);
+      }
+    }
+    void* t2 = nullptr;
+    void* tt = nullptr;
+    e = cudaMalloc(&t2, (size_t)n_mod * d * 2);
+    if (e == cudaSuccess) e = cudaMalloc(&tt, tj.size() * sizeof(PackChunk) + tr.size() * 4 + 64);
+    if (e != cudaSuccess) {
+      if (t2) cudaFree(t2);
+      return set_err(h, FM_ERR_OOM, "time_w2 staging: %s", cudaGetErrorString(e));
+    }
+    PackChunk* dj = static_cast<PackChunk*>(tt);
+    int32_t* dr = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(tt) + tj.size() * sizeof(PackChunk));
+    uint16_t** dm = reinterpret_cast<uint16_t**>(d_mats);
+    // reuse a small device table for the matrix pointer / width
+    void* tm = nullptr;
+    e = cudaMalloc(&tm, sizeof(void*) + sizeof(int));
+    if (e == cudaSuccess) {
+      uint16_t* mp = static_cast<uint16_t*>(t2);
+      int kk = d;
+      e = cudaMemcpy(tm, &mp, sizeof(void*), cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(static_cast<uint8_t*>(tm) + sizeof(void*), &kk, sizeof(int), cudaMemcpyHostToDevice);
+    }
+    (void)dm;
+    if (e == cudaSuccess && !w->time_w2) e = cudaErrorInvalidValue;
+    if (e == cudaSuccess) e = cudaMemcpy(t2, w->time_w2, (size_t)n_mod * d * 2, cudaMemcpyDefault);
+    if (e == cudaSuccess) e = cudaMemcpy(dj, tj.data(), tj.size() * sizeof(PackChunk), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(dr, tr.data(), tr.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess)
+      e = launch_pack(dj, (int)tj.size(), dr, static_cast<uint16_t* const*>(tm),
+                      reinterpret_cast<const int*>(static_cast<uint8_t*>(tm) + sizeof(void*)), h->w2_packed, 0);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    cudaFree(t2);
+    cudaFree(tt);
+    if (tm) cudaFree(tm);
+    if (e != cudaSuccess) return set_err(h, FM_ERR_CUDA, "packing time_w2: %s", cudaGetErrorString(e));
+  }
+  DALLOC(h->w_in, (size_t)d * c.action_dim * 2);
+  st = upload_rows(h, h->w_in, w->in_proj, (size_t)d * c.action_dim, "in_proj");
+  if (st != FM_OK) return st;
+  DALLOC(h->w_out, (size_t)d * c.action_dim * 2);
+  st = upload_rows(h, h->w_out, w->out_proj, (size_t)d * c.action_dim, "out_proj");
+  if (st != FM_OK) return st;
+  if (w->out_bias) {
+    DALLOC(h->out_bias, (size_t)c.action_dim * 4);
+    CK(cudaMemcpy(h->out_bias, w->out_bias, (size_t)c.action_dim * 4, cudaMemcpyDefault));
+  }
+  return FM_OK;
+}
+
+fm_status check_config(const fm_config* c) {
+  fm_expert* h = nullptr;
+  if (!c) return set_err(h, FM_ERR_INVALID_ARG, "config is NULL");
+  if (c->n_layers < 1 || c->d_model < 64 || c->n_q_heads < 1 || c->n_kv_heads < 1 ||
+      c->d_ff < 64 || c->action_dim < 1 || c->chunk_len < 1 || c->max_prefix < 0 ||
+      c->max_batch < 1 || c->max_steps < 1)
+    return set_err(h, FM_ERR_INVALID_ARG, "non-positive size in config");
+  if (c->d_model % 64 || c->d_ff % 64 || (c->n_q_heads * c->head_dim) % 64)
+    return set_err(h, FM_ERR_INVALID_ARG, "d_model, d_ff and n_q_heads*head_dim must be multiples of 64");
+  if (c->head_dim != 64 && c->head_dim != 128)
+    return set_err(h, FM_ERR_UNSUPPORTED, "head_dim must be 64 or 128");
+  if (c->n_q_heads % c->n_kv_heads)
+    return set_err(h, FM_ERR_INVALID_ARG, "n_q_heads must be a multiple of n_kv_heads");
+  if (c->chunk_len > kMaxT) return set_err(h, FM_ERR_UNSUPPORTED, "chunk_len must be <= %d", kMaxT);
+  if (c->action_dim > 128) return set_err(h, FM_ERR_UNSUPPORTED, "action_dim must be <= 128");
+  if (c->d_model > 1024) return set_err(h, FM_ERR_UNSUPPORTED, "d_model must be <= 1024");
+  if (c->max_steps > kRows) return set_err(h, FM_ERR_INVALID_ARG, "max_steps must be <= %d", kRows);
+  if (!(c->rms_eps > 0.f) || !(c->rope_base > 0.f))
+    return set_err(h, FM_ERR_INVALID_ARG, "rms_eps and rope_base must be positive");
+  if (c->wtype != FM_W_BF16 && c->wtype != FM_W_FP8_E4M3)
+    return set_err(h, FM_ERR_INVALID_ARG, "unknown wtype %d", c->wtype);
+  return FM_OK;
+}
+
+void free_all(fm_expert* h) {
+  for (auto& kv : h->graphs) cudaGraphExecDestroy(kv.second);
+  for (auto& kv : h->graph_defs) cudaGraphDestroy(kv.second);
+  h->graphs.clear();
+  h->graph_defs.clear();
+  for (auto& b : h->bufs) cudaFree(b.p);
+  h->bufs.clear();
+  if (h->cap_stream) cudaStreamDestroy(h->cap_stream);
+  h->cap_stream = nullptr;
+}
+
+bool is_device_ptr(const void* p) {
+  cudaPointerAttributes a{};
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged;
+}
+
+StepParams base_params(const fm_expert* h) {
+  const fm_config& c = h->cfg;
+  StepParams p{};
+  p.L = c.n_layers;
+  p.d = c.d_model;
+  p.Hq = c.n_q_heads;
+  p.Hkv = c.n_kv_heads;
+  p.hd = c.head_dim;
+  p.F = c.d_ff;
+  p.A = c.action_dim;
+  p.T = c.chunk_len;
+  p.S_max = h->S_max;
+  p.B_cap = c.max_batch;
+  p.b = 0;
+  p.P_dev = h->P_dev;
+  p.eps = c.rms_eps;
+  p.n_clusters = h->n_clusters;
+  p.n_ctas = h->n_ctas;
+  for (int g = 0; g < 4; ++g) p.g[g] = h->plan[g];
+  p.uc = h->uc;
+  p.arena = h->arena;
+  p.layer_bytes = h->layer_bytes;
+  p.span_off = h->span_off;
+  p.w_in = h->w_in;
+  p.w_out = h->w_out;
+  p.out_bias = h->out_bias;
+  p.mod = h->mod;
+  p.n_mod = h->n_mod;
+  p.rope = h->rope;
+  p.x = h->x;
+  p.vbuf = h->vbuf;
+  p.h_a = h->h_a;
+  p.h_b = h->h_b;
+  p.z_a = h->z_a;
+  p.z_f = h->z_f;
+  p.o_act = h->o_act;
+  p.u_act = h->u_act;
+  p.sumsq_a = h->sumsq_a;
+  p.sumsq_f = h->sumsq_f;
+  p.qbuf = h->qbuf;
+  p.kcache = h->kcache;
+  p.vcache = h->vcache;
+  p.bar_count = h->bar_count;
+  p.err = h->err_word;
+  p.step0 = 0;
+  p.step1 = 0;
+  p.layer0 = 0;
+  p.layer1 = c.n_layers;
+  p.do_inproj = 1;
+  p.do_outproj = 1;
+  p.update_x = 1;
+  p.dt = 0.f;
+  p.spin_budget = 4000000000LL;   // ~2 s at 2 GHz
+  return p;
+}
+
+TimeParams time_params(const fm_expert* h, int steps) {
+  TimeParams t{};
+  t.n_steps = steps;
+  t.d = h->cfg.d_model;
+  t.n_mod = h->n_mod;
+  t.w1 = h->w1;
+  t.w2_packed = h->w2_packed;
+  t.h1_act = h->h1_act;
+  t.mod = h->mod;
+  t.err = h->err_word;
+  t.spin_budget = 4000000000LL;
+  return t;
+}
+
+// Enqueues one full denoise of `batch` requests (x already in h->x).
+cudaError_t enqueue_denoise(fm_expert* h, int batch, int steps, cudaStream_t st) {
+  cudaError_t e = cudaMemsetAsync(h->bar_count, 0, 4, st);
+  if (e != cudaSuccess) return e;
+  e = launch_time(time_params(h, steps), h->n_sms, st);
+  if (e != cudaSuccess) return e;
+  const size_t xs = (size_t)h->cfg.chunk_len * h->cfg.action_dim;
+  for (int b = 0; b < batch; ++b) {
+    StepParams p = base_params(h);
+    p.b = b;
+    p.x = h->x + b * xs;
+    p.vbuf = h->vbuf + b * xs;
+    p.step0 = 0;
+    p.step1 = steps;
+    p.dt = -1.0f / (float)steps;
+    if (b > 0) {
+      e = cudaMemsetAsync(h->bar_count, 0, 4, st);
+      if (e != cudaSuccess) return e;
+    }
+    e = launch_step(p, st);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+fm_status check_err_word(fm_expert* h) {
+  uint32_t w = 0;
+  CK(cudaMemcpy(&w, h->err_word, 4, cudaMemcpyDeviceToHost));
+  if (w) {
+    CK(cudaMemset(h->err_word, 0, 4));
+    return set_err(h, FM_ERR_TIMEOUT, "a device-side wait gave up (code 0x%x)", w);
+  }
+  return FM_OK;
+}
+
+}  // namespace
+
+extern "C" {
+#pragma GCC visibility push(default)
+
+int fm_abi_version(void) { return FM_ABI_VERSION; }
+
+const char* fm_status_string(fm_status s) {
+  switch (s) {
+    case FM_OK: return "FM_OK";
+    case FM_ERR_INVALID_ARG: return "FM_ERR_INVALID_ARG";
+    case FM_ERR_NOT_READY: return "FM_ERR_NOT_READY";
+    case FM_ERR_OOM: return "FM_ERR_OOM";
+    case FM_ERR_CUDA: return "FM_ERR_CUDA";
+    case FM_ERR_TIMEOUT: return "FM_ERR_TIMEOUT";
+    case FM_ERR_UNSUPPORTED: return "FM_ERR_UNSUPPORTED";
+  }
+  return "unknown fm_status";
+}
+
+const char* fm_last_error(const fm_expert* h) {
+  return h ? h->err.c_str() : g_create_error.c_str();
+}
+
+fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device, fm_expert** out) {
+  fm_expert* h = nullptr;
+  g_create_error.clear();
+  if (!out) return set_err(h, FM_ERR_INVALID_ARG, "out is NULL");
+  *out = nullptr;
+  fm_status st = check_config(cfg);
+  if (st != FM_OK) return st;
+  if (!w || !w->layers || !w->time_w1 || !w->time_w2 || !w->in_proj || !w->out_proj)
+    return set_err(h, FM_ERR_INVALID_ARG, "weights or a weight pointer is NULL");
+  int ndev = 0;
+  if (cudaGetDeviceCount(&ndev) != cudaSuccess || ndev == 0) {
+    cudaGetLastError();
+    return set_err(h, FM_ERR_UNSUPPORTED, "no CUDA device");
+  }
+  if (device < 0 || device >= ndev) return set_err(h, FM_ERR_INVALID_ARG, "device %d out of range", device);
+  cudaDeviceProp prop{};
+  if (cudaGetDeviceProperties(&prop, device) != cudaSuccess)
+    return set_err(h, FM_ERR_CUDA, "cudaGetDeviceProperties failed");
+  if (prop.major != 10 || prop.minor != 0)
+    return set_err(h, FM_ERR_UNSUPPORTED, "device %d is sm_%d%d; this build targets sm_100a", device,
+                   prop.major, prop.minor);
+  if (cudaSetDevice(device) != cudaSuccess) return set_err(h, FM_ERR_CUDA, "cudaSetDevice failed");
+
+  h = new fm_expert();
+  h->cfg = *cfg;
+  h->device = device;
+  h->n_sms = prop.multiProcessorCount;
+  const fm_config& c = h->cfg;
+  h->n_mod = c.n_layers * 6 * c.d_model + 2 * c.d_model;
+  h->S_max = c.max_prefix + c.chunk_len;
+  auto bail = [&](fm_status s) {
+    g_create_error = h->err;
+    free_all(h);
+    delete h;
+    return s;
+  };
+  int ncl = 0;
+  if (step_max_clusters(&ncl) != cudaSuccess || ncl < 1) {
+    cudaGetLastError();
+    set_err(h, FM_ERR_UNSUPPORTED, "no co-resident clusters of %d CTAs", kClusterSize);
+    return bail(FM_ERR_UNSUPPORTED);
+  }
+  h->n_clusters = std::min(ncl, h->n_sms / kClusterSize);
+  h->n_ctas = h->n_clusters * kClusterSize;
+  if ((st = build_plan(h)) != FM_OK) return bail(st);
+  if (cfg->wtype == FM_W_FP8_E4M3) {
+    set_err(h, FM_ERR_UNSUPPORTED, "FP8 weights are not available in this build yet");
+    return bail(FM_ERR_UNSUPPORTED);
+  }
+  if (cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
+    set_err(h, FM_ERR_CUDA, "stream creation failed");
+    return bail(FM_ERR_CUDA);
+  }
+  if ((st = pack_weights(h, w)) != FM_OK) return bail(st);
+
+  const size_t T = c.chunk_len, A = c.action_dim, d = c.d_model;
+  const size_t B = c.max_batch;
+#define ALLOC_OR_BAIL(ptr, bytes)                           \
+  do {                                                      \
+    fm_status s_ = dalloc(h, &(ptr), (bytes));              \
+    if (s_ != FM_OK) return bail(s_);                       \
+  } while (0)
+  ALLOC_OR_BAIL(h->mod, (size_t)c.max_steps * h->n_mod * 4);
+  ALLOC_OR_BAIL(h->h1_act, (size_t)kRows * d * 2);
+  ALLOC_OR_BAIL(h->rope, T * c.head_dim * 4);
+  ALLOC_OR_BAIL(h->P_dev, 4);
+  ALLOC_OR_BAIL(h->x, B * T * A * 4);
+  ALLOC_OR_BAIL(h->vbuf, B * T * A * 4);
+  ALLOC_OR_BAIL(h->h_a, T * d * 4);
+  ALLOC_OR_BAIL(h->h_b, T * d * 4);
+  ALLOC_OR_BAIL(h->z_a, (size_t)kRows * d * 2);
+  ALLOC_OR_BAIL(h->z_f, (size_t)kRows * d * 2);
+  ALLOC_OR_BAIL(h->o_act, (size_t)kRows * c.n_q_heads * c.head_dim * 2);
+  ALLOC_OR_BAIL(h->u_act, (size_t)kRows * c.d_ff * 2);
+  ALLOC_OR_BAIL(h->sumsq_a, (size_t)h->n_clusters * kRows * 4);
+  ALLOC_OR_BAIL(h->sumsq_f, (size_t)h->n_clusters * kRows * 4);
+  ALLOC_OR_BAIL(h->qbuf, (size_t)c.n_q_heads * kRows * c.head_dim * 2);
+  const size_t kv = (size_t)c.n_layers * B * c.n_kv_heads * h->S_max * c.head_dim * 2;
+  ALLOC_OR_BAIL(h->kcache, kv);
+  ALLOC_OR_BAIL(h->vcache, kv);
+  ALLOC_OR_BAIL(h->bar_count, 4);
+  ALLOC_OR_BAIL(h->err_word, 4);
+#undef ALLOC_OR_BAIL
+  if (cudaDeviceSynchronize() != cudaSuccess) {
+    set_err(h, FM_ERR_CUDA, "set-up failed: %s", cudaGetErrorString(cudaGetLastError()));
+    return bail(FM_ERR_CUDA);
+  }
+  *out = h;
+  return FM_OK;
+}
+
+fm_status fm_set_prefix(fm_expert* h, const uint16_t* const* k, const uint16_t* const* v, int batch,
+                        int prefix_len, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (batch < 1 || batch > c.max_batch)
+    return set_err(h, FM_ERR_INVALID_ARG, "batch %d outside [1, %d]", batch, c.max_batch);
+  if (prefix_len < 0 || prefix_len > c.max_prefix)
+    return set_err(h, FM_ERR_INVALID_ARG, "prefix_len %d outside [0, %d]", prefix_len, c.max_prefix);
+  if (prefix_len > 0 && (!k || !v)) return set_err(h, FM_ERR_INVALID_ARG, "k or v is NULL");
+  CK(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const size_t per = (size_t)batch * prefix_len * c.n_kv_heads * c.head_dim;
+  const size_t lay = (size_t)c.max_batch * c.n_kv_heads * h->S_max * c.head_dim;
+  void* tmp = nullptr;
+  if (prefix_len > 0) {
+    for (int l = 0; l < c.n_layers; ++l)
+      if (!k[l] || !v[l]) return set_err(h, FM_ERR_INVALID_ARG, "prefix pointer of layer %d is NULL", l);
+    CK(cudaMalloc(&tmp, per * 2 * 2));
+  }
+  fm_status out = FM_OK;
+  for (int l = 0; l < c.n_layers && prefix_len > 0; ++l) {
+    const uint16_t* srcs[2] = {k[l], v[l]};
+    uint16_t* dsts[2] = {h->kcache + l * lay, h->vcache + l * lay};
+    for (int i = 0; i < 2; ++i) {
+      const uint16_t* src = srcs[i];
+      if (!is_device_ptr(src)) {
+        uint16_t* t = static_cast<uint16_t*>(tmp) + i * per;
+        cudaError_t e = cudaMemcpyAsync(t, src, per * 2, cudaMemcpyDefault, st);
+        if (e != cudaSuccess) { out = set_err(h, FM_ERR_CUDA, "prefix upload: %s", cudaGetErrorString(e)); break; }
+        src = t;
+      }
+      cudaError_t e = launch_kv_copy(src, batch, prefix_len, c.n_kv_heads, c.head_dim, h->S_max, dsts[i], st);
+      if (e != cudaSuccess) { out = set_err(h, FM_ERR_CUDA, "kv copy: %s", cudaGetErrorString(e)); break; }
+    }
+    if (out != FM_OK) break;
+    if (tmp) {
+      // the staging buffer is reused by the next layer
+      cudaError_t e = cudaStreamSynchronize(st);
+      if (e != cudaSuccess) { out = set_err(h, FM_ERR_CUDA, "prefix sync: %s", cudaGetErrorString(e)); break; }
+    }
+  }
+  if (tmp) cudaFree(tmp);
+  if (out != FM_OK) return out;
+  CK(cudaMemcpyAsync(h->P_dev, &prefix_len, 4, cudaMemcpyHostToDevice, st));
+  CK(launch_rope_table(c.chunk_len, c.head_dim, prefix_len, (double)c.rope_base, h->rope, st));
+  CK(cudaStreamSynchronize(st));
+  h->prefix_batch = batch;
+  h->prefix_len = prefix_len;
+  return FM_OK;
+}
+
+static fm_status get_graph(fm_expert* h, int batch, int steps, cudaGraphExec_t* out) {
+  auto key = std::make_pair(batch, steps);
+  auto it = h->graphs.find(key);
+  if (it != h->graphs.end()) {
+    *out = it->second;
+    return FM_OK;
+  }
+  cudaGraph_t g = nullptr;
+  CK(cudaStreamBeginCapture(h->cap_stream, cudaStreamCaptureModeThreadLocal));
+  cudaError_t e = enqueue_denoise(h, batch, steps, h->cap_stream);
+  cudaError_t e2 = cudaStreamEndCapture(h->cap_stream, &g);
+  if (e != cudaSuccess || e2 != cudaSuccess) {
+    if (g) cudaGraphDestroy(g);
+    return set_err(h, FM_ERR_CUDA, "graph capture: %s / %s", cudaGetErrorString(e), cudaGetErrorString(e2));
+  }
+  cudaGraphExec_t ex = nullptr;
+  e = cudaGraphInstantiate(&ex, g, 0);
+  if (e != cudaSuccess) {
+    cudaGraphDestroy(g);
+    return set_err(h, FM_ERR_CUDA, "graph instantiate: %s", cudaGetErrorString(e));
+  }
+  h->graphs[key] = ex;
+  h->graph_defs[key] = g;
+  *out = ex;
+  return FM_OK;
+}
+
+fm_status fm_denoise(fm_expert* h, const float* x0, int batch, int steps, float* out, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (!x0 || !out) return set_err(h, FM_ERR_INVALID_ARG, "x0 or out is NULL");
+  if (steps < 1 || steps > c.max_steps)
+    return set_err(h, FM_ERR_INVALID_ARG, "steps %d outside [1, %d]", steps, c.max_steps);
+  if (batch < 1 || batch > c.max_batch)
+    return set_err(h, FM_ERR_INVALID_ARG, "batch %d outside [1, %d]", batch, c.max_batch);
+  if (h->prefix_batch != batch)
+    return set_err(h, FM_ERR_NOT_READY, "fm_set_prefix was not called for batch %d", batch);
+  CK(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaGraphExec_t ex = nullptr;
+  fm_status s = get_graph(h, batch, steps, &ex);
+  if (s != FM_OK) return s;
+  const size_t bytes = (size_t)batch * c.chunk_len * c.action_dim * 4;
+  const bool host_out = !is_device_ptr(out);
+  CK(cudaMemcpyAsync(h->x, x0, bytes, cudaMemcpyDefault, st));
+  CK(cudaGraphLaunch(ex, st));
+  CK(cudaMemcpyAsync(out, h->x, bytes, cudaMemcpyDefault, st));
+  if (host_out) {
+    CK(cudaStreamSynchronize(st));
+    return check_err_word(h);
+  }
+  return FM_OK;
+}
+
+fm_status fm_time_modulation(fm_expert* h, int steps, float* m_out, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  if (!m_out) return set_err(h, FM_ERR_INVALID_ARG, "m_out is NULL");
+  if (steps < 1 || steps > h->cfg.max_steps)
+    return set_err(h, FM_ERR_INVALID_ARG, "steps %d outside [1, %d]", steps, h->cfg.max_steps);
+  CK(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  CK(launch_time(time_params(h, steps), h->n_sms, st));
+  CK(cudaMemcpyAsync(m_out, h->mod, (size_t)steps * h->n_mod * 4, cudaMemcpyDefault, st));
+  CK(cudaStreamSynchronize(st));
+  return check_err_word(h);
+}
+
+static fm_status velocity_common(fm_expert* h, const float* x, int batch, int step_index, int steps,
+                                 cudaStream_t st) {
+  const fm_config& c = h->cfg;
+  if (!x) return set_err(h, FM_ERR_INVALID_ARG, "x is NULL");
+  if (steps < 1 || steps > c.max_steps || step_index < 0 || step_index >= steps)
+    return set_err(h, FM_ERR_INVALID_ARG, "step_index %d / steps %d invalid", step_index, steps);
+  if (batch < 1 || batch > c.max_batch)
+    return set_err(h, FM_ERR_INVALID_ARG, "batch %d outside [1, %d]", batch, c.max_batch);
+  if (h->prefix_batch != batch)
+    return set_err(h, FM_ERR_NOT_READY, "fm_set_prefix was not called for batch %d", batch);
+  CK(cudaSetDevice(h->device));
+  CK(cudaMemcpyAsync(h->x, x, (size_t)batch * c.chunk_len * c.action_dim * 4, cudaMemcpyDefault, st));
+  CK(launch_time(time_params(h, steps), h->n_sms, st));
+  return FM_OK;
+}
+
+fm_status fm_velocity(fm_expert* h, const float* x, int batch, int step_index, int steps, float* v_out,
+                      void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  if (!v_out) return set_err(h, FM_ERR_INVALID_ARG, "v_out is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  fm_status s = velocity_common(h, x, batch, step_index, steps, st);
+  if (s != FM_OK) return s;
+  const fm_config& c = h->cfg;
+  const size_t xs = (size_t)c.chunk_len * c.action_dim;
+  for (int b = 0; b < batch; ++b) {
+    StepParams p = base_params(h);
+    p.b = b;
+    p.x = h->x + b * xs;
+    p.vbuf = h->vbuf + b * xs;
+    p.step0 = step_index;
+    p.step1 = step_index + 1;
+    p.update_x = 0;
+    CK(cudaMemsetAsync(h->bar_count, 0, 4, st));
+    CK(launch_step(p, st));
+  }
+  CK(cudaMemcpyAsync(v_out, h->vbuf, (size_t)batch * xs * 4, cudaMemcpyDefault, st));
+  if (!is_device_ptr(v_out)) {
+    CK(cudaStreamSynchronize(st));
+    return check_err_word(h);
+  }
+  return FM_OK;
+}
+
+size_t fm_trace_bytes(const fm_expert* h) {
+  if (!h) return 0;
+  const fm_config& c = h->cfg;
+  const size_t T = c.chunk_len, d = c.d_model, qn = (size_t)c.n_q_heads * c.head_dim,
+               kn = (size_t)c.n_kv_heads * c.head_dim;
+  const size_t per = T * (d + qn + kn + kn + qn + d + c.d_ff + d);
+  return 4 * (c.n_layers * per + T * c.action_dim);
+}
+
+namespace {
+float bf2f(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  std::memcpy(&f, &u, 4);
+  return f;
+}
+// Reads element (r, col) of a host copy of an ACT64 matrix.
+float act64_get(const std::vector<uint16_t>& a, int r, int col) {
+  const size_t idx = (size_t)(col >> 6) * (kRows * 64) + (size_t)r * 64 +
+                     ((((col & 63) >> 3) ^ (r & 7)) << 3) + (col & 7);
+  return bf2f(a[idx]);
+}
+float swz_get(const std::vector<uint16_t>& a, size_t row_base, int row, int e) {
+  return bf2f(a[row_base + ((((e >> 3) ^ (row & 7))) << 3) + (e & 7)]);
+}
+}  // namespace
+
+fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int steps, float* trace,
+                            void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  if (!trace) return set_err(h, FM_ERR_INVALID_ARG, "trace is NULL");
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  fm_status s = velocity_common(h, x, 1, step_index, steps, st);
+  if (s != FM_OK) return s;
+  const fm_config& c = h->cfg;
+  const int T = c.chunk_len, d = c.d_model, qn = c.n_q_heads * c.head_dim,
+            kn = c.n_kv_heads * c.head_dim, F = c.d_ff, hd = c.head_dim;
+  float* out = trace;
+  std::vector<float> hbuf((size_t)T * d);
+  std::vector<uint16_t> qh((size_t)c.n_q_heads * kRows * hd), oh((size_t)kRows * qn),
+      uh((size_t)kRows * F), kvh((size_t)h->S_max * hd);
+  const size_t lay = (size_t)c.max_batch * c.n_kv_heads * h->S_max * hd;
+  auto run = [&](int layer0, int layer1, int inproj, int outproj) -> fm_status {
+    StepParams p = base_params(h);
+    p.step0 = step_index;
+    p.step1 = step_index + 1;
+    p.layer0 = layer0;
+    p.layer1 = layer1;
+    p.do_inproj = inproj;
+    p.do_outproj = outproj;
+    p.update_x = 0;
+    CK(cudaMemsetAsync(h->bar_count, 0, 4, st));
+    CK(launch_step(p, st));
+    CK(cudaStreamSynchronize(st));
+    return check_err_word(h);
+  };
+  // in-proj only (layer range empty)
+  if ((s = run(0, 0, 1, 0)) != FM_OK) return s;
+  for (int l = 0; l < c.n_layers; ++l) {
+    CK(cudaMemcpy(out, h->h_a, (size_t)T * d * 4, cudaMemcpyDeviceToHost));   // h_in
+    out += (size_t)T * d;
+    if ((s = run(l, l + 1, 0, 0)) != FM_OK) return s;
+    CK(cudaMemcpy(qh.data(), h->qbuf, qh.size() * 2, cudaMemcpyDeviceToHost));
+    for (int t = 0; t < T; ++t)
+      for (int n = 0; n < qn; ++n) {
+        const int head = n / hd, e = n % hd;
+        out[(size_t)t * qn + n] = swz_get(qh, ((size_t)head * kRows + t) * hd, t, e);
+      }
+    out += (size_t)T * qn;
+    for (int which = 0; which < 2; ++which) {
+      const uint16_t* cache = (which == 0 ? h->kcache : h->vcache) + l * lay;
+      for (int g = 0; g < c.n_kv_heads; ++g) {
+        CK(cudaMemcpy(kvh.data(), cache + (size_t)g * h->S_max * hd, kvh.size() * 2, cudaMemcpyDeviceToHost));
+        for (int t = 0; t < T; ++t)
+          for (int e = 0; e < hd; ++e) {
+            const int row = h->prefix_len + t;
+            out[(size_t)t * kn + g * hd + e] = swz_get(kvh, (size_t)row * hd, row, e);
+          }
+      }
+      out += (size_t)T * kn;
+    }
+    CK(cudaMemcpy(oh.data(), h->o_act, oh.size() * 2, cudaMemcpyDeviceToHost));
+    for (int t = 0; t < T; ++t)
+      for (int n = 0; n < qn; ++n) out[(size_t)t * qn + n] = act64_get(oh, t, n);
+    out += (size_t)T * qn;
+    CK(cudaMemcpy(out, h->h_b, (size_t)T * d * 4, cudaMemcpyDeviceToHost));   // h_mid
+    out += (size_t)T * d;
+    CK(cudaMemcpy(uh.data(), h->u_act, uh.size() * 2, cudaMemcpyDeviceToHost));
+    for (int t = 0; t < T; ++t)
+      for (int n = 0; n < F; ++n) out[(size_t)t * F + n] = act64_get(uh, t, n);
+    out += (size_t)T * F;
+    CK(cudaMemcpy(out, h->h_a, (size_t)T * d * 4, cudaMemcpyDeviceToHost));   // h_out
+    out += (size_t)T * d;
+  }
+  if ((s = run(c.n_layers, c.n_layers, 0, 1)) != FM_OK) return s;
+  CK(cudaMemcpy(out, h->vbuf, (size_t)T * c.action_dim * 4, cudaMemcpyDeviceToHost));
+  return FM_OK;
+}
+
+fm_status fm_get_fp8_weights(fm_expert* h, int layer, int which, uint8_t* codes, float* scale) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  if (h->cfg.wtype != FM_W_FP8_E4M3) return set_err(h, FM_ERR_INVALID_ARG, "handle holds bf16 weights");
+  (void)layer; (void)which; (void)codes; (void)scale;
+  return set_err(h, FM_ERR_UNSUPPORTED, "not available");
+}
+
+fm_status fm_sync(fm_expert* h, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  CK(cudaSetDevice(h->device));
+  CK(cudaStreamSynchronize(static_cast<cudaStream_t>(stream)));
+  return check_err_word(h);
+}
+
+fm_status fm_get_geometry(const fm_expert* h, int* cluster_size, int* n_clusters, int* n_ctas) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  if (cluster_size) *cluster_size = kClusterSize;
+  if (n_clusters) *n_clusters = h->n_clusters;
+  if (n_ctas) *n_ctas = h->n_ctas;
+  return FM_OK;
+}
+
+size_t fm_expert_destroy(fm_expert* h) {
+  if (!h) return 0;
+  cudaSetDevice(h->device);
+  cudaDeviceSynchronize();
+  const size_t n = h->bytes;
+  free_all(h);
+  delete h;
+  return n;
+}
+
+#pragma GCC visibility pop
+}  // extern "C"

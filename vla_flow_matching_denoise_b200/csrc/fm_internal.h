@@ -1,0 +1,117 @@
+// Internal structures shared by the host engine (fm_api.cu) and the kernels.
+//
+// Data layouts (device memory):
+//  * "ACT64": a bf16 activation matrix of 64 rows (rows >= valid tokens are
+//    padding) and K columns, stored as K/64 blocks of 8 KB.  Block kb holds
+//    columns [64 kb, 64 kb + 64) as 64 rows of 128 bytes; the 16-byte piece c
+//    of row r sits at piece (c ^ (r & 7)).  This is the 128-byte-swizzled,
+//    K-major image the tensor cores read, so one bulk copy moves a block from
+//    global to shared memory ready for tcgen05.mma.
+//  * Packed weights: the same image with rows = output channels: a "chunk" is
+//    R rows x 64 input columns (R * 128 bytes).  The engine lays every CTA's
+//    chunks of one layer out contiguously, in the order the CTA consumes them.
+//  * KV cache: [L][B][H_kv][S_max][hd] bf16, each 256-byte row (hd = 128)
+//    split in 16-byte pieces stored at piece (c ^ (row & 7)); rows 0..P-1 are
+//    the prefix, rows P..P+T-1 the chunk of the current velocity evaluation.
+//  * q buffer: [H_q][64][hd] bf16, same per-row piece swizzle.
+#pragma once
+#include <cstdint>
+
+namespace fm {
+
+constexpr int kClusterSize = 8;        // CTAs per cluster (portable maximum)
+constexpr int kComputeWarps = 4;       // warps 2..5
+constexpr int kThreads = 192;          // producer warp, MMA warp, 4 compute warps
+constexpr int kRows = 64;              // MMA M: token rows per tile
+constexpr int kMaxT = 50;              // valid token rows (one chunk)
+constexpr int kBiasRow = 50;           // row carrying the AdaRMSNorm shift vector
+constexpr int kTimeDim = 256;
+constexpr int kRingSlots = 16;         // mbarrier pairs of the weight ring
+constexpr int kWorkBytes = 64 * 1024;  // activation / staging region
+constexpr int kSmemMax = 232448;       // dynamic shared memory per CTA (227 KB)
+
+enum GemmId { G_QKV = 0, G_O = 1, G_GU = 2, G_DOWN = 3 };
+
+// One GEMM of a layer, partitioned over clusters: cluster c owns Nc packed
+// output channels; inside it CTA j works on n-group j / KS (Ng channels) and
+// K-slice j % KS (kslice columns); after the in-cluster reduction CTA j owns
+// `own` output columns of its n-group.
+struct GemmPlan {
+  int N;          // logical output channels
+  int K;          // reduction length
+  int NS, KS;     // n-groups and K-slices per cluster (NS * KS = 8)
+  int Ng;         // packed channels per n-group (MMA N, multiple of 8, <= 256)
+  int own;        // columns owned per CTA after the reduction
+  int kslice;     // K per slice (multiple of 64)
+  int busy_clusters;  // clusters with at least one channel
+  uint32_t chunk_bytes;  // Ng * 128
+  int nchunk;     // kslice / 64
+};
+
+struct StepParams {
+  int L, d, Hq, Hkv, hd, F, A, T, S_max;
+  int B_cap;                 // request slots in the KV cache
+  int b;                     // request handled by this launch
+  const int* P_dev;          // prefix length, read on the device (no recapture on change)
+  float eps;
+  int n_clusters, n_ctas;
+  GemmPlan g[4];
+  int uc;            // u columns per n-group (gate/up pairs)
+  // weights
+  const uint8_t* arena;      // packed per-layer weights
+  uint64_t layer_bytes;      // bytes of one layer in the arena
+  const uint32_t* span_off;  // [n_ctas + 1]: byte offset of each CTA's span in a layer
+  const uint16_t* w_in;      // [d, A] bf16
+  const uint16_t* w_out;     // [A, d] bf16
+  const float* out_bias;     // [A] or null
+  // per-call tables
+  const float* mod;          // [steps][n_mod] fp32 modulation rows
+  int n_mod;
+  const float* rope;         // [T][hd/2][2] cos, sin for positions P .. P+T-1
+  // buffers
+  float* x;                  // [T, A]
+  float* vbuf;               // [T, A]
+  float* h_a;                // [T, d]
+  float* h_b;                // [T, d]
+  uint16_t* z_a;             // ACT64 [64, d]: h (1 + s_a), row 50 = b_a
+  uint16_t* z_f;             // ACT64 [64, d]: h (1 + s_f), row 50 = b_f
+  uint16_t* o_act;           // ACT64 [64, H_q hd]
+  uint16_t* u_act;           // ACT64 [64, F]
+  float* sumsq_a;            // [n_clusters][64] per-cluster row sums of h^2
+  float* sumsq_f;
+  uint16_t* qbuf;            // [H_q][64][hd]
+  uint16_t* kcache;          // [L][B][H_kv][S_max][hd]
+  uint16_t* vcache;
+  uint32_t* bar_count;       // grid barrier counter (zeroed before launch)
+  uint32_t* err;             // error word (non-zero: a bounded wait gave up)
+  // schedule of this launch
+  int step0, step1;          // modulation rows used
+  int layer0, layer1;        // layers run per step
+  int do_inproj, do_outproj, update_x;
+  float dt;
+  long long spin_budget;     // cycles before a wait gives up
+};
+
+struct TimeParams {
+  int n_steps, d, n_mod;
+  const uint16_t* w1;        // [d, 256] bf16
+  const uint8_t* w2_packed;  // chunks of 128 rows x 64 cols, [n_mod/128][d/64]
+  uint16_t* h1_act;          // ACT64 [64, d]
+  float* mod;                // [n_steps][n_mod]
+  uint32_t* err;
+  long long spin_budget;
+};
+
+// One packing job: copy `nrows` source rows (row indices from `rowidx`, -1 =
+// zero row) x 64 columns starting at column 64*kb into the swizzled image at
+// byte offset dst_off.
+struct PackChunk {
+  uint64_t dst_off;
+  uint32_t rowidx_off;
+  uint16_t nrows;
+  uint8_t mat;
+  uint8_t fp8;
+  uint32_t kb;
+};
+
+}  // namespace fm

@@ -1,0 +1,28 @@
+// Host-side launch wrappers of the kernels (internal to the library).
+#pragma once
+#include <cuda_runtime.h>
+#include <cstddef>
+#include <cstdint>
+
+#include "fm_internal.h"
+
+namespace fm {
+
+cudaError_t launch_pack(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
+                        const uint16_t* const* mats, const int* mat_k, uint8_t* dst,
+                        cudaStream_t st);
+cudaError_t launch_fp8_quantize(const uint16_t* w, int rows, int K, float* scale, uint8_t* q,
+                                cudaStream_t st);
+cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, int Hkv, int hd, int S_max,
+                           uint16_t* cache, cudaStream_t st);
+cudaError_t launch_rope_table(int T, int hd, int P, double base, float* tab, cudaStream_t st);
+
+size_t time_gemm_smem_bytes(int d);
+cudaError_t launch_time(const TimeParams& p, int n_sms, cudaStream_t st);
+
+// Latency-mode denoise megakernel (one request, persistent, clusters of 8).
+size_t step_smem_bytes();
+cudaError_t step_max_clusters(int* n_clusters);
+cudaError_t launch_step(const StepParams& p, cudaStream_t st);
+
+}  // namespace fm

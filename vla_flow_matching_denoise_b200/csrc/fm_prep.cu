@@ -1,0 +1,119 @@
+// Set-up kernels (run at fm_expert_create / fm_set_prefix, not in the loop):
+//  * weight packing into the swizzled, per-CTA-ordered arena (bf16 or E4M3);
+//  * per-row absmax scales and E4M3 quantisation of the per-layer linears;
+//  * prefix K/V copy into the swizzled KV cache;
+//  * the RoPE cos/sin table for the chunk positions P .. P+T-1.
+#include <cuda_bf16.h>
+#include <cuda_fp8.h>
+#include <cstdint>
+
+#include "fm_internal.h"
+#include "fm_launch.h"
+
+namespace fm {
+
+// Copies 16-byte pieces of source rows into the swizzled chunk image.
+__global__ void pack_kernel(const PackChunk* __restrict__ chunks, const int32_t* __restrict__ rowidx,
+                            const uint16_t* const* __restrict__ mats, const int* __restrict__ mat_k,
+                            uint8_t* __restrict__ dst) {
+  const PackChunk ch = chunks[blockIdx.x];
+  const uint16_t* src = mats[ch.mat];
+  const int K = mat_k[ch.mat];
+  const int pieces = ch.nrows * 8;
+  for (int p = threadIdx.x; p < pieces; p += blockDim.x) {
+    const int row = p >> 3, c = p & 7;
+    const int sr = rowidx[ch.rowidx_off + row];
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (sr >= 0) v = *reinterpret_cast<const uint4*>(src + (size_t)sr * K + (size_t)ch.kb * 64 + c * 8);
+    *reinterpret_cast<uint4*>(dst + ch.dst_off + (size_t)row * 128 + ((c ^ (row & 7)) << 4)) = v;
+  }
+}
+
+// Per-row absmax / 448 of a bf16 matrix [rows, K] (R8: s = absmax / 448, 1 for
+// an all-zero row).  One warp per row.
+__global__ void fp8_row_scale_kernel(const uint16_t* __restrict__ w, int rows, int K,
+                                     float* __restrict__ scale) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (warp >= rows) return;
+  float m = 0.f;
+  for (int k = lane; k < K; k += 32) {
+    const float x = __uint_as_float((uint32_t)w[(size_t)warp * K + k] << 16);
+    m = fmaxf(m, fabsf(x));
+  }
+  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+  if (lane == 0) scale[warp] = m > 0.f ? __fdiv_rn(m, 448.0f) : 1.0f;
+}
+
+// E4M3 codes of w / s (true fp32 division, nearest-even, saturating finite).
+__global__ void fp8_quantize_kernel(const uint16_t* __restrict__ w, const float* __restrict__ scale,
+                                    int rows, int K, uint8_t* __restrict__ q) {
+  const size_t n = (size_t)rows * K;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const float x = __uint_as_float((uint32_t)w[i] << 16);
+    const float r = __fdiv_rn(x, scale[i / K]);
+    q[i] = (uint8_t)__nv_cvt_float_to_fp8(r, __NV_SATFINITE, __NV_E4M3);
+  }
+}
+
+// Prefix K or V of one layer: src [B, P, H_kv, hd] -> cache [B_cap][H_kv][S_max][hd]
+// with 16-byte pieces swizzled by (row & 7).
+__global__ void kv_copy_kernel(const uint16_t* __restrict__ src, int B, int P, int Hkv, int hd,
+                               int S_max, uint16_t* __restrict__ cache) {
+  const int pieces = hd / 8;
+  const size_t total = (size_t)B * P * Hkv * pieces;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
+       i += (size_t)gridDim.x * blockDim.x) {
+    const int c = (int)(i % pieces);
+    size_t r = i / pieces;
+    const int g = (int)(r % Hkv); r /= Hkv;
+    const int s = (int)(r % P);
+    const int b = (int)(r / P);
+    const uint4 v = *reinterpret_cast<const uint4*>(src + (((size_t)b * P + s) * Hkv + g) * hd + c * 8);
+    uint16_t* row = cache + (((size_t)b * Hkv + g) * S_max + s) * hd;
+    *reinterpret_cast<uint4*>(row + ((c ^ (s & 7)) << 3)) = v;
+  }
+}
+
+// cos / sin of pos * base^(-2i/hd) for pos = P + t, in double, stored fp32.
+__global__ void rope_table_kernel(int T, int hd, int P, double base, float* __restrict__ tab) {
+  const int half = hd / 2;
+  const int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= T * half) return;
+  const int t = i / half, j = i % half;
+  const double theta = pow(base, -2.0 * j / hd);
+  const double ang = (double)(P + t) * theta;
+  tab[2 * i] = (float)cos(ang);
+  tab[2 * i + 1] = (float)sin(ang);
+}
+
+cudaError_t launch_pack(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
+                        const uint16_t* const* mats, const int* mat_k, uint8_t* dst,
+                        cudaStream_t st) {
+  if (nchunks == 0) return cudaSuccess;
+  pack_kernel<<<nchunks, 256, 0, st>>>(chunks, rowidx, mats, mat_k, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_quantize(const uint16_t* w, int rows, int K, float* scale, uint8_t* q,
+                                cudaStream_t st) {
+  fp8_row_scale_kernel<<<(rows * 32 + 255) / 256, 256, 0, st>>>(w, rows, K, scale);
+  fp8_quantize_kernel<<<1024, 256, 0, st>>>(w, scale, rows, K, q);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, int Hkv, int hd, int S_max,
+                           uint16_t* cache, cudaStream_t st) {
+  if ((size_t)B * P == 0) return cudaSuccess;
+  kv_copy_kernel<<<512, 256, 0, st>>>(src, B, P, Hkv, hd, S_max, cache);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(int T, int hd, int P, double base, float* tab, cudaStream_t st) {
+  const int n = T * hd / 2;
+  rope_table_kernel<<<(n + 127) / 128, 128, 0, st>>>(T, hd, P, base, tab);
+  return cudaGetLastError();
+}
+
+}  // namespace fm
