@@ -1,0 +1,352 @@
+"""Benchmark of the denoise loop on B200: one JSON line on rank 0.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl reference]
+
+A "step" of this benchmark is one full denoise call: the time MLP once, then
+`euler_steps` Euler steps of the 36-layer expert over one 50 x 75 chunk per
+request (the workload of "LingBot-VLA on Thor (sm_110)", §1 and §5: chunk
+[1, 50, 75], 10 denoise steps, CUDA-graph replay).  Weights are synthetic
+N(0, 0.02) bf16 (no checkpoint is available), prefix K/V N(0, 1), x0 N(0, 1).
+
+value      = Euler steps per second over the whole job (all ranks), device
+             timed with CUDA events, inputs resident in HBM.
+e2e        = the same metric through fm_denoise with pinned host buffers, the
+             host->device copy of x0 and the device->host copy of the result
+             inside the timed region.
+roofline   = the denoise-loop kernel: algorithmic bytes (weights + prefix/chunk
+             KV per Euler step) / its event-timed duration, against the
+             measured HBM copy bandwidth.
+The one-request path does not shard: with N GPUs every rank runs its own
+replica (weak scaling, no collective on the data path).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from vla_flow_matching_denoise_b200 import synth  # noqa: E402
+
+METRIC = "ms per 10-step 50x75 chunk & denoise steps/s (B=1); % HBM roofline"
+UNIT = "denoise steps/s"
+
+# DRAM bytes of one launch of the loop kernel from an ncu capture, keyed by
+# workload, with the hash of the kernel sources it was taken on; reported as
+# null when the sources changed since.
+NCU_TRAFFIC = {}
+
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for f in ("fm_step.cu", "fm_ptx.cuh", "fm_internal.h"):
+        with open(os.path.join(ROOT, "vla_flow_matching_denoise_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), float(d["bf16_tflops"]), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def loop_bytes(shape: synth.ExpertShape, steps: int, batch: int) -> float:
+    """Algorithmic bytes of the denoise-loop kernel for one call.
+
+    Per Euler step: every per-layer weight once (bf16, or E4M3 plus one fp32
+    scale per row), the in/out projections, and per request the prefix K/V and
+    the chunk K/V of every layer read once."""
+    s = shape
+    ws = s.weight_shapes()
+    per_layer = sum(int(np.prod(ws[k])) for k in synth.LAYER_KEYS)
+    rows = sum(ws[k][0] for k in synth.LAYER_KEYS)
+    wbytes = s.n_layers * (per_layer * (1.0 if s.fp8 else 2.0) + (rows * 4.0 if s.fp8 else 0.0))
+    io = (int(np.prod(ws["in_proj"])) + int(np.prod(ws["out_proj"]))) * 2.0
+    kv = batch * s.n_layers * 2 * (s.prefix_len + s.chunk_len) * s.n_kv_heads * s.head_dim * 2.0
+    return steps * (wbytes + io + kv)
+
+
+def time_mlp_bytes(shape: synth.ExpertShape) -> float:
+    ws = shape.weight_shapes()
+    return (int(np.prod(ws["time_w1"])) + int(np.prod(ws["time_w2"]))) * 2.0
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    mx = float(parts[2])
+                except ValueError:
+                    continue
+                for n, v in zip(names, parts[5:9]):
+                    if v.lower().startswith("active"):
+                        reasons.add(n)
+        os.unlink(self.path)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+class OracleRunner:
+    """The oracle as it stands, on request 0 of the same workload."""
+
+    def __init__(self, shape: synth.ExpertShape, seed: int = 0):
+        from oracle import fm_oracle as O
+        self.O = O
+        self.shape = shape
+        raw = synth.make_weights(shape, seed)
+        kp, vp = synth.make_prefix(shape, seed, batch=1)
+        self.x0 = synth.make_x0(shape, seed, batch=1)[0]
+        self.W = O.Weights(raw, fp8=shape.fp8)
+        self.kp = [O.decode_bf16(k[0]) for k in kp]
+        self.vp = [O.decode_bf16(v[0]) for v in vp]
+        try:
+            from threadpoolctl import threadpool_info
+            self.cores = max([i.get("num_threads", 1) for i in threadpool_info()] or [os.cpu_count()])
+        except Exception:
+            self.cores = os.cpu_count()
+
+    def run(self, n_sample: int) -> float:
+        """Seconds for `n_sample` Euler steps (whole chunks repeat from x0), each
+        chunk with its own time MLP."""
+        O, s = self.O, self.shape
+        t0 = time.perf_counter()
+        done = 0
+        while done < n_sample:
+            ts, dt = O.time_schedule(s.steps)
+            M = O.time_modulation(ts, self.W.time_w1, self.W.time_w2)
+            x = self.x0.astype(np.float64)
+            for k in range(min(s.steps, n_sample - done)):
+                v = O.expert_velocity(x, M[k], self.W, self.kp, self.vp, s.rms_eps, s.rope_base, s.n_q_heads,
+                                      s.n_kv_heads)
+                x = x + dt * v
+                done += 1
+        return time.perf_counter() - t0
+
+    def sample_text(self, n_sample: int, el: float) -> str:
+        return (f"{n_sample} Euler steps of request 0 ({self.shape.steps}-step chunks, time MLP per chunk), "
+                f"fp64 numpy, {el:.1f} s")
+
+
+def cpu_baseline(shape: synth.ExpertShape, n_sample: int, seed: int = 0):
+    r = OracleRunner(shape, seed)
+    el = r.run(n_sample)
+    return {"value": n_sample / el, "unit": UNIT, "cores": r.cores, "kind": "oracle",
+            "sample": r.sample_text(n_sample, el)}
+
+
+def dist_setup(gpus: int):
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    pg = None
+    if ws > 1:
+        import torch.distributed as dist
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        pg = dist
+    return ws, rank, local, pg
+
+
+def run_reference(args, shape):
+    # Rank 0 alone times the oracle; other ranks exit without work.
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    n_sample = 1
+    runner = OracleRunner(shape)
+    vals, el = [], 0.0
+    for i in range(args.warmup + args.steps):
+        el = runner.run(n_sample)
+        if i >= args.warmup:
+            vals.append(n_sample / el)
+    r = {"cores": runner.cores, "sample": runner.sample_text(n_sample, el)}
+    v = statistics.mean(vals)
+    line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / v,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": args.workload},
+            "cpu_baseline": {"value": v, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
+                             "sample": r["sample"]},
+            "e2e": {"value": v, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="lingbot_p256_n10", choices=sorted(synth.WORKLOADS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-sample-steps", type=int, default=30)
+    ap.add_argument("--once", action="store_true",
+                    help="one fm_velocity call of the workload and exit (profiling driver)")
+    args = ap.parse_args()
+    shape = synth.WORKLOADS[args.workload]
+    if args.impl == "reference":
+        run_reference(args, shape)
+        return
+
+    import torch
+    ws, rank, local, pg = dist_setup(args.gpus)
+    torch.cuda.set_device(local)
+    from vla_flow_matching_denoise_b200.binding import Expert
+
+    B, n = shape.batch, shape.steps
+    raw = synth.make_weights(shape, seed=0)
+    kp, vp = synth.make_prefix(shape, seed=rank)
+    x0 = synth.make_x0(shape, seed=rank)
+    e = Expert(shape, raw, device=local)
+    del raw
+    e.set_prefix(kp, vp, B, shape.prefix_len)
+    if args.once:
+        v = e.velocity(x0, 0, n)
+        torch.cuda.synchronize()
+        print(json.dumps({"once": args.workload, "mean_abs_v": float(np.abs(v).mean())}), flush=True)
+        e.close()
+        return
+    x_dev = torch.from_numpy(x0).cuda()
+    out_dev = torch.empty_like(x_dev)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if pg is not None:
+            pg.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(max(args.warmup, 3)):
+        e.denoise(x_dev, n, out=out_dev)
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clk:
+        barrier()
+        ev0.record(stream)
+        for _ in range(args.steps):
+            e.denoise(x_dev, n, out=out_dev)
+        ev1.record(stream)
+        barrier()
+    ms_total = ev0.elapsed_time(ev1)
+    if pg is not None:
+        t = torch.tensor([ms_total], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_total = float(t.item())
+    ms_call = ms_total / args.steps
+    euler_total = ws * B * n * args.steps
+    value = euler_total / (ms_total / 1000.0)
+
+    # end to end through the public API with pinned host buffers
+    xh = torch.from_numpy(x0).pin_memory()
+    oh = torch.empty_like(xh).pin_memory()
+    for _ in range(2):
+        e.denoise(xh, n, out=oh)
+    barrier()
+    ev0.record(stream)
+    for _ in range(args.steps):
+        e.denoise(xh, n, out=oh)
+    ev1.record(stream)
+    barrier()
+    ms_e2e = ev0.elapsed_time(ev1)
+    if pg is not None:
+        t = torch.tensor([ms_e2e], device="cuda")
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms_e2e = float(t.item())
+    e2e_value = euler_total / (ms_e2e / 1000.0)
+
+    # the loop kernel alone (event-timed, outside the graph)
+    ms_time_mlp, ms_loop = e.profile(B, n, max(3, min(args.steps, 10)))
+    hbm, tflops, peak_kind = measured_peaks()
+    lb = loop_bytes(shape, n, B)
+    achieved = lb / (ms_loop / 1000.0) / 1e9
+    traffic = None
+    rec = NCU_TRAFFIC.get(args.workload)
+    if rec and rec.get("source_hash") == kernel_source_hash():
+        traffic = rec["dram_bytes"]
+    e.close()
+
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_call, "ms_per_chunk": ms_call,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": args.workload, "layers": shape.n_layers, "d_model": shape.d_model,
+                   "heads": f"{shape.n_q_heads}q/{shape.n_kv_heads}kv x {shape.head_dim}",
+                   "d_ff": shape.d_ff, "prefix_len": shape.prefix_len,
+                   "chunk": f"{shape.chunk_len}x{shape.action_dim}", "euler_steps": n,
+                   "requests_per_gpu": B, "weights": "fp8-e4m3" if shape.fp8 else "bf16",
+                   "parallelism": f"replicas x{ws}",
+                   "l2": "inputs larger than L2: 1.25 GB of weights stream per Euler step (L2 126 MB)"},
+        "clocks": clk.summary(),
+        "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_chunk": ms_e2e / args.steps,
+                "h2d_bytes_per_step": int(x0.nbytes), "d2h_bytes_per_step": int(x0.nbytes)},
+        "gpu_launches": 3 * args.steps,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
+                     "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,
+                     "kernel": "step_kernel", "bytes_per_launch": lb, "ms_per_launch": ms_loop,
+                     "frac_of_8TBs": achieved / 8000.0},
+        "time_mlp_ms": ms_time_mlp,
+        "time_mlp_gbs": time_mlp_bytes(shape) / (ms_time_mlp / 1000.0) / 1e9,
+    }
+    if ws == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(shape, args.cpu_sample_steps)
+    print(json.dumps(line), flush=True)
+    if pg is not None:
+        pg.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -179,6 +179,28 @@ fm_status fm_trace_velocity(fm_expert *h, const float *x, int step_index, int st
 fm_status fm_get_fp8_weights(fm_expert *h, int layer, int which, uint8_t *codes,
                              float *scale);
 
+/* Profiling hook: runs `iters` times the two kernels of one denoise (the
+ * time MLP, then the denoise loop for every request) outside any graph, with
+ * CUDA events on `stream` around each, and writes their mean durations in
+ * milliseconds to ms[0] (time MLP) and ms[1] (loop).  Advances the handle's
+ * internal chunk state; synchronises `stream`. */
+fm_status fm_profile_denoise(fm_expert *h, int batch, int steps, int iters, float *ms,
+                             void *stream);
+
+/* Profiling hook: one denoise of request 0 (`steps` Euler steps, outside any
+ * graph) that records %globaltimer (ns) on every CTA.  With out == NULL,
+ * writes the required number of uint64 values to *n and returns.  Otherwise
+ * fills host `out` [n_ctas][stride], stride = 16*n_phases + 2*n_gemms +
+ * 2*n_chunks: per grid-barrier-separated phase 16 marks (start, MMAs or
+ * attention done, partials pushed, partials received, epilogue done,
+ * barrier arrival issued, partials staged, staging synchronised, then
+ * phase-specific points); per linear the MMA warp's marks
+ * (activations landed, last weight chunk landed); per weight chunk the time
+ * it landed, then per weight chunk the time the producer issued it.  Unused
+ * slots are 0.  n_phases = steps*(2 + 5L), n_gemms = steps*4L, n_chunks =
+ * steps*L*(chunks per CTA per layer, at most 32). */
+fm_status fm_profile_phases(fm_expert *h, int steps, uint64_t *out, size_t *n, void *stream);
+
 /* Wait for `stream`, then report (and clear) any device-side timeout. */
 fm_status fm_sync(fm_expert *h, void *stream);
 

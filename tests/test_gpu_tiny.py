@@ -183,7 +183,14 @@ def test_zero_and_constant_velocity_fields_are_exact():
     c = np.array([0.5, -2.0, 0.125] * 25, dtype=np.float32)
     e2 = Expert(shape, raw, out_bias=c)
     e2.set_prefix(kp, vp, 1, shape.prefix_len)
-    assert np.array_equal(e2.denoise(x0, 16), x0 - c)     # dt = -1/16, c powers of two
+    got = e2.denoise(x0, 16)
+    # v = c exactly; each update x <- x + dt c rounds once in fp32 (dt c is exact),
+    # so the exact reference is the fp32 recurrence, within 16 ulp of x0 - c
+    want = x0.copy()
+    for _ in range(16):
+        want = (want + np.float32(-1 / 16) * c).astype(np.float32)
+    assert np.array_equal(got, want)
+    assert np.all(np.abs(got - (x0.astype(np.float64) - c)) <= 16 * np.spacing(np.abs(x0 - c) + 2.0))
 
 
 def test_gqa_head_to_kv_group_map():

@@ -27,7 +27,8 @@ STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_NOT_READY", 3: "FM_ERR
 # Every symbol include/fm_expert.h declares.
 EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity", "fm_time_modulation",
            "fm_trace_bytes", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
-           "fm_get_geometry", "fm_expert_destroy", "fm_last_error", "fm_status_string",
+           "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases",
+           "fm_expert_destroy", "fm_last_error", "fm_status_string",
            "fm_abi_version")
 
 
@@ -82,6 +83,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_trace_velocity.argtypes = [vp, vp, ip, ip, vp, vp]
     lib.fm_get_fp8_weights.argtypes = [vp, ip, ip, vp, vp]
     lib.fm_sync.argtypes = [vp, vp]
+    lib.fm_profile_denoise.argtypes = [vp, ip, ip, ip, vp, vp]
+    lib.fm_profile_phases.argtypes = [vp, ip, vp, ctypes.POINTER(sz), vp]
     lib.fm_get_geometry.argtypes = [vp, ctypes.POINTER(ip), ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.fm_expert_destroy.argtypes = [vp]
     lib.fm_expert_destroy.restype = sz
@@ -92,7 +95,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_abi_version.restype = ip
     for name in ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity",
                  "fm_time_modulation", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
-                 "fm_get_geometry"):
+                 "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases"):
         getattr(lib, name).restype = ip
     _lib = lib
     return lib
@@ -234,6 +237,31 @@ class Expert:
         self._check("fm_get_fp8_weights", self.lib.fm_get_fp8_weights(self.h, layer, which, _ptr(codes),
                                                                        _ptr(scale)))
         return codes, scale
+
+    def profile(self, batch: int, steps: int, iters: int, stream=None):
+        """Mean (time-MLP ms, loop ms) over `iters` event-timed runs."""
+        ms = np.zeros(2, dtype=np.float32)
+        self._check("fm_profile_denoise", self.lib.fm_profile_denoise(self.h, batch, steps, iters, _ptr(ms),
+                                                                       _stream(stream)))
+        return float(ms[0]), float(ms[1])
+
+    def profile_phases(self, steps: int, stream=None):
+        """Timeline of one denoise (globaltimer ns, 0 where unused): compute
+        marks [n_ctas, n_phases, 8], MMA marks [n_ctas, n_gemms, 2], chunk
+        landed [n_ctas, n_chunks], chunk issued [n_ctas, n_chunks]."""
+        n = ctypes.c_size_t(0)
+        self._check("fm_profile_phases", self.lib.fm_profile_phases(self.h, steps, None, ctypes.byref(n), None))
+        buf = np.zeros(n.value, dtype=np.uint64)
+        self._check("fm_profile_phases", self.lib.fm_profile_phases(self.h, steps, _ptr(buf), ctypes.byref(n),
+                                                                     _stream(stream)))
+        L = self.shape.n_layers
+        n_ph, n_g = steps * (2 + 5 * L), steps * 4 * L
+        _, _, n_ctas = self.geometry()
+        rows = buf.reshape(n_ctas, -1)
+        n_ch = (rows.shape[1] - 16 * n_ph - 2 * n_g) // 2
+        a, b = 16 * n_ph, 16 * n_ph + 2 * n_g
+        return (rows[:, :a].reshape(n_ctas, n_ph, 16), rows[:, a:b].reshape(n_ctas, n_g, 2),
+                rows[:, b:b + n_ch], rows[:, b + n_ch:b + 2 * n_ch])
 
     def sync(self, stream=None):
         self._check("fm_sync", self.lib.fm_sync(self.h, _stream(stream)))

@@ -23,6 +23,7 @@ namespace {
 
 thread_local std::string g_create_error;
 
+
 struct DevBuf {
   void* p = nullptr;
   size_t n = 0;
@@ -38,7 +39,8 @@ struct fm_expert {
   int n_ctas = 0;
   int n_mod = 0;
   GemmPlan plan[4]{};
-  int uc = 0;
+  int att_blocks = 0;
+  int q_rows = 0;
   std::string err;
   std::vector<DevBuf> bufs;
   size_t bytes = 0;
@@ -124,38 +126,67 @@ fm_status dalloc(fm_expert* h, T** out, size_t bytes) {
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
-// Plans one linear over `nc` clusters (see GemmPlan).  `own_mult` is the
-// granularity of the columns a CTA owns after the reduction.
-bool plan_gemm(GemmPlan& g, int N, int K, int nc, int pref_ks, int own_mult) {
-  g.N = N;
-  g.K = K;
-  int ks = pref_ks;
-  while (ks > 1 && ((K / 64) % ks != 0)) ks /= 2;
-  if (K % 64 != 0) return false;
-  g.KS = ks;
-  g.NS = kClusterSize / ks;
-  const int per = (N + nc * g.NS - 1) / (nc * g.NS);
-  g.Ng = round_up(std::max(per, 1), std::max(16, ks * own_mult));
-  if (g.Ng > 256) return false;
-  g.own = g.Ng / ks;
-  g.kslice = K / ks;
-  g.nchunk = g.kslice / 64;
-  g.chunk_bytes = (uint32_t)g.Ng * 128u;
-  g.busy_clusters = std::min(nc, (N + g.NS * g.Ng - 1) / (g.NS * g.Ng));
-  if ((size_t)g.nchunk * 8192 > (size_t)kWorkBytes) return false;
-  if ((size_t)(kBiasRow + 1) * g.Ng * 4 > (size_t)kWorkBytes) return false;
-  return true;
+// Plans one linear over `nc` clusters (see GemmPlan).  Channels are dealt to
+// clusters in units of NS x 16 so that per-cluster work differs by at most one
+// unit; the K split starts at `max_ks` and is halved (more n-groups per
+// cluster) until an n-group fits one MMA (N <= 256) and the work region
+// (activation blocks + receive buffer).  `pair_cols`: owned columns come in
+// gate/up pairs of even width (gate_up).
+bool plan_gemm(GemmPlan& g, int N, int K, int nc, int max_ks, bool pair_cols) {
+  if (K % 64 != 0 || nc < 1 || nc > kMaxClusters) return false;
+  for (int ks = max_ks; ks >= 1; ks /= 2) {
+    if ((K / 64) % ks != 0) continue;
+    const int NS = kClusterSize / ks;
+    const int unit = std::max(16, ks * (pair_cols ? 4 : 2));
+    const int cunit = NS * unit;
+    const int U = (N + cunit - 1) / cunit;
+    const int q = U / nc, r = U % nc;
+    g = GemmPlan{};
+    g.N = N;
+    g.K = K;
+    g.KS = ks;
+    g.NS = NS;
+    g.kslice = K / ks;
+    g.nchunk = g.kslice / 64;
+    int off = 0;
+    for (int c = 0; c < nc; ++c) {
+      const int units = q + (c < r ? 1 : 0);
+      g.ng[c] = units * unit;
+      g.ch_off[c] = off;
+      off += pair_cols ? NS * g.ng[c] / 2 : NS * g.ng[c];
+      if (g.ng[c] > 0) g.busy_clusters++;
+      g.max_ng = std::max(g.max_ng, g.ng[c]);
+    }
+    if (g.max_ng > 256) continue;
+    // work region: activation blocks (later the outgoing partials), then the
+    // receive buffer; the receive blocks have rows padded to 4 floats
+    const size_t ownp = (size_t)((g.max_ng / ks + 3) & ~3);
+    const size_t blocks = (size_t)ks * kRecvRows * ownp * 4;
+    const size_t a_bytes = (size_t)g.nchunk * 8192;
+    const size_t recv_off = ((a_bytes > blocks ? a_bytes : blocks) + 15) & ~(size_t)15;
+    if (recv_off + blocks > (size_t)kWorkBytes) continue;
+    return true;
+  }
+  return false;
 }
 
 // Source row (in the concatenated matrix of gemm g) of packed channel q of the
-// n-group (cluster c, group ng); -1 for padding.
-int source_row(const fm_expert* h, int g, int c, int ng, int q) {
+// n-group (cluster c, group grp); -1 for padding.
+int source_row(const fm_expert* h, int g, int c, int grp, int q) {
   const fm_config& cf = h->cfg;
   const GemmPlan& gp = h->plan[g];
-  const int pc = (c * gp.NS + ng) * gp.Ng + q;
+  const int ng = gp.ng[c];
+  if (g == G_GU) {
+    const int own = ng / gp.KS, uown = own / 2;
+    const int ks = q / own, rr = q % own;
+    const int u = gp.ch_off[c] + grp * (ng / 2) + ks * uown + (rr % uown);
+    if (u >= cf.d_ff) return -1;
+    return rr < uown ? u : cf.d_ff + u;
+  }
+  const int pc = gp.ch_off[c] + grp * ng + q;
+  if (pc >= gp.N) return -1;
   if (g == G_QKV) {
     const int qn = cf.n_q_heads * cf.head_dim, kn = cf.n_kv_heads * cf.head_dim;
-    if (pc >= gp.N) return -1;
     if (pc < qn + kn) {
       // rotate-half partners (i, i + hd/2) are packed next to each other
       const int base = pc < qn ? 0 : qn;
@@ -164,27 +195,46 @@ int source_row(const fm_expert* h, int g, int c, int ng, int q) {
       const int i = w >> 1;
       return base + head * cf.head_dim + i + (w & 1) * (cf.head_dim / 2);
     }
-    return pc;
   }
-  if (g == G_GU) {
-    const int ks = q / gp.own, rr = q % gp.own, uown = gp.own / 2;
-    const int u = (c * gp.NS + ng) * h->uc + ks * uown + (rr % uown);
-    if (u >= cf.d_ff) return -1;
-    return rr < uown ? u : cf.d_ff + u;
-  }
-  return pc < gp.N ? pc : -1;
+  return pc;
 }
 
 fm_status build_plan(fm_expert* h) {
   const fm_config& c = h->cfg;
   const int nc = h->n_clusters;
   const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
-  if (!plan_gemm(h->plan[G_QKV], qkv, c.d_model, nc, 8, 2) ||
-      !plan_gemm(h->plan[G_O], c.d_model, c.n_q_heads * c.head_dim, nc, 8, 8) ||
-      !plan_gemm(h->plan[G_GU], 2 * c.d_ff, c.d_model, nc, 4, 16) ||
-      !plan_gemm(h->plan[G_DOWN], c.d_model, c.d_ff, nc, 8, 8))
+  if (!plan_gemm(h->plan[G_QKV], qkv, c.d_model, nc, 8, false) ||
+      !plan_gemm(h->plan[G_O], c.d_model, c.n_q_heads * c.head_dim, nc, 8, false) ||
+      !plan_gemm(h->plan[G_GU], 2 * c.d_ff, c.d_model, nc, 8, true) ||
+      !plan_gemm(h->plan[G_DOWN], c.d_model, c.d_ff, nc, 8, false))
     return set_err(h, FM_ERR_UNSUPPORTED, "no work plan for this shape on %d clusters", nc);
-  h->uc = h->plan[G_GU].Ng / 2;
+  // epilogue work per compute thread: QKV rows per thread fit the 8 KB
+  // rotation area at the end of the work region (8 rows x 128 threads); a
+  // residual thread holds at most 4 column pairs in registers
+  {
+    const GemmPlan& pq = h->plan[G_QKV];
+    const int npair_q = pq.max_ng / pq.KS / 2;
+    const int per = npair_q > 0 ? 128 / npair_q : 0;
+    const size_t ownp = (size_t)((pq.max_ng / pq.KS + 3) & ~3);
+    const size_t blocks = (size_t)pq.KS * kRecvRows * ownp * 4;
+    const size_t a_bytes = (size_t)pq.nchunk * 8192;
+    const size_t recv_off = ((a_bytes > blocks ? a_bytes : blocks) + 15) & ~(size_t)15;
+    if (per < 1 || (c.chunk_len + per - 1) / per > 8 || recv_off + blocks + 8192 > (size_t)kWorkBytes ||
+        h->plan[G_O].max_ng / h->plan[G_O].KS > 16 || h->plan[G_DOWN].max_ng / h->plan[G_DOWN].KS > 16 ||
+        h->plan[G_GU].max_ng / h->plan[G_GU].KS / 4 > 128)
+      return set_err(h, FM_ERR_UNSUPPORTED, "too many owned columns per CTA on %d clusters", nc);
+  }
+  const int G = c.n_q_heads / c.n_kv_heads;
+  h->att_blocks = (G * c.chunk_len + 63) / 64;
+  h->q_rows = h->att_blocks * 64;
+  // attention work region: q, K and V tiles and the combine buffer
+  const size_t att = (size_t)3 * 64 * c.head_dim * 2 + (size_t)kClusterSize * 8 * (c.head_dim + 4) * 4;
+  const size_t inproj = (size_t)c.chunk_len * c.action_dim * 4 +
+                        (size_t)(h->plan[G_DOWN].max_ng / h->plan[G_DOWN].KS) * (c.action_dim + c.chunk_len) * 4;
+  if (c.chunk_len * c.action_dim % 2 != 0 || (h->plan[G_DOWN].max_ng / h->plan[G_DOWN].KS) * c.action_dim > 32 * 128)
+    return set_err(h, FM_ERR_UNSUPPORTED, "in-proj tile: chunk_len * action_dim must be even, owned rows x A <= 4096");
+  if (att > (size_t)kWorkBytes || inproj > (size_t)kWorkBytes)
+    return set_err(h, FM_ERR_UNSUPPORTED, "attention or in-proj tiles exceed shared memory");
   return FM_OK;
 }
 
@@ -208,19 +258,20 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
     const int cl = cta / kClusterSize, rank = cta % kClusterSize;
     for (int g = 0; g < 4; ++g) {
       const GemmPlan& gp = h->plan[g];
-      if (cl >= gp.busy_clusters) continue;
-      const int ng = rank / gp.KS, ks = rank % gp.KS;
+      const int ng = gp.ng[cl];
+      if (ng == 0) continue;
+      const int grp = rank / gp.KS, ks = rank % gp.KS;
       const uint32_t roff = (uint32_t)rows.size();
-      for (int q = 0; q < gp.Ng; ++q) rows.push_back(source_row(h, g, cl, ng, q));
+      for (int q = 0; q < ng; ++q) rows.push_back(source_row(h, g, cl, grp, q));
       for (int i = 0; i < gp.nchunk; ++i) {
         PackChunk pc{};
         pc.dst_off = off;
         pc.rowidx_off = roff;
-        pc.nrows = (uint16_t)gp.Ng;
+        pc.nrows = (uint16_t)ng;
         pc.mat = (uint8_t)g;
         pc.kb = (uint32_t)(ks * gp.nchunk + i);
         jobs.push_back(pc);
-        off += gp.chunk_bytes;
+        off += (uint64_t)ng * 128;
       }
     }
   }
@@ -417,7 +468,8 @@ StepParams base_params(const fm_expert* h) {
   p.n_clusters = h->n_clusters;
   p.n_ctas = h->n_ctas;
   for (int g = 0; g < 4; ++g) p.g[g] = h->plan[g];
-  p.uc = h->uc;
+  p.att_blocks = h->att_blocks;
+  p.q_rows = h->q_rows;
   p.arena = h->arena;
   p.layer_bytes = h->layer_bytes;
   p.span_off = h->span_off;
@@ -451,6 +503,11 @@ StepParams base_params(const fm_expert* h) {
   p.update_x = 1;
   p.dt = 0.f;
   p.spin_budget = 4000000000LL;   // ~2 s at 2 GHz
+  p.tlog = nullptr;
+  p.tlog_stride = 0;
+  p.tlog_mma_off = 0;
+  p.tlog_chunk_off = 0;
+  p.tlog_chunks = 0;
   return p;
 }
 
@@ -470,7 +527,7 @@ TimeParams time_params(const fm_expert* h, int steps) {
 
 // Enqueues one full denoise of `batch` requests (x already in h->x).
 cudaError_t enqueue_denoise(fm_expert* h, int batch, int steps, cudaStream_t st) {
-  cudaError_t e = cudaMemsetAsync(h->bar_count, 0, 4, st);
+  cudaError_t e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
   if (e != cudaSuccess) return e;
   e = launch_time(time_params(h, steps), h->n_sms, st);
   if (e != cudaSuccess) return e;
@@ -484,7 +541,7 @@ cudaError_t enqueue_denoise(fm_expert* h, int batch, int steps, cudaStream_t st)
     p.step1 = steps;
     p.dt = -1.0f / (float)steps;
     if (b > 0) {
-      e = cudaMemsetAsync(h->bar_count, 0, 4, st);
+      e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
       if (e != cudaSuccess) return e;
     }
     e = launch_step(p, st);
@@ -569,7 +626,7 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
     set_err(h, FM_ERR_UNSUPPORTED, "no co-resident clusters of %d CTAs", kClusterSize);
     return bail(FM_ERR_UNSUPPORTED);
   }
-  h->n_clusters = std::min(ncl, h->n_sms / kClusterSize);
+  h->n_clusters = std::min(std::min(ncl, h->n_sms / kClusterSize), kMaxClusters);
   h->n_ctas = h->n_clusters * kClusterSize;
   if ((st = build_plan(h)) != FM_OK) return bail(st);
   if (cfg->wtype == FM_W_FP8_E4M3) {
@@ -601,13 +658,13 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
   ALLOC_OR_BAIL(h->z_f, (size_t)kRows * d * 2);
   ALLOC_OR_BAIL(h->o_act, (size_t)kRows * c.n_q_heads * c.head_dim * 2);
   ALLOC_OR_BAIL(h->u_act, (size_t)kRows * c.d_ff * 2);
-  ALLOC_OR_BAIL(h->sumsq_a, (size_t)h->n_clusters * kRows * 4);
-  ALLOC_OR_BAIL(h->sumsq_f, (size_t)h->n_clusters * kRows * 4);
-  ALLOC_OR_BAIL(h->qbuf, (size_t)c.n_q_heads * kRows * c.head_dim * 2);
+  ALLOC_OR_BAIL(h->sumsq_a, (size_t)h->n_ctas * kRows * 4);
+  ALLOC_OR_BAIL(h->sumsq_f, (size_t)h->n_ctas * kRows * 4);
+  ALLOC_OR_BAIL(h->qbuf, (size_t)c.n_kv_heads * h->q_rows * c.head_dim * 2);
   const size_t kv = (size_t)c.n_layers * B * c.n_kv_heads * h->S_max * c.head_dim * 2;
   ALLOC_OR_BAIL(h->kcache, kv);
   ALLOC_OR_BAIL(h->vcache, kv);
-  ALLOC_OR_BAIL(h->bar_count, 4);
+  ALLOC_OR_BAIL(h->bar_count, (size_t)(h->n_ctas + 4) * 4);
   ALLOC_OR_BAIL(h->err_word, 4);
 #undef ALLOC_OR_BAIL
   if (cudaDeviceSynchronize() != cudaSuccess) {
@@ -769,7 +826,7 @@ fm_status fm_velocity(fm_expert* h, const float* x, int batch, int step_index, i
     p.step0 = step_index;
     p.step1 = step_index + 1;
     p.update_x = 0;
-    CK(cudaMemsetAsync(h->bar_count, 0, 4, st));
+    CK(cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st));
     CK(launch_step(p, st));
   }
   CK(cudaMemcpyAsync(v_out, h->vbuf, (size_t)batch * xs * 4, cudaMemcpyDefault, st));
@@ -819,7 +876,7 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
             kn = c.n_kv_heads * c.head_dim, F = c.d_ff, hd = c.head_dim;
   float* out = trace;
   std::vector<float> hbuf((size_t)T * d);
-  std::vector<uint16_t> qh((size_t)c.n_q_heads * kRows * hd), oh((size_t)kRows * qn),
+  std::vector<uint16_t> qh((size_t)c.n_kv_heads * h->q_rows * hd), oh((size_t)kRows * qn),
       uh((size_t)kRows * F), kvh((size_t)h->S_max * hd);
   const size_t lay = (size_t)c.max_batch * c.n_kv_heads * h->S_max * hd;
   auto run = [&](int layer0, int layer1, int inproj, int outproj) -> fm_status {
@@ -831,7 +888,7 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
     p.do_inproj = inproj;
     p.do_outproj = outproj;
     p.update_x = 0;
-    CK(cudaMemsetAsync(h->bar_count, 0, 4, st));
+    CK(cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st));
     CK(launch_step(p, st));
     CK(cudaStreamSynchronize(st));
     return check_err_word(h);
@@ -843,10 +900,12 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
     out += (size_t)T * d;
     if ((s = run(l, l + 1, 0, 0)) != FM_OK) return s;
     CK(cudaMemcpy(qh.data(), h->qbuf, qh.size() * 2, cudaMemcpyDeviceToHost));
+    const int G = c.n_q_heads / c.n_kv_heads;
     for (int t = 0; t < T; ++t)
       for (int n = 0; n < qn; ++n) {
         const int head = n / hd, e = n % hd;
-        out[(size_t)t * qn + n] = swz_get(qh, ((size_t)head * kRows + t) * hd, t, e);
+        const int row = (head % G) * T + t;
+        out[(size_t)t * qn + n] = swz_get(qh, ((size_t)(head / G) * h->q_rows + row) * hd, row, e);
       }
     out += (size_t)T * qn;
     for (int which = 0; which < 2; ++which) {
@@ -884,6 +943,92 @@ fm_status fm_get_fp8_weights(fm_expert* h, int layer, int which, uint8_t* codes,
   if (h->cfg.wtype != FM_W_FP8_E4M3) return set_err(h, FM_ERR_INVALID_ARG, "handle holds bf16 weights");
   (void)layer; (void)which; (void)codes; (void)scale;
   return set_err(h, FM_ERR_UNSUPPORTED, "not available");
+}
+
+fm_status fm_profile_denoise(fm_expert* h, int batch, int steps, int iters, float* ms, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (!ms || iters < 1) return set_err(h, FM_ERR_INVALID_ARG, "ms is NULL or iters < 1");
+  if (steps < 1 || steps > c.max_steps || batch < 1 || batch > c.max_batch)
+    return set_err(h, FM_ERR_INVALID_ARG, "batch %d / steps %d invalid", batch, steps);
+  if (h->prefix_batch != batch)
+    return set_err(h, FM_ERR_NOT_READY, "fm_set_prefix was not called for batch %d", batch);
+  CK(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  cudaEvent_t ev[3];
+  for (auto& e : ev) CK(cudaEventCreate(&e));
+  double t_time = 0.0, t_loop = 0.0;
+  const size_t xs = (size_t)c.chunk_len * c.action_dim;
+  fm_status out = FM_OK;
+  for (int i = 0; i < iters && out == FM_OK; ++i) {
+    cudaError_t e = cudaEventRecord(ev[0], st);
+    if (e == cudaSuccess) e = launch_time(time_params(h, steps), h->n_sms, st);
+    if (e == cudaSuccess) e = cudaEventRecord(ev[1], st);
+    for (int b = 0; b < batch && e == cudaSuccess; ++b) {
+      StepParams p = base_params(h);
+      p.b = b;
+      p.x = h->x + b * xs;
+      p.vbuf = h->vbuf + b * xs;
+      p.step1 = steps;
+      p.dt = -1.0f / (float)steps;
+      e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
+      if (e == cudaSuccess) e = launch_step(p, st);
+    }
+    if (e == cudaSuccess) e = cudaEventRecord(ev[2], st);
+    if (e == cudaSuccess) e = cudaEventSynchronize(ev[2]);
+    float a = 0.f, b2 = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&a, ev[0], ev[1]);
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&b2, ev[1], ev[2]);
+    if (e != cudaSuccess) out = set_err(h, FM_ERR_CUDA, "profile: %s", cudaGetErrorString(e));
+    t_time += a;
+    t_loop += b2;
+  }
+  for (auto& e : ev) cudaEventDestroy(e);
+  if (out != FM_OK) return out;
+  ms[0] = (float)(t_time / iters);
+  ms[1] = (float)(t_loop / iters);
+  return check_err_word(h);
+}
+
+fm_status fm_profile_phases(fm_expert* h, int steps, uint64_t* out, size_t* n, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (!n) return set_err(h, FM_ERR_INVALID_ARG, "n is NULL");
+  if (steps < 1 || steps > c.max_steps) return set_err(h, FM_ERR_INVALID_ARG, "steps %d invalid", steps);
+  const int n_phases = steps * (2 + 5 * c.n_layers), n_gemms = steps * 4 * c.n_layers;
+  int per_layer = 0;
+  for (int g = 0; g < 4; ++g) per_layer += h->plan[g].nchunk;
+  const int n_chunks = steps * c.n_layers * per_layer;
+  const int stride = 16 * n_phases + 2 * n_gemms + 2 * n_chunks;
+  const size_t need = (size_t)h->n_ctas * stride;
+  if (!out) {
+    *n = need;
+    return FM_OK;
+  }
+  if (*n < need) return set_err(h, FM_ERR_INVALID_ARG, "out holds %zu values, %zu needed", *n, need);
+  if (h->prefix_batch < 1) return set_err(h, FM_ERR_NOT_READY, "fm_set_prefix was not called");
+  CK(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  unsigned long long* d = nullptr;
+  CK(cudaMalloc(&d, need * 8));
+  cudaError_t e = cudaMemsetAsync(d, 0, need * 8, st);
+  if (e == cudaSuccess) e = launch_time(time_params(h, steps), h->n_sms, st);
+  StepParams p = base_params(h);
+  p.step1 = steps;
+  p.dt = -1.0f / (float)steps;
+  p.tlog = d;
+  p.tlog_stride = stride;
+  p.tlog_mma_off = 16 * n_phases;
+  p.tlog_chunk_off = 16 * n_phases + 2 * n_gemms;
+  p.tlog_chunks = n_chunks;
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
+  if (e == cudaSuccess) e = launch_step(p, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(out, d, need * 8, cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  cudaFree(d);
+  if (e != cudaSuccess) return set_err(h, FM_ERR_CUDA, "profile phases: %s", cudaGetErrorString(e));
+  *n = need;
+  return check_err_word(h);
 }
 
 fm_status fm_sync(fm_expert* h, void* stream) {

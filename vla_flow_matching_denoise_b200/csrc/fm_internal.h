@@ -13,39 +13,45 @@
 //  * KV cache: [L][B][H_kv][S_max][hd] bf16, each 256-byte row (hd = 128)
 //    split in 16-byte pieces stored at piece (c ^ (row & 7)); rows 0..P-1 are
 //    the prefix, rows P..P+T-1 the chunk of the current velocity evaluation.
-//  * q buffer: [H_q][64][hd] bf16, same per-row piece swizzle.
+//  * q buffer: per KV group g, rows (h % G) * T + t for the G query heads
+//    of the group, [H_kv][q_rows][hd] bf16, same per-row piece swizzle.
 #pragma once
 #include <cstdint>
 
 namespace fm {
 
 constexpr int kClusterSize = 8;        // CTAs per cluster (portable maximum)
+constexpr int kMaxClusters = 24;       // 8-CTA clusters a B200 can hold (148 SMs)
 constexpr int kComputeWarps = 4;       // warps 2..5
 constexpr int kThreads = 192;          // producer warp, MMA warp, 4 compute warps
 constexpr int kRows = 64;              // MMA M: token rows per tile
 constexpr int kMaxT = 50;              // valid token rows (one chunk)
 constexpr int kBiasRow = 50;           // row carrying the AdaRMSNorm shift vector
+constexpr int kRecvRows = 51;          // rows 0..50 travel in the split-K reduction
 constexpr int kTimeDim = 256;
 constexpr int kRingSlots = 16;         // mbarrier pairs of the weight ring
-constexpr int kWorkBytes = 64 * 1024;  // activation / staging region
+constexpr int kRingBytes = 126 * 1024; // weight ring
+constexpr int kWorkBytes = 96 * 1024;  // activation / receive region
 constexpr int kSmemMax = 232448;       // dynamic shared memory per CTA (227 KB)
 
 enum GemmId { G_QKV = 0, G_O = 1, G_GU = 2, G_DOWN = 3 };
 
-// One GEMM of a layer, partitioned over clusters: cluster c owns Nc packed
-// output channels; inside it CTA j works on n-group j / KS (Ng channels) and
-// K-slice j % KS (kslice columns); after the in-cluster reduction CTA j owns
-// `own` output columns of its n-group.
+// One linear of a layer, partitioned over clusters.  Cluster c works on
+// NS n-groups of ng[c] packed output channels each (0 = idle cluster); CTA j
+// of the cluster takes n-group j / KS and K-slice j % KS (kslice columns).
+// After the in-cluster split-K reduction CTA j owns ng[c] / KS consecutive
+// columns of its n-group.  Packed channels of cluster c start at ch_off[c]
+// (for gate_up: u columns, each n-group holding gate and up rows in pairs).
 struct GemmPlan {
-  int N;          // logical output channels
+  int N;          // logical output channels (gate_up: 2 F packed rows)
   int K;          // reduction length
   int NS, KS;     // n-groups and K-slices per cluster (NS * KS = 8)
-  int Ng;         // packed channels per n-group (MMA N, multiple of 8, <= 256)
-  int own;        // columns owned per CTA after the reduction
   int kslice;     // K per slice (multiple of 64)
-  int busy_clusters;  // clusters with at least one channel
-  uint32_t chunk_bytes;  // Ng * 128
-  int nchunk;     // kslice / 64
+  int nchunk;     // kslice / 64: weight chunks and activation blocks per CTA
+  int busy_clusters;
+  int max_ng;
+  int ch_off[kMaxClusters];
+  int ng[kMaxClusters];
 };
 
 struct StepParams {
@@ -56,7 +62,9 @@ struct StepParams {
   float eps;
   int n_clusters, n_ctas;
   GemmPlan g[4];
-  int uc;            // u columns per n-group (gate/up pairs)
+  // attention: per KV group, G*T query rows (head-major) in blocks of 64
+  int att_blocks;            // 64-row blocks per KV group
+  int q_rows;                // padded rows per KV group in the q buffer (multiple of 64)
   // weights
   const uint8_t* arena;      // packed per-layer weights
   uint64_t layer_bytes;      // bytes of one layer in the arena
@@ -77,12 +85,13 @@ struct StepParams {
   uint16_t* z_f;             // ACT64 [64, d]: h (1 + s_f), row 50 = b_f
   uint16_t* o_act;           // ACT64 [64, H_q hd]
   uint16_t* u_act;           // ACT64 [64, F]
-  float* sumsq_a;            // [n_clusters][64] per-cluster row sums of h^2
+  float* sumsq_a;            // [n_ctas][64] per-CTA partial row sums of h^2
   float* sumsq_f;
-  uint16_t* qbuf;            // [H_q][64][hd]
+  uint16_t* qbuf;            // [H_kv][q_rows][hd]: row (h % G) * T + t of group h / G
   uint16_t* kcache;          // [L][B][H_kv][S_max][hd]
   uint16_t* vcache;
-  uint32_t* bar_count;       // grid barrier counter (zeroed before launch)
+  uint32_t* bar_count;       // grid barrier: one arrival word per CTA, 16-byte aligned,
+                             // zeroed before launch (word = barriers passed)
   uint32_t* err;             // error word (non-zero: a bounded wait gave up)
   // schedule of this launch
   int step0, step1;          // modulation rows used
@@ -90,6 +99,12 @@ struct StepParams {
   int do_inproj, do_outproj, update_x;
   float dt;
   long long spin_budget;     // cycles before a wait gives up
+  // optional phase timeline (globaltimer ns); null when not profiling
+  unsigned long long* tlog;  // [n_ctas][tlog_stride]: 8 marks per phase, 2 per GEMM (MMA warp),
+  int tlog_stride;           // then per weight chunk: landed (MMA warp) and issued (producer)
+  int tlog_mma_off;          // offset of the MMA-warp marks inside a CTA's row
+  int tlog_chunk_off;        // offset of the per-chunk marks
+  int tlog_chunks;           // chunk slots per section
 };
 
 struct TimeParams {

@@ -13,21 +13,27 @@
 //    global counter, bounded spin).
 //  * Weights dominate the bytes (34.6 MB per layer at d = 1024), so warp 0 of
 //    every CTA streams its share of every layer, in consumption order, through
-//    a 160 KB shared-memory ring with 1-D bulk (TMA) copies.  The stream runs
+//    a 128 KB shared-memory ring with 1-D bulk (TMA) copies.  The stream runs
 //    ahead across phases and barriers; only ring space throttles it.
-//  * Each linear is split over clusters by output channels and, inside a
-//    cluster, over its 8 CTAs by K (and n-groups).  Warp 1 issues tcgen05.mma
-//    with M = 64 token rows (50 valid + the shift row + padding), N = the
-//    CTA's channels, accumulating fp32 in TMEM.  The split-K partial sums are
-//    reduced in a fixed order through distributed shared memory, so results
-//    are bit-reproducible.
+//  * Each linear is split over clusters by output channels (balanced per
+//    cluster) and, inside a cluster, over its 8 CTAs by K and n-groups.  Warp
+//    1 issues tcgen05.mma with M = 64 token rows (50 valid + the shift row +
+//    padding), N = the CTA's channels, accumulating fp32 in TMEM.
+//  * Split-K partials go straight from TMEM registers to the CTA that owns
+//    the output columns: st.async into its receive buffer completes bytes on
+//    its mbarrier, so the owner waits once and reduces from local shared
+//    memory in a fixed order (results are bit-reproducible).
 //  * AdaRMSNorm is folded into the linears: the owner of a residual column
 //    writes z = bf16(h (1 + s)) and, in row 50, the shift b; the consumer
 //    linear's epilogue applies rstd(row) to rows 0..49 and adds row 50
-//    (= b W^T).  This equals y W^T with y = h rstd (1 + s) + b.
-//  * Attention (tiny: 50 queries) uses mma.sync with an online softmax per
-//    key split and a log-sum-exp combine across the cluster.
+//    (= b W^T).  This equals y W^T with y = h rstd (1 + s) + b.  Row sums of
+//    h^2 are published per CTA and summed by the consumer in a fixed order.
+//  * Attention (50 queries per head) runs per (KV group, block of 64 query
+//    rows of that group's heads) on one cluster, keys split over its 8 CTAs,
+//    mma.sync with an online softmax, partials pushed to the row owners for
+//    the log-sum-exp combine.
 #include <cuda_bf16.h>
+#include <cstddef>
 #include <cstdint>
 
 #include "fm_internal.h"
@@ -38,34 +44,32 @@ namespace fm {
 
 namespace {
 
-constexpr uint32_t kRingBytes = 160 * 1024;
-
 struct Ctrl {
   uint64_t full[kRingSlots];
   uint64_t empty[kRingSlots];
   uint64_t act_full;
   uint64_t mma_done;
-  uint64_t xa;        // cluster exchange: partial sums / attention partials
-  uint64_t xb;        // cluster exchange: row sums of squares, attention reuse
+  uint64_t recv;      // split-K / attention partials pushed by the cluster
   uint64_t att;       // attention tile loads
   uint64_t drain;
+  uint64_t xsync;     // cluster rendezvous (8 arrivals)
   uint32_t tmem_slot;
   int abort;
-  float rstd[kRows];
-  float sq_own[kRows];
+  alignas(16) float rstd[kRows];
+  alignas(16) float red[8][kRows];   // written with float4 stores
 };
+static_assert(offsetof(Ctrl, red) % 16 == 0 && offsetof(Ctrl, rstd) % 16 == 0, "vector alignment");
 
 constexpr size_t kSmemBytes = 1024 + kRingBytes + kWorkBytes + ((sizeof(Ctrl) + 127) / 128) * 128;
+static_assert(kSmemBytes <= (size_t)kSmemMax, "shared memory budget");
 
 // Error codes (bit flags in p.err).
 enum : uint32_t {
   E_GRID = 1u << 0,
   E_RING_PROD = 1u << 1,
   E_RING_MMA = 1u << 2,
-  E_ACT = 1u << 3,
+  E_RECV = 1u << 3,
   E_MMA_DONE = 1u << 4,
-  E_XA = 1u << 5,
-  E_XB = 1u << 6,
   E_ATT = 1u << 7,
 };
 
@@ -73,17 +77,7 @@ __device__ __forceinline__ bool wait_ab(uint32_t bar, uint32_t parity, long long
                                         volatile int* abort) {
   if (mbar_test(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_test(bar, parity)) {
-    if (*abort) return false;
-    if (clock64() - t0 > budget) return false;
-  }
-  return true;
-}
-__device__ __forceinline__ bool wait_cl(uint32_t bar, uint32_t parity, long long budget,
-                                        volatile int* abort) {
-  if (mbar_test_cluster(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_test_cluster(bar, parity)) {
+  while (!mbar_test_sleep(bar, parity, 1000000u)) {
     if (*abort) return false;
     if (clock64() - t0 > budget) return false;
   }
@@ -93,13 +87,9 @@ __device__ __forceinline__ bool wait_cl(uint32_t bar, uint32_t parity, long long
 // Ring placement shared by producer and consumer: a chunk of `sz` bytes goes
 // right after the previous one, or wraps to offset 0 when it does not fit.
 __device__ __forceinline__ uint32_t ring_place(uint32_t& pos, uint32_t sz) {
-  const uint32_t p = (pos + sz > kRingBytes) ? 0u : pos;
+  const uint32_t p = (pos + sz > (uint32_t)kRingBytes) ? 0u : pos;
   pos = p + sz;
   return p;
-}
-
-__device__ __forceinline__ bool gemm_busy(const GemmPlan& g, int cluster) {
-  return cluster < g.busy_clusters;
 }
 
 __device__ __forceinline__ uint16_t bf16_bits(float x) {
@@ -107,18 +97,9 @@ __device__ __forceinline__ uint16_t bf16_bits(float x) {
   return *reinterpret_cast<uint16_t*>(&b);
 }
 
-// 16-byte piece address inside an ACT64 matrix (row r, columns c .. c+7).
-__device__ __forceinline__ uint16_t* act64_piece(uint16_t* base, int r, int c) {
-  return base + (size_t)(c >> 6) * (kRows * 64) + (size_t)r * 64 + ((((c & 63) >> 3) ^ (r & 7)) << 3);
-}
-
-__device__ __forceinline__ uint4 pack8_bf16(const float (&v)[8]) {
-  uint4 u;
-  u.x = pack_bf16(v[0], v[1]);
-  u.y = pack_bf16(v[2], v[3]);
-  u.z = pack_bf16(v[4], v[5]);
-  u.w = pack_bf16(v[6], v[7]);
-  return u;
+// Element offset of (row r, column c) inside an ACT64 matrix.
+__device__ __forceinline__ size_t act64_off(int r, int c) {
+  return (size_t)(c >> 6) * (kRows * 64) + (size_t)r * 64 + ((((c & 63) >> 3) ^ (r & 7)) << 3) + (c & 7);
 }
 
 // Element index inside a row of hd bf16 values stored with 16-byte pieces
@@ -127,9 +108,14 @@ __device__ __forceinline__ int swz(int row, int e) {
   return ((((e >> 3) ^ (row & 7))) << 3) | (e & 7);
 }
 
+__device__ __forceinline__ unsigned long long gtimer() {
+  unsigned long long t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
 struct Ctx {
   const StepParams* p;
-  uint8_t* ring;
   uint8_t* work;
   Ctrl* ctl;
   uint32_t tmem;
@@ -138,7 +124,7 @@ struct Ctx {
   int warp;             // 2..5
   int lane;
   uint32_t gemm_count;  // GEMM phases run (parity of act_full / mma_done)
-  uint32_t xa_count, xb_count, att_count;
+  uint32_t recv_count, att_count, xs_count;
   uint32_t epoch;       // grid barriers passed
   int P;                // prefix length (read from the device)
   bool ok;
@@ -146,58 +132,80 @@ struct Ctx {
 
 __device__ __forceinline__ void compute_sync() { named_bar_sync(1, kComputeWarps * 32); }
 
+// Phase timeline (profiling only): mark `slot` of the current phase: 0 start,
+// 1 MMA / attention compute done, 2 partials pushed, 3 partials received,
+// 4 epilogue done, 5 barrier arrival issued, 6 partials staged, 7 staging
+// synchronised, 8.. phase-specific points.
+__device__ __forceinline__ void tmark(const Ctx& c, int slot) {
+  if (c.p->tlog != nullptr && c.tid == 0) {
+    const int idx = (int)c.epoch * 16 + slot;
+    if (idx < c.p->tlog_mma_off) c.p->tlog[(size_t)c.cta * c.p->tlog_stride + idx] = gtimer();
+  }
+}
+
 __device__ void fail(Ctx& c, uint32_t code) {
   atomicOr(c.p->err, code);
   c.ctl->abort = 1;
   c.ok = false;
 }
 
-// Grid barrier among the compute warps of every CTA.
+// Grid barrier among the compute warps of every CTA.  Each CTA publishes the
+// number of barriers it has passed in its own word (a release store, no
+// contended atomic); warp 0 of the compute warps polls all words with vector
+// loads until every CTA has arrived.
 __device__ void grid_sync(Ctx& c) {
   if (!c.ok) return;
+  tmark(c, 4);
   fence_proxy_async_global();
-  __threadfence();
   compute_sync();
+  const uint32_t target = c.epoch + 1;
+  uint32_t* flags = c.p->bar_count;
   if (c.tid == 0) {
-    red_release_add(c.p->bar_count, 1u);
-    const uint32_t target = (c.epoch + 1) * (uint32_t)c.p->n_ctas;
+    // cumulative: the CTA barrier above orders every compute thread's writes
+    // before this release
+    fence_acq_rel_gpu();
+    st_release_u32(flags + c.cta, target);
+    tmark(c, 5);
+  }
+  if (c.warp == 2) {
+    const int n4 = (c.p->n_ctas + 3) / 4;
     const long long t0 = clock64();
     bool good = true;
-    while (ld_acquire_u32(c.p->bar_count) < target) {
+    for (;;) {
+      bool mine = true;
+      for (int i = c.lane; i < n4; i += 32) {
+        const uint4 f = ld_relaxed_v4(flags + 4 * i);
+        const int base = 4 * i, n = c.p->n_ctas;
+        mine = mine && f.x >= target && (base + 1 >= n || f.y >= target) && (base + 2 >= n || f.z >= target) &&
+               (base + 3 >= n || f.w >= target);
+      }
+      if (__all_sync(0xffffffffu, mine)) break;
       if (*(volatile uint32_t*)c.p->err != 0u || clock64() - t0 > c.p->spin_budget) {
         good = false;
         break;
       }
     }
-    if (!good) fail(c, E_GRID);
-    __threadfence();
-    fence_proxy_async_global();
+    if (c.lane == 0) {
+      if (!good) fail(c, E_GRID);
+      fence_acq_rel_gpu();
+      fence_proxy_async_global();
+    }
+    __syncwarp();
   }
   compute_sync();
   if (*(volatile int*)&c.ctl->abort) c.ok = false;
   ++c.epoch;
-}
-
-// Cluster exchange among the compute warps: after it, every CTA of the
-// cluster may read what the others wrote to their shared memory before it.
-__device__ void cluster_exchange(Ctx& c, uint64_t* bar, uint32_t& count, uint32_t code) {
-  if (!c.ok) return;
-  compute_sync();
-  if (c.tid == 0) {
-    asm volatile("fence.acq_rel.cluster;" ::: "memory");
-    for (int r = 0; r < kClusterSize; ++r) mbar_arrive_cluster(smem_u32(bar), r);
-  }
-  if (!wait_cl(smem_u32(bar), count & 1, c.p->spin_budget, &c.ctl->abort)) fail(c, code);
-  ++count;
+  tmark(c, 0);
 }
 
 // ------------------------------------------------------------ producer warp
-__device__ void producer(const StepParams& p, uint8_t* ring, Ctrl* ctl, int cta, int cluster) {
+__device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* ctl, int cta, int cluster) {
   const uint64_t pol = policy_evict_first();
   uint32_t nch[4], bytes[4];
   for (int g = 0; g < 4; ++g) {
-    nch[g] = gemm_busy(p.g[g], cluster) ? (uint32_t)p.g[g].nchunk : 0u;
-    bytes[g] = p.g[g].chunk_bytes;
+    const int ng = p.g[g].ng[cluster];
+    nch[g] = ng > 0 ? (uint32_t)p.g[g].nchunk : 0u;
+    bytes[g] = (uint32_t)ng * 128u;
   }
   uint32_t st[kRingSlots], en[kRingSlots];
   uint32_t head = 0, tail = 0, pos = 0;
@@ -230,6 +238,8 @@ __device__ void producer(const StepParams& p, uint8_t* ring, Ctrl* ctl, int cta,
           const uint32_t slot = head % kRingSlots;
           st[slot] = at;
           en[slot] = at + sz;
+          if (p.tlog != nullptr && (int)head < p.tlog_chunks)
+            p.tlog[(size_t)cta * p.tlog_stride + p.tlog_chunk_off + p.tlog_chunks + head] = gtimer();
           mbar_arrive_expect_tx(smem_u32(&ctl->full[slot]), sz);
           bulk_g2s(smem_u32(ring + at), src, sz, smem_u32(&ctl->full[slot]), pol);
           src += sz;
@@ -248,13 +258,14 @@ __device__ void producer(const StepParams& p, uint8_t* ring, Ctrl* ctl, int cta,
 }
 
 // ------------------------------------------------------------ MMA warp
-__device__ void mma_issuer(const StepParams& p, uint8_t* ring, uint8_t* work, Ctrl* ctl,
+__device__ __noinline__ void mma_issuer(const StepParams& p, uint8_t* ring, uint8_t* work, Ctrl* ctl,
                            uint32_t tmem, int cluster) {
   uint32_t nch[4], bytes[4], idesc[4];
   for (int g = 0; g < 4; ++g) {
-    nch[g] = gemm_busy(p.g[g], cluster) ? (uint32_t)p.g[g].nchunk : 0u;
-    bytes[g] = p.g[g].chunk_bytes;
-    idesc[g] = idesc_bf16(kRows, p.g[g].Ng);
+    const int ng = p.g[g].ng[cluster];
+    nch[g] = ng > 0 ? (uint32_t)p.g[g].nchunk : 0u;
+    bytes[g] = (uint32_t)ng * 128u;
+    idesc[g] = idesc_bf16(kRows, ng > 0 ? ng : 16);
   }
   uint32_t it = 0, pos = 0, gemm_count = 0;
   bool good = true;
@@ -269,6 +280,10 @@ __device__ void mma_issuer(const StepParams& p, uint8_t* ring, uint8_t* work, Ct
           break;
         }
         tc_fence_after();
+        if (p.tlog != nullptr) {
+          const int idx = p.tlog_mma_off + 2 * (int)gemm_count;
+          if (idx < p.tlog_stride) p.tlog[(size_t)blockIdx.x * p.tlog_stride + idx] = gtimer();
+        }
         for (uint32_t c = 0; c < nch[g]; ++c, ++it) {
           const uint32_t at = ring_place(pos, bytes[g]);
           const uint32_t slot = it % kRingSlots;
@@ -277,6 +292,8 @@ __device__ void mma_issuer(const StepParams& p, uint8_t* ring, uint8_t* work, Ct
             good = false;
             break;
           }
+          if (p.tlog != nullptr && (int)it < p.tlog_chunks)
+            p.tlog[(size_t)blockIdx.x * p.tlog_stride + p.tlog_chunk_off + it] = gtimer();
           tc_fence_after();
 #pragma unroll
           for (int k16 = 0; k16 < 4; ++k16)
@@ -285,6 +302,10 @@ __device__ void mma_issuer(const StepParams& p, uint8_t* ring, uint8_t* work, Ct
           mma_commit(smem_u32(&ctl->empty[slot]));
         }
         if (!good) break;
+        if (p.tlog != nullptr) {
+          const int idx = p.tlog_mma_off + 2 * (int)gemm_count + 1;
+          if (idx < p.tlog_stride) p.tlog[(size_t)blockIdx.x * p.tlog_stride + idx] = gtimer();
+        }
         mma_commit(smem_u32(&ctl->mma_done));
         ++gemm_count;
       }
@@ -300,236 +321,289 @@ __device__ void mma_issuer(const StepParams& p, uint8_t* ring, uint8_t* work, Ct
 }
 
 // ------------------------------------------------------------ compute warps
-// Loads this CTA's K-slice of the activation operand of GEMM g.
-__device__ void load_act(Ctx& c, int g, const uint16_t* act) {
+__device__ __forceinline__ const float* mod_vec(const StepParams& p, int step, int l, int which) {
+  return p.mod + (size_t)step * p.n_mod + ((size_t)6 * l + which) * p.d;
+}
+
+constexpr int kMaxPairs = 4;    // owned column pairs per residual thread (checked by the planner)
+constexpr int kAuxBytes = 8 * 1024;   // end of the work region: per-thread epilogue operands
+
+// This CTA's share of one linear.
+struct GemmView {
+  int ng;        // channels of its n-group (0: idle cluster)
+  int KS, ks, grp;
+  int own;       // owned output columns
+  int ownp;      // row stride (floats) of the staging / receive blocks, multiple of 4
+  int nchunk;
+  int base;      // first owned packed channel (gate_up: first owned u column)
+  uint32_t recv_off;   // byte offset of the receive buffer in the work region
+};
+
+__device__ __forceinline__ GemmView gemm_view(const Ctx& c, int g) {
   const GemmPlan& gp = c.p->g[g];
+  GemmView v;
+  v.ng = gp.ng[c.cluster];
+  v.KS = gp.KS;
+  v.ks = c.rank % gp.KS;
+  v.grp = c.rank / gp.KS;
+  v.own = v.ng / gp.KS;
+  v.ownp = (v.own + 3) & ~3;
+  v.nchunk = gp.nchunk;
+  v.base = (g == G_GU) ? gp.ch_off[c.cluster] + v.grp * (v.ng / 2) + v.ks * (v.own / 2)
+                       : gp.ch_off[c.cluster] + v.grp * v.ng + v.ks * v.own;
+  const uint32_t a_bytes = (uint32_t)v.nchunk * 8192u;
+  const uint32_t s_bytes = (uint32_t)(v.KS * kRecvRows * v.ownp * 4);
+  v.recv_off = ((a_bytes > s_bytes ? a_bytes : s_bytes) + 15u) & ~15u;
+  return v;
+}
+
+// Starts GEMM g: arms the receive barrier for the partials the cluster will
+// push here and loads this CTA's K-slice of the activations.
+__device__ __noinline__ void gemm_begin(const Ctx& c, const GemmView& v, const uint16_t* act) {
   if (c.tid == 0) {
+    Ctrl* ctl = c.ctl;
+    mbar_arrive_expect_tx(smem_u32(&ctl->recv), (uint32_t)(v.KS * kRecvRows * v.ownp * 4));
     fence_proxy_async_smem();
-    const int ks = c.rank % gp.KS;
-    const uint32_t bytes = (uint32_t)gp.nchunk * 8192u;
     const uint64_t pol = policy_evict_last();
-    mbar_arrive_expect_tx(smem_u32(&c.ctl->act_full), bytes);
-    for (int i = 0; i < gp.nchunk; ++i)
-      bulk_g2s(smem_u32(c.work + i * 8192),
-               act + (size_t)(ks * gp.nchunk + i) * (kRows * 64), 8192,
-               smem_u32(&c.ctl->act_full), pol);
+    const uint32_t bar = smem_u32(&ctl->act_full);
+    const int nch = v.nchunk;
+    mbar_arrive_expect_tx(bar, (uint32_t)nch * 8192u);
+    const uint16_t* src = act + (size_t)(v.ks * nch) * (kRows * 64);
+    const uint32_t dst = smem_u32(c.work);
+#pragma unroll 1
+    for (int i = 0; i < nch; ++i) bulk_g2s(dst + i * 8192, src + (size_t)i * (kRows * 64), 8192, bar, pol);
   }
 }
 
-// Waits for the MMAs of GEMM g, copies rows 0..50 of the fp32 accumulator
-// to the staging area (row stride Ng floats) and opens the cluster exchange.
-__device__ void stage_partials(Ctx& c, int g) {
-  const GemmPlan& gp = c.p->g[g];
+// Waits for the MMAs, stages rows 0..50 of the fp32 partial sums as one
+// contiguous block per owner ([owner][row][ownp]) and sends block o to owner
+// o's receive slot `ks` with one bulk copy each.  Returns once this CTA's own
+// receive buffer is complete.
+__device__ __noinline__ void push_partials(Ctx& c, const GemmView& v) {
   if (!c.ok) return;
-  if (!wait_ab(smem_u32(&c.ctl->mma_done), c.gemm_count & 1, c.p->spin_budget, &c.ctl->abort)) {
+  Ctrl* const ctl = c.ctl;
+  const long long budget = c.p->spin_budget;
+  const int tid = c.tid;
+  if (!wait_ab(smem_u32(&ctl->mma_done), c.gemm_count & 1, budget, &ctl->abort)) {
     fail(c, E_MMA_DONE);
     return;
   }
   ++c.gemm_count;
   tc_fence_after();
+  tmark(c, 1);
+  const int ng = v.ng, own = v.own, ownp = v.ownp;
   const int sp = c.warp & 3;
   const int row = 16 * sp + c.lane;
-  const bool ok = c.lane < 16 && row <= kBiasRow;
+  const bool valid = c.lane < 16 && row < kRecvRows;
   const uint32_t tb = c.tmem + ((uint32_t)(32 * sp) << 16);
-  float* stg = reinterpret_cast<float*>(c.work);
+  float* const stg = reinterpret_cast<float*>(c.work);
 #pragma unroll 1
-  for (int cb = 0; cb < gp.Ng; cb += 16) {
-    float v[16];
-    tmem_ld16(tb + cb, v);
-    tmem_ld_wait();
-    if (ok) {
-      float4* dst = reinterpret_cast<float4*>(stg + (size_t)row * gp.Ng + cb);
+  for (int cb = 0; cb < ng; cb += 64) {
+    float x[4][16];
+    const int nb = min(4, (ng - cb) >> 4);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    for (int i = 0; i < 4; ++i)
+      if (i < nb) tmem_ld16(tb + cb + 16 * i, x[i]);
+    tmem_ld_wait();
+    if (valid) {
+      int o = cb / own, lc = cb - o * own;
+      float* rowp = stg + (o * kRecvRows + row) * ownp;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (i >= nb) break;
+#pragma unroll
+        for (int q = 0; q < 8; ++q) {
+          if (lc >= own) {
+            ++o;
+            lc -= own;
+            rowp += kRecvRows * ownp;
+          }
+          *reinterpret_cast<float2*>(rowp + lc) = make_float2(x[i][2 * q], x[i][2 * q + 1]);
+          lc += 2;
+        }
+      }
     }
   }
   tc_fence_before();
-  cluster_exchange(c, &c.ctl->xa, c.xa_count, E_XA);
-}
-
-// rstd[t] = (sum of per-cluster partial sums of h^2 / d + eps)^-1/2, rows < T.
-__device__ void load_rstd(Ctx& c, const float* sumsq) {
-  const StepParams& p = *c.p;
-  if (c.tid < p.T) {
-    float s = 0.f;
-    for (int q = 0; q < p.n_clusters; ++q) s += sumsq[q * kRows + c.tid];
-    c.ctl->rstd[c.tid] = 1.0f / sqrtf(s / (float)p.d + p.eps);
-  }
-  compute_sync();
-}
-
-// Writes the cluster's row sums of squares: rank 0 adds the 8 CTAs' partials.
-__device__ void publish_sumsq(Ctx& c, float* sumsq) {
-  cluster_exchange(c, &c.ctl->xb, c.xb_count, E_XB);
-  if (!c.ok) return;
-  if (c.rank == 0 && c.tid < c.p->T) {
-    const uint32_t a = smem_u32(&c.ctl->sq_own[c.tid]);
-    float s = 0.f;
-    for (int r = 0; r < kClusterSize; ++r) s += ld_dsmem_f1(map_shared_rank(a, r));
-    sumsq[c.cluster * kRows + c.tid] = s;
-  }
-}
-
-// Residual-column owner: h_new = h_old + gate * acc for 8 columns starting at
-// global column hc, row t; writes h_new, z = bf16(h_new (1 + s)) and returns
-// sum of squares.
-__device__ __forceinline__ float residual8(const float* h_old, float* h_new, uint16_t* z,
-                                           const float* gate, const float* sc, int d, int t, int hc,
-                                           const float (&acc)[8]) {
-  const float4* ho = reinterpret_cast<const float4*>(h_old + (size_t)t * d + hc);
-  const float4 h0 = ho[0], h1 = ho[1];
-  const float hv[8] = {h0.x, h0.y, h0.z, h0.w, h1.x, h1.y, h1.z, h1.w};
-  float out[8], zv[8], sq = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    out[i] = fmaf(gate[hc + i], acc[i], hv[i]);
-    sq = fmaf(out[i], out[i], sq);
-  }
-  float4* hn = reinterpret_cast<float4*>(h_new + (size_t)t * d + hc);
-  hn[0] = make_float4(out[0], out[1], out[2], out[3]);
-  hn[1] = make_float4(out[4], out[5], out[6], out[7]);
-  if (z != nullptr) {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) zv[i] = out[i] * (1.0f + sc[hc + i]);
-    *reinterpret_cast<uint4*>(act64_piece(z, t, hc)) = pack8_bf16(zv);
-  }
-  return sq;
-}
-
-__device__ __forceinline__ void write_shift_row(uint16_t* z, const float* shift, int hc) {
-  float v[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) v[i] = shift[hc + i];
-  *reinterpret_cast<uint4*>(act64_piece(z, kBiasRow, hc)) = pack8_bf16(v);
-}
-
-__device__ __forceinline__ const float* mod_vec(const StepParams& p, int step, int l, int which) {
-  return p.mod + (size_t)step * p.n_mod + ((size_t)6 * l + which) * p.d;
-}
-
-// In-proj: h = x W_in^T for the CTA's residual columns; z_a for layer0.
-__device__ void phase_inproj(Ctx& c, int step) {
-  const StepParams& p = *c.p;
-  // Same column ownership as the down projection: both write sumsq_a.
-  const GemmPlan& go = p.g[G_DOWN];
-  if (!c.ok) return;
-  const bool busy = gemm_busy(go, c.cluster);
-  if (busy) {
-    const int base = c.cluster * go.NS * go.Ng + (c.rank / go.KS) * go.Ng + (c.rank % go.KS) * go.own;
-    const float* s_a = mod_vec(p, step, p.layer0, 0);
-    const float* b_a = mod_vec(p, step, p.layer0, 1);
-    float sq = 0.f;
-    for (int q = 0; q < go.own; q += 8) {
-      const int hc = base + q;
-      if (hc >= p.d) break;
-      if (c.tid < p.T) {
-        float acc[8];
-        const float* xr = p.x + (size_t)c.tid * p.A;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint16_t* w = p.w_in + (size_t)(hc + i) * p.A;
-          float a = 0.f;
-          for (int k = 0; k < p.A; ++k) a = fmaf(xr[k], __uint_as_float((uint32_t)w[k] << 16), a);
-          acc[i] = a;
-        }
-        float* hr = p.h_a + (size_t)c.tid * p.d + hc;
-        float zv[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          hr[i] = acc[i];
-          sq = fmaf(acc[i], acc[i], sq);
-          zv[i] = acc[i] * (1.0f + s_a[hc + i]);
-        }
-        *reinterpret_cast<uint4*>(act64_piece(p.z_a, c.tid, hc)) = pack8_bf16(zv);
-      } else if (c.tid == kBiasRow) {
-        write_shift_row(p.z_a, b_a, hc);
-      }
-    }
-    if (c.tid < p.T) c.ctl->sq_own[c.tid] = sq;
-    publish_sumsq(c, p.sumsq_a);
-  }
-}
-
-// QKV: z_a K-slice x packed W_qkv -> cluster reduce -> rstd, shift row, RoPE
-// -> q buffer and the chunk rows of the KV cache.
-__device__ void phase_qkv(Ctx& c, int step, int l) {
-  const StepParams& p = *c.p;
-  const GemmPlan& gp = p.g[G_QKV];
-  if (!c.ok || !gemm_busy(gp, c.cluster)) return;
-  load_act(c, G_QKV, p.z_a);
-  load_rstd(c, p.sumsq_a);
-  stage_partials(c, G_QKV);
-  if (!c.ok) return;
-  const int ng = c.rank / gp.KS, ks = c.rank % gp.KS;
-  const int col0 = ks * gp.own;
-  const int npair = gp.own / 2;
-  const uint32_t stg = smem_u32(c.work);
-  const int qn = p.Hq * p.hd, kn = p.Hkv * p.hd;
-  const int half = p.hd / 2;
-  const int Nc = gp.NS * gp.Ng;
-  for (int item = c.tid; item < p.T * npair; item += kComputeWarps * 32) {
-    const int t = item / npair, pr = item % npair;
-    const int col = col0 + 2 * pr;
-    const int n = c.cluster * Nc + ng * gp.Ng + col;
-    if (n >= gp.N) continue;
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-    for (int r = 0; r < gp.KS; ++r) {
-      const int peer = ng * gp.KS + r;
-      const float2 va = ld_dsmem_f2(map_shared_rank(stg + 4u * (uint32_t)(t * gp.Ng + col), peer));
-      const float2 vb = ld_dsmem_f2(map_shared_rank(stg + 4u * (uint32_t)(kBiasRow * gp.Ng + col), peer));
-      a0 += va.x; a1 += va.y; b0 += vb.x; b1 += vb.y;
-    }
-    const float rs = c.ctl->rstd[t];
-    const float y0 = fmaf(rs, a0, b0), y1 = fmaf(rs, a1, b1);
-    if (n < qn + kn) {
-      const bool is_q = n < qn;
-      const int nn = is_q ? n : n - qn;
-      const int head = nn / p.hd, w = nn % p.hd, i = w >> 1;
-      const float cs = p.rope[(t * half + i) * 2], sn = p.rope[(t * half + i) * 2 + 1];
-      const float o1 = y0 * cs - y1 * sn;
-      const float o2 = y1 * cs + y0 * sn;
-      uint16_t* row;
-      int rr;
-      if (is_q) {
-        rr = t;
-        row = p.qbuf + ((size_t)head * kRows + t) * p.hd;
-      } else {
-        rr = c.P + t;
-        row = p.kcache + ((((size_t)l * p.B_cap + p.b) * p.Hkv + head) * p.S_max + rr) * p.hd;
-      }
-      row[swz(rr, i)] = bf16_bits(o1);
-      row[swz(rr, i + half)] = bf16_bits(o2);
-    } else {
-      const int nn = n - qn - kn;
-      const int head = nn / p.hd, w = nn % p.hd;
-      const int rr = c.P + t;
-      uint16_t* row = p.vcache + ((((size_t)l * p.B_cap + p.b) * p.Hkv + head) * p.S_max + rr) * p.hd;
-      row[swz(rr, w)] = bf16_bits(y0);
-      row[swz(rr, w + 1)] = bf16_bits(y1);
-    }
-  }
+  tmark(c, 6);
   fence_proxy_async_smem();
+  compute_sync();
+  tmark(c, 7);
+  const uint32_t recv_local = smem_u32(c.work + v.recv_off);
+  const uint32_t bar_local = smem_u32(&ctl->recv);
+  if (tid < v.KS) {
+    // one thread per owner issues that owner's copy
+    const uint32_t blk = (uint32_t)(kRecvRows * ownp * 4);
+    const uint32_t dst = (uint32_t)(v.grp * v.KS + tid);
+    bulk_s2cluster(map_shared_rank(recv_local + (uint32_t)v.ks * blk, dst), smem_u32(stg) + (uint32_t)tid * blk,
+                   blk, map_shared_rank(bar_local, dst));
+  }
+  tmark(c, 2);
+  if (!wait_ab(bar_local, c.recv_count & 1, budget, &ctl->abort)) {
+    fail(c, E_RECV);
+    return;
+  }
+  ++c.recv_count;
+  tmark(c, 3);
 }
 
-// GQA attention for the cluster's query head(s); this CTA takes one key range.
+// rstd[t] = (sum over CTAs of the partial sums of h^2 / d + eps)^-1/2.
+// Thread tid adds rows 4*(tid%16)..+3 of CTAs tid/16 + 8k (independent float4
+// loads, four per round); the eight groups are then added in a fixed order.
+__device__ __noinline__ void load_rstd(const Ctx& c, const float* sumsq) {
+  const int T = c.p->T, n = c.p->n_ctas, d = c.p->d;
+  const float eps = c.p->eps;
+  const int tid = c.tid;
+  Ctrl* const ctl = c.ctl;
+  const float4* src = reinterpret_cast<const float4*>(sumsq);
+  const int nf4 = n * (kRows / 4);
+  float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 1
+  for (int f = tid; f < nf4; f += 4 * 128) {
+    float4 x[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) x[j] = f + 128 * j < nf4 ? src[f + 128 * j] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      a.x += x[j].x; a.y += x[j].y; a.z += x[j].z; a.w += x[j].w;
+    }
+  }
+  *reinterpret_cast<float4*>(&ctl->red[tid >> 4][4 * (tid & 15)]) = a;
+  compute_sync();
+  if (tid < T) {
+    float s = 0.f;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) s += ctl->red[g][tid];
+    ctl->rstd[tid] = 1.0f / sqrtf(s / (float)d + eps);
+  }
+}
+
+// Sum over the KS senders of two adjacent received columns of row r.
+__device__ __forceinline__ float2 recv_sum2(const float* rb, int KS, int ownp, int r, int lc) {
+  float2 a = make_float2(0.f, 0.f);
+  const float* p0 = rb + r * ownp + lc;
+#pragma unroll 1
+  for (int s = 0; s < KS; s += 2) {
+    const float2 x = *reinterpret_cast<const float2*>(p0 + s * kRecvRows * ownp);
+    const float2 y = s + 1 < KS ? *reinterpret_cast<const float2*>(p0 + (s + 1) * kRecvRows * ownp)
+                                : make_float2(0.f, 0.f);
+    a.x += x.x;
+    a.y += x.y;
+    a.x += y.x;
+    a.y += y.y;
+  }
+  return a;
+}
+
+// Fixed item assignment of the epilogues: thread tid takes column pair
+// tid % npair for rows tid / npair + k * (128 / npair).
+struct PairRows {
+  int pr, t0, dt;
+  bool active;
+};
+__device__ __forceinline__ PairRows pair_rows(int tid, int npair) {
+  PairRows r;
+  const int per = 128 / npair;
+  r.pr = tid % npair;
+  r.t0 = tid / npair;
+  r.dt = per;
+  r.active = npair > 0 && tid < per * npair;
+  return r;
+}
+
+// QKV: reduce, rstd + shift row, RoPE -> q buffer and the chunk rows of the
+// KV cache.
+__device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
+  if (!c.ok) return;
+  const StepParams& p = *c.p;
+  const GemmView v = gemm_view(c, G_QKV);
+  if (v.ng == 0) return;
+  gemm_begin(c, v, p.z_a);
+  load_rstd(c, p.sumsq_a);
+  const int T = p.T, hd = p.hd, half = hd / 2, G = p.Hq / p.Hkv;
+  const int qn = p.Hq * hd, kn = p.Hkv * hd, N = p.g[G_QKV].N;
+  const int P = c.P;
+  const PairRows pa = pair_rows(c.tid, v.own / 2);
+  const int n = v.base + 2 * pa.pr;
+  const bool act = pa.active && n < N;
+  // destination of this thread's column pair: q (kind 0), k (1) or v (2)
+  const int kind = n < qn ? 0 : n < qn + kn ? 1 : 2;
+  const int nn = kind == 0 ? n : kind == 1 ? n - qn : n - qn - kn;
+  const int head = nn / hd, w = nn % hd, ri = w >> 1;
+  uint16_t* dst;
+  int row_off;    // row index of token 0
+  if (kind == 0) {
+    dst = p.qbuf + (size_t)(head / G) * p.q_rows * hd;
+    row_off = (head % G) * T;
+  } else {
+    dst = (kind == 1 ? p.kcache : p.vcache) + (((size_t)l * p.B_cap + p.b) * p.Hkv + head) * p.S_max * hd;
+    row_off = P;
+  }
+  // stage the rotation of every row of this thread
+  float2* aux = reinterpret_cast<float2*>(c.work + kWorkBytes - kAuxBytes) + c.tid;
+  if (act && kind < 2) {
+    const float2* rope = reinterpret_cast<const float2*>(p.rope) + ri;
+#pragma unroll 1
+    for (int t = pa.t0, k = 0; t < T; t += pa.dt, ++k) aux[k * 128] = rope[t * half];
+  }
+  push_partials(c, v);
+  if (!c.ok || !act) return;
+  const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
+  const float* rstd = c.ctl->rstd;
+  const float2 bsh = recv_sum2(rb, v.KS, v.ownp, kBiasRow, 2 * pa.pr);
+  tmark(c, 8);
+#pragma unroll 1
+  for (int t = pa.t0, k = 0; t < T; t += pa.dt, ++k) {
+    const float2 a = recv_sum2(rb, v.KS, v.ownp, t, 2 * pa.pr);
+    const float rs = rstd[t];
+    const float y0 = fmaf(rs, a.x, bsh.x), y1 = fmaf(rs, a.y, bsh.y);
+    const int rr = row_off + t;
+    uint16_t* rowp = dst + (size_t)rr * hd;
+    if (kind < 2) {
+      const float2 r = aux[k * 128];
+      rowp[swz(rr, ri)] = bf16_bits(y0 * r.x - y1 * r.y);
+      rowp[swz(rr, ri + half)] = bf16_bits(y1 * r.x + y0 * r.y);
+    } else {
+      *reinterpret_cast<uint32_t*>(rowp + swz(rr, w)) = pack_bf16(y0, y1);
+    }
+  }
+}
+
+// Attention for one (KV group, 64-row block of the group's G*T query rows);
+// this CTA takes one key range of [prefix ; chunk].
 template <int HD>
-__device__ void attention_head(Ctx& c, int l, int head) {
+__device__ __noinline__ void attention_unit(Ctx& c, int l, int grp, int blk) {
   const StepParams& p = *c.p;
   constexpr int KSTEPS = HD / 16;
   constexpr int DT = HD / 8;         // n-tiles of the output
+  constexpr int RWP = HD + 4;        // floats per pushed row: o, m, l, padding
   const int G = p.Hq / p.Hkv;
-  const int g = head / G;
-  const int S = c.P + p.T;
+  const int T = p.T;
+  const int S = c.P + T;
   const int kpc = ((S + kClusterSize * 16 - 1) / (kClusterSize * 16)) * 16;
-  const int k0 = c.rank * kpc;
+  const int rank = c.rank, tid = c.tid, lane = c.lane;
+  const int k0 = rank * kpc;
   const int k1 = min(S, k0 + kpc);
-  uint8_t* qs = c.work;
-  uint8_t* ks_ = c.work + kRows * HD * 2;
-  uint8_t* vs_ = ks_ + 64 * HD * 2;
+  const int row0 = blk * 64;                       // first query row of the block
+  const int nrows = min(64, G * T - row0);
+  const long long budget = p.spin_budget;
+  Ctrl* const ctl = c.ctl;
+  uint8_t* const qs = c.work;
+  uint8_t* const ks_ = c.work + 64 * HD * 2;
+  uint8_t* const vs_ = ks_ + 64 * HD * 2;
+  float* const rb = reinterpret_cast<float*>(vs_ + 64 * HD * 2);    // [8 senders][8 rows][RWP]
+  float* const stg = reinterpret_cast<float*>(c.work);              // [64 rows][RWP], after compute
   const uint32_t qa = smem_u32(qs), ka = smem_u32(ks_), va = smem_u32(vs_);
+  const uint32_t att_bar = smem_u32(&ctl->att);
   const uint64_t pol = policy_evict_last();
-  const uint16_t* kg = p.kcache + ((((size_t)l * p.B_cap + p.b) * p.Hkv + g) * p.S_max) * HD;
-  const uint16_t* vg = p.vcache + ((((size_t)l * p.B_cap + p.b) * p.Hkv + g) * p.S_max) * HD;
+  const size_t kvoff = ((((size_t)l * p.B_cap + p.b) * p.Hkv + grp) * p.S_max) * HD;
+  const uint16_t* kg = p.kcache + kvoff;
+  const uint16_t* vg = p.vcache + kvoff;
+  const uint16_t* qg = p.qbuf + ((size_t)grp * p.q_rows + row0) * HD;
+  if (tid == 0) {
+    // every CTA of the cluster sends 8 rows to each owner
+    mbar_arrive_expect_tx(smem_u32(&ctl->recv), (uint32_t)(kClusterSize * 8 * RWP * 4));
+  }
 
   const int w4 = c.warp - 2;               // rows 16*w4 .. +15
   const int r0 = 16 * w4;
@@ -538,67 +612,76 @@ __device__ void attention_head(Ctx& c, int l, int head) {
   float o[DT][4];
 #pragma unroll
   for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  uint32_t qf[KSTEPS][4];
+  // ldmatrix lane addresses (row-swizzled 16-byte pieces)
+  const int qrow = r0 + (lane & 15);
+  const uint32_t q_lane = qa + qrow * HD * 2;
+  const int q_sw = (row0 + qrow) & 7;
+  const int q_pc = lane >> 4;
+  const int kkey = (lane & 7) + ((lane >> 4) << 3);
+  const int k_pc = (lane >> 3) & 1;
+  const int vkey = (lane & 7) + (((lane >> 3) & 1) << 3);
+  const int v_pc = lane >> 4;
 
   bool first = true;
+#pragma unroll 1
   for (int kb = k0; kb < k1 || first; kb += 64) {
     const int nk = max(0, min(64, k1 - kb));
-    if (c.tid == 0) {
+    if (tid == 0) {
       fence_proxy_async_smem();
-      uint32_t bytes = 2u * (uint32_t)nk * HD * 2u + (first ? (uint32_t)(kRows * HD * 2) : 0u);
-      mbar_arrive_expect_tx(smem_u32(&c.ctl->att), bytes);
-      if (first)
-        bulk_g2s(qa, p.qbuf + (size_t)head * kRows * HD, kRows * HD * 2, smem_u32(&c.ctl->att), pol);
+      const uint32_t bytes = 2u * (uint32_t)nk * HD * 2u + (first ? (uint32_t)(nrows * HD * 2) : 0u);
+      mbar_arrive_expect_tx(att_bar, bytes);
+      if (first) bulk_g2s(qa, qg, (uint32_t)nrows * HD * 2, att_bar, pol);
       if (nk > 0) {
-        bulk_g2s(ka, kg + (size_t)kb * HD, (uint32_t)nk * HD * 2, smem_u32(&c.ctl->att), pol);
-        bulk_g2s(va, vg + (size_t)kb * HD, (uint32_t)nk * HD * 2, smem_u32(&c.ctl->att), pol);
+        bulk_g2s(ka, kg + (size_t)kb * HD, (uint32_t)nk * HD * 2, att_bar, pol);
+        bulk_g2s(va, vg + (size_t)kb * HD, (uint32_t)nk * HD * 2, att_bar, pol);
       }
     }
-    if (!wait_ab(smem_u32(&c.ctl->att), c.att_count & 1, p.spin_budget, &c.ctl->abort)) {
+    if (!wait_ab(att_bar, c.att_count & 1, budget, &ctl->abort)) {
       fail(c, E_ATT);
       return;
     }
     ++c.att_count;
     {
-      // Keys past nk in the last 16-key tile get zero V rows, so that their
-      // zero softmax weights cannot meet stale (possibly non-finite) data.
+      // Keys past nk in the last 16-key tile get zero V rows, and query rows
+      // past the block get zero q rows, so no stale (possibly non-finite)
+      // shared memory meets a zero weight.
       const int nk16 = (nk + 15) & ~15;
+      bool synced = false;
       if (nk16 > nk) {
         uint4* zr = reinterpret_cast<uint4*>(vs_ + (size_t)nk * HD * 2);
-        for (int i = c.tid; i < (nk16 - nk) * HD * 2 / 16; i += kComputeWarps * 32)
-          zr[i] = make_uint4(0u, 0u, 0u, 0u);
-        compute_sync();
+#pragma unroll 1
+        for (int i = tid; i < (nk16 - nk) * HD * 2 / 16; i += kComputeWarps * 32) zr[i] = make_uint4(0u, 0u, 0u, 0u);
+        synced = true;
       }
-    }
-    if (first) {
-#pragma unroll
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        const int row = r0 + (c.lane & 15);
-        const int pc = 2 * kk + (c.lane >> 4);
-        ldsm_x4(qa + row * HD * 2 + ((pc ^ (row & 7)) << 4), qf[kk][0], qf[kk][1], qf[kk][2],
-                qf[kk][3]);
+      if (first && nrows < 64) {
+        uint4* zq = reinterpret_cast<uint4*>(qs + (size_t)nrows * HD * 2);
+#pragma unroll 1
+        for (int i = tid; i < (64 - nrows) * HD * 2 / 16; i += kComputeWarps * 32) zq[i] = make_uint4(0u, 0u, 0u, 0u);
+        synced = true;
       }
-      first = false;
+      if (synced) compute_sync();
     }
+    first = false;
+    const int ksw = kb & 7;   // K/V rows are swizzled by their absolute row (kb is a multiple of 16)
+#pragma unroll 1
     for (int kt = 0; kt < nk; kt += 16) {
       float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-#pragma unroll
+      const uint32_t k_lane = ka + (kt + kkey) * HD * 2;
+      const int k_sw = (kt + kkey + ksw) & 7;
+#pragma unroll 2
       for (int kk = 0; kk < KSTEPS; ++kk) {
-        const int key = kt + (c.lane & 7) + ((c.lane >> 4) << 3);
-        const int pc = 2 * kk + ((c.lane >> 3) & 1);
-        const int gk = kb + key;   // absolute row decides the swizzle
-        uint32_t b0, b1, b2, b3;
-        ldsm_x4(ka + key * HD * 2 + ((pc ^ (gk & 7)) << 4), b0, b1, b2, b3);
-        mma16816(s[0], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b0, b1);
-        mma16816(s[1], qf[kk][0], qf[kk][1], qf[kk][2], qf[kk][3], b2, b3);
+        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
+        ldsm_x4(q_lane + (((2 * kk + q_pc) ^ q_sw) << 4), a0, a1, a2, a3);
+        ldsm_x4(k_lane + (((2 * kk + k_pc) ^ k_sw) << 4), b0, b1, b2, b3);
+        mma16816(s[0], a0, a1, a2, a3, b0, b1);
+        mma16816(s[1], a0, a1, a2, a3, b2, b3);
       }
-      // scale, mask, online softmax (rows lane/4 and lane/4 + 8)
       float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
       for (int t = 0; t < 2; ++t) {
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int key = kt + 8 * t + 2 * (c.lane & 3) + (e & 1);
+          const int key = kt + 8 * t + 2 * (lane & 3) + (e & 1);
           s[t][e] = key < nk ? s[t][e] * sl2 : -INFINITY;
           mx[e >> 1] = fmaxf(mx[e >> 1], s[t][e]);
         }
@@ -633,13 +716,12 @@ __device__ void attention_head(Ctx& c, int l, int head) {
       const uint32_t pa1 = pack_bf16(s[0][2], s[0][3]);
       const uint32_t pa2 = pack_bf16(s[1][0], s[1][1]);
       const uint32_t pa3 = pack_bf16(s[1][2], s[1][3]);
+      const uint32_t v_lane = va + (kt + vkey) * HD * 2;
+      const int v_sw = (kt + vkey + ksw) & 7;
 #pragma unroll
       for (int dp = 0; dp < DT / 2; ++dp) {
-        const int key = kt + (c.lane & 7) + (((c.lane >> 3) & 1) << 3);
-        const int pc = 2 * dp + (c.lane >> 4);
-        const int gk = kb + key;
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(va + key * HD * 2 + ((pc ^ (gk & 7)) << 4), b0, b1, b2, b3);
+        ldsm_x4_t(v_lane + (((2 * dp + v_pc) ^ v_sw) << 4), b0, b1, b2, b3);
         mma16816(o[2 * dp], pa0, pa1, pa2, pa3, b0, b1);
         mma16816(o[2 * dp + 1], pa0, pa1, pa2, pa3, b2, b3);
       }
@@ -652,238 +734,347 @@ __device__ void attention_head(Ctx& c, int l, int head) {
     l_r[h2] += __shfl_xor_sync(0xffffffffu, l_r[h2], 1);
     l_r[h2] += __shfl_xor_sync(0xffffffffu, l_r[h2], 2);
   }
-  // Partials to staging: [64 rows][HD + 4] fp32: o (unnormalised), m, l.
-  constexpr int RS = HD + 4;
-  float* stg = reinterpret_cast<float*>(c.work);
-  compute_sync();   // q tile is dead; staging overlaps it
-  {
-    const int ra = r0 + (c.lane >> 2), rb = ra + 8;
+  tmark(c, 1);
+  // Stage (o, m, l) of rows r and r + 8 (row r goes to owner r / 8), then one
+  // bulk copy per owner into its receive slot `rank`.
 #pragma unroll
-    for (int i = 0; i < DT; ++i) {
-      const int col = 8 * i + 2 * (c.lane & 3);
-      *reinterpret_cast<float2*>(stg + ra * RS + col) = make_float2(o[i][0], o[i][1]);
-      *reinterpret_cast<float2*>(stg + rb * RS + col) = make_float2(o[i][2], o[i][3]);
-    }
-    if ((c.lane & 3) == 0) {
-      stg[ra * RS + HD] = m_r[0];
-      stg[ra * RS + HD + 1] = l_r[0];
-      stg[rb * RS + HD] = m_r[1];
-      stg[rb * RS + HD + 1] = l_r[1];
-    }
+  for (int h2 = 0; h2 < 2; ++h2) {
+    const int r = r0 + (lane >> 2) + 8 * h2;
+    float* dst = stg + r * RWP + 2 * (lane & 3);
+#pragma unroll
+    for (int i = 0; i < DT; ++i) *reinterpret_cast<float2*>(dst + 8 * i) = make_float2(o[i][2 * h2], o[i][2 * h2 + 1]);
+    if ((lane & 3) == 0) *reinterpret_cast<float2*>(stg + r * RWP + HD) = make_float2(m_r[h2], l_r[h2]);
   }
-  cluster_exchange(c, &c.ctl->xa, c.xa_count, E_XA);
-  if (!c.ok) return;
-  // Combine: this CTA finalises rows 8*rank .. +7.
+  fence_proxy_async_smem();
+  compute_sync();
+  if (tid < kClusterSize) {
+    // one thread per owner issues that owner's copy
+    const uint32_t blk8 = 8u * RWP * 4u;
+    const uint32_t recv_local = smem_u32(rb), bar_local = smem_u32(&ctl->recv);
+    bulk_s2cluster(map_shared_rank(recv_local + (uint32_t)rank * blk8, tid), smem_u32(stg) + (uint32_t)tid * blk8,
+                   blk8, map_shared_rank(bar_local, tid));
+  }
+  tmark(c, 2);
+  if (!wait_ab(smem_u32(&ctl->recv), c.recv_count & 1, budget, &ctl->abort)) {
+    fail(c, E_RECV);
+    return;
+  }
+  ++c.recv_count;
+  tmark(c, 3);
+  // Combine the 8 key ranges for rows 8*rank .. +7 of the block.
   {
     constexpr int SEGS = HD / 8;
-    const int rloc = c.tid / 16, seg = c.tid % 16;
-    const int t = 8 * c.rank + rloc;
-    if (seg < SEGS && t < p.T) {
-      const uint32_t base = smem_u32(stg);
-      float mr[kClusterSize], lr[kClusterSize];
+    const int rloc = tid / 16, seg = tid % 16;
+    const int rblk = 8 * rank + rloc;
+    if (seg < SEGS && rblk < nrows) {
+      const float* src = rb + rloc * RWP;
       float M = -INFINITY;
-#pragma unroll
-      for (int r = 0; r < kClusterSize; ++r) {
-        const float2 ml = ld_dsmem_f2(map_shared_rank(base + 4u * (uint32_t)(t * RS + HD), r));
-        mr[r] = ml.x;
-        lr[r] = ml.y;
-        M = fmaxf(M, ml.x);
-      }
+#pragma unroll 1
+      for (int s = 0; s < kClusterSize; ++s) M = fmaxf(M, src[s * 8 * RWP + HD]);
       float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int r = 0; r < kClusterSize; ++r) {
-        if (lr[r] == 0.f) continue;
-        const float wgt = exp2f(mr[r] - M);
-        L = fmaf(lr[r], wgt, L);
-        const uint32_t a = map_shared_rank(base + 4u * (uint32_t)(t * RS + 8 * seg), r);
-        const float4 x0 = ld_dsmem_f4(a), x1 = ld_dsmem_f4(a + 16);
+#pragma unroll 1
+      for (int s = 0; s < kClusterSize; ++s) {
+        const float* sr = src + s * 8 * RWP;
+        const float ls = sr[HD + 1];
+        const float wgt = ls == 0.f ? 0.f : exp2f(sr[HD] - M);
+        L = fmaf(ls, wgt, L);
+        const float4 x0 = *reinterpret_cast<const float4*>(sr + 8 * seg);
+        const float4 x1 = *reinterpret_cast<const float4*>(sr + 8 * seg + 4);
         acc[0] = fmaf(x0.x, wgt, acc[0]); acc[1] = fmaf(x0.y, wgt, acc[1]);
         acc[2] = fmaf(x0.z, wgt, acc[2]); acc[3] = fmaf(x0.w, wgt, acc[3]);
         acc[4] = fmaf(x1.x, wgt, acc[4]); acc[5] = fmaf(x1.y, wgt, acc[5]);
         acc[6] = fmaf(x1.z, wgt, acc[6]); acc[7] = fmaf(x1.w, wgt, acc[7]);
       }
       const float inv = 1.0f / L;
+      const int R = row0 + rblk;
+      const int head = grp * G + R / T, t = R % T;
+      uint32_t pk[4];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] *= inv;
-      *reinterpret_cast<uint4*>(act64_piece(p.o_act, t, head * HD + 8 * seg)) = pack8_bf16(acc);
+      for (int i = 0; i < 4; ++i) pk[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
+      *reinterpret_cast<uint4*>(p.o_act + act64_off(t, head * HD + 8 * seg)) =
+          make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
-  fence_proxy_async_smem();
 }
 
-__device__ void phase_attn(Ctx& c, int l) {
+__device__ __noinline__ void phase_attn(Ctx& c, int l) {
   const StepParams& p = *c.p;
   if (!c.ok) return;
+  const int units = p.Hkv * p.att_blocks;
   bool more = false;
-  for (int head = c.cluster; head < p.Hq; head += p.n_clusters) {
+  for (int u = c.cluster; u < units; u += p.n_clusters) {
     if (more) {
-      // The staging area is reused: wait until every CTA finished reading it.
-      cluster_exchange(c, &c.ctl->xb, c.xb_count, E_XB);
-      if (!c.ok) return;
+      // A second unit on this cluster reuses shared memory: every CTA of the
+      // cluster must be done with the first one before anyone sends again.
+      fence_proxy_async_smem();
+      compute_sync();
+      if (c.tid == 0) {
+        asm volatile("fence.acq_rel.cluster;" ::: "memory");
+        for (int r = 0; r < kClusterSize; ++r) mbar_arrive_cluster(smem_u32(&c.ctl->xsync), r);
+      }
+      if (!wait_ab(smem_u32(&c.ctl->xsync), c.xs_count & 1, p.spin_budget, &c.ctl->abort)) {
+        fail(c, E_RECV);
+        return;
+      }
+      ++c.xs_count;
     }
-    if (p.hd == 128) attention_head<128>(c, l, head);
-    else attention_head<64>(c, l, head);
+    if (p.hd == 128) attention_unit<128>(c, l, u / p.att_blocks, u % p.att_blocks);
+    else attention_unit<64>(c, l, u / p.att_blocks, u % p.att_blocks);
     if (!c.ok) return;
     more = true;
   }
 }
 
-// o_proj / down: reduce the split-K partial sums of the CTA's 8-column
-// groups, apply the gated residual, emit z for the next linear and the row
-// sums of squares.
-__device__ void residual_epilogue(Ctx& c, int g, const float* h_old, float* h_new,
-                                  const float* gate, const float* sc, const float* shift,
-                                  uint16_t* z, float* sumsq) {
-  const StepParams& p = *c.p;
-  const GemmPlan& gp = p.g[g];
-  const int ng = c.rank / gp.KS, ks = c.rank % gp.KS;
-  const uint32_t stg = smem_u32(c.work);
-  const int Nc = gp.NS * gp.Ng;
+// o_proj / down: gated residual on the owned columns, two threads per row t
+// (each half of the owned column pairs); z for the next linear, row sum of
+// squares.  Operands of the epilogue are fetched before the MMAs finish.
+__device__ __noinline__ void residual_phase(Ctx& c, int g, const uint16_t* act, const float* h_old,
+                                            float* h_new, const float* gate, const float* sc,
+                                            const float* shift, uint16_t* z, float* sumsq) {
+  if (!c.ok) return;
+  const GemmView v = gemm_view(c, g);
+  if (v.ng == 0) return;
+  gemm_begin(c, v, act);
+  const int T = c.p->T, d = c.p->d;
+  const int tid = c.tid;
+  const int t = tid >> 1, hf = tid & 1;
+  const int npair = v.own / 2;
+  const int p0 = hf ? npair / 2 : 0, p1 = hf ? npair : npair / 2;
+  const int hc0 = v.base + 2 * p0;
+  const int np = min(p1 - p0, (d - hc0) / 2);
+  float2 ho[kMaxPairs], gt[kMaxPairs], sv[kMaxPairs];
+#pragma unroll
+  for (int k = 0; k < kMaxPairs; ++k) {
+    const int hc = hc0 + 2 * k;
+    ho[k] = gt[k] = sv[k] = make_float2(0.f, 0.f);
+    if (k < np) {
+      gt[k] = *reinterpret_cast<const float2*>(gate + hc);
+      if (t < T) ho[k] = *reinterpret_cast<const float2*>(h_old + (size_t)t * d + hc);
+      if (z != nullptr) sv[k] = *reinterpret_cast<const float2*>((t == kBiasRow ? shift : sc) + hc);
+    }
+  }
+  push_partials(c, v);
+  if (!c.ok) return;
+  const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
   float sq = 0.f;
-  for (int q = 0; q < gp.own; q += 8) {
-    const int col = ks * gp.own + q;
-    const int hc = c.cluster * Nc + ng * gp.Ng + col;
-    if (hc >= p.d) break;
-    if (c.tid < p.T) {
-      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-      for (int r = 0; r < gp.KS; ++r) {
-        const uint32_t a = map_shared_rank(stg + 4u * (uint32_t)(c.tid * gp.Ng + col), ng * gp.KS + r);
-        const float4 x0 = ld_dsmem_f4(a), x1 = ld_dsmem_f4(a + 16);
-        acc[0] += x0.x; acc[1] += x0.y; acc[2] += x0.z; acc[3] += x0.w;
-        acc[4] += x1.x; acc[5] += x1.y; acc[6] += x1.z; acc[7] += x1.w;
-      }
-      sq += residual8(h_old, h_new, z, gate, sc, p.d, c.tid, hc, acc);
-    } else if (c.tid == kBiasRow && z != nullptr) {
-      write_shift_row(z, shift, hc);
+#pragma unroll
+  for (int k = 0; k < kMaxPairs; ++k) {
+    if (k >= np) break;
+    const int hc = hc0 + 2 * k;
+    if (t < T) {
+      const float2 a = recv_sum2(rb, v.KS, v.ownp, t, 2 * (p0 + k));
+      const float n0 = fmaf(gt[k].x, a.x, ho[k].x), n1 = fmaf(gt[k].y, a.y, ho[k].y);
+      *reinterpret_cast<float2*>(h_new + (size_t)t * d + hc) = make_float2(n0, n1);
+      sq = fmaf(n0, n0, fmaf(n1, n1, sq));
+      if (z != nullptr)
+        *reinterpret_cast<uint32_t*>(z + act64_off(t, hc)) = pack_bf16(n0 * (1.0f + sv[k].x), n1 * (1.0f + sv[k].y));
+    } else if (t == kBiasRow && z != nullptr) {
+      *reinterpret_cast<uint32_t*>(z + act64_off(kBiasRow, hc)) = pack_bf16(sv[k].x, sv[k].y);
     }
   }
-  if (c.tid < p.T) c.ctl->sq_own[c.tid] = sq;
-  publish_sumsq(c, sumsq);
+  sq += __shfl_xor_sync(0xffffffffu, sq, 1);
+  if (hf == 0 && t < T) sumsq[c.cta * kRows + t] = sq;
 }
 
-__device__ void phase_o(Ctx& c, int step, int l) {
-  const StepParams& p = *c.p;
-  const GemmPlan& gp = p.g[G_O];
-  if (!c.ok || !gemm_busy(gp, c.cluster)) return;
-  load_act(c, G_O, p.o_act);
-  stage_partials(c, G_O);
+// gate_up: reduce, rstd + shift row, SwiGLU -> u (bf16, ACT64).  The owned
+// columns hold own/2 gate rows then own/2 matching up rows.
+__device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
   if (!c.ok) return;
-  residual_epilogue(c, G_O, p.h_a, p.h_b, mod_vec(p, step, l, 2), mod_vec(p, step, l, 3),
-                    mod_vec(p, step, l, 4), p.z_f, p.sumsq_f);
-  fence_proxy_async_smem();
-}
-
-__device__ void phase_down(Ctx& c, int step, int l) {
   const StepParams& p = *c.p;
-  const GemmPlan& gp = p.g[G_DOWN];
-  if (!c.ok || !gemm_busy(gp, c.cluster)) return;
-  load_act(c, G_DOWN, p.u_act);
-  stage_partials(c, G_DOWN);
-  if (!c.ok) return;
-  const bool next = l + 1 < p.L;
-  residual_epilogue(c, G_DOWN, p.h_b, p.h_a, mod_vec(p, step, l, 5),
-                    next ? mod_vec(p, step, l + 1, 0) : nullptr,
-                    next ? mod_vec(p, step, l + 1, 1) : nullptr, next ? p.z_a : nullptr,
-                    p.sumsq_a);
-  fence_proxy_async_smem();
-}
-
-// gate_up: reduce, rstd + shift row, SwiGLU -> u (bf16, ACT64).
-__device__ void phase_gu(Ctx& c, int step, int l) {
-  const StepParams& p = *c.p;
-  const GemmPlan& gp = p.g[G_GU];
-  if (!c.ok || !gemm_busy(gp, c.cluster)) return;
-  load_act(c, G_GU, p.z_f);
+  const GemmView v = gemm_view(c, G_GU);
+  if (v.ng == 0) return;
+  gemm_begin(c, v, p.z_f);
   load_rstd(c, p.sumsq_f);
-  stage_partials(c, G_GU);
+  push_partials(c, v);
   if (!c.ok) return;
-  const int ng = c.rank / gp.KS, ks = c.rank % gp.KS;
-  const int uown = gp.own / 2;                  // u columns owned
-  const int npiece = uown / 8;
-  const uint32_t stg = smem_u32(c.work);
-  const int ubase = (c.cluster * gp.NS + ng) * p.uc + ks * uown;
-  const int gcol0 = ks * gp.own;                // gate columns, then up columns
-  for (int item = c.tid; item < p.T * npiece; item += kComputeWarps * 32) {
-    const int t = item / npiece, q = item % npiece;
-    const int uc = ubase + 8 * q;
-    if (uc >= p.F) continue;
-    float ag[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, au[8], bg[8], bu[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) au[i] = bg[i] = bu[i] = 0.f;
-    for (int r = 0; r < gp.KS; ++r) {
-      const int peer = ng * gp.KS + r;
-      const uint32_t rg = map_shared_rank(stg + 4u * (uint32_t)(t * gp.Ng + gcol0 + 8 * q), peer);
-      const uint32_t ru = rg + 4u * (uint32_t)uown;
-      const uint32_t bgp = map_shared_rank(stg + 4u * (uint32_t)(kBiasRow * gp.Ng + gcol0 + 8 * q), peer);
-      const uint32_t bup = bgp + 4u * (uint32_t)uown;
-      float4 x;
-      x = ld_dsmem_f4(rg); ag[0] += x.x; ag[1] += x.y; ag[2] += x.z; ag[3] += x.w;
-      x = ld_dsmem_f4(rg + 16); ag[4] += x.x; ag[5] += x.y; ag[6] += x.z; ag[7] += x.w;
-      x = ld_dsmem_f4(ru); au[0] += x.x; au[1] += x.y; au[2] += x.z; au[3] += x.w;
-      x = ld_dsmem_f4(ru + 16); au[4] += x.x; au[5] += x.y; au[6] += x.z; au[7] += x.w;
-      x = ld_dsmem_f4(bgp); bg[0] += x.x; bg[1] += x.y; bg[2] += x.z; bg[3] += x.w;
-      x = ld_dsmem_f4(bgp + 16); bg[4] += x.x; bg[5] += x.y; bg[6] += x.z; bg[7] += x.w;
-      x = ld_dsmem_f4(bup); bu[0] += x.x; bu[1] += x.y; bu[2] += x.z; bu[3] += x.w;
-      x = ld_dsmem_f4(bup + 16); bu[4] += x.x; bu[5] += x.y; bu[6] += x.z; bu[7] += x.w;
-    }
-    const float rs = c.ctl->rstd[t];
-    float uv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float gt = fmaf(rs, ag[i], bg[i]);
-      const float up = fmaf(rs, au[i], bu[i]);
-      uv[i] = gt / (1.0f + expf(-gt)) * up;
-    }
-    *reinterpret_cast<uint4*>(act64_piece(p.u_act, t, uc)) = pack8_bf16(uv);
+  const int T = p.T, F = p.F;
+  const int uown = v.own / 2;
+  const PairRows pa = pair_rows(c.tid, uown / 2);
+  const int uc = v.base + 2 * pa.pr;
+  if (!pa.active || uc >= F) return;
+  const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
+  const float* rstd = c.ctl->rstd;
+  uint16_t* u_act = p.u_act;
+  const int lg = 2 * pa.pr, lu = uown + 2 * pa.pr;
+  const float2 bg = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lg);
+  const float2 bu = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lu);
+  tmark(c, 8);
+#pragma unroll 1
+  for (int t = pa.t0; t < T; t += pa.dt) {
+    const float2 ag = recv_sum2(rb, v.KS, v.ownp, t, lg);
+    const float2 au = recv_sum2(rb, v.KS, v.ownp, t, lu);
+    const float rs = rstd[t];
+    const float g0 = fmaf(rs, ag.x, bg.x), g1 = fmaf(rs, ag.y, bg.y);
+    const float u0 = fmaf(rs, au.x, bu.x), u1 = fmaf(rs, au.y, bu.y);
+    const float v0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+    const float v1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
+    *reinterpret_cast<uint32_t*>(u_act + act64_off(t, uc)) = pack_bf16(v0, v1);
   }
-  fence_proxy_async_smem();
 }
 
-// Final AdaRMSNorm (s_o, b_o) + out-proj + Euler, spread over every warp.
-__device__ void phase_outproj(Ctx& c, int step) {
-  const StepParams& p = *c.p;
+// In-proj: h = x W_in^T for the residual columns this CTA owns in the down
+// projection (same owners as sumsq_a); z_a for layer0.
+__device__ __noinline__ void phase_inproj(Ctx& c, int step) {
   if (!c.ok) return;
-  const float* s_o = p.mod + (size_t)step * p.n_mod + (size_t)6 * p.L * p.d;
-  const float* b_o = s_o + p.d;
-  const int nw = p.n_ctas * kComputeWarps;
+  const StepParams& p = *c.p;
+  const GemmView v = gemm_view(c, G_DOWN);
+  if (v.ng == 0) return;
+  const int T = p.T, A = p.A, d = p.d, own = v.own, base = v.base;
+  const int tid = c.tid;
+  float* xs = reinterpret_cast<float*>(c.work);            // [T][A]
+  float* ws = xs + T * A;                                   // [own][A]
+  float* sq = ws + own * A;                                 // [T][own/2]
+  {
+    const float2* x2 = reinterpret_cast<const float2*>(p.x);
+    const int n2 = T * A / 2;
+#pragma unroll 1
+    for (int i = tid; i < n2; i += 4 * 128) {
+      float2 xv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) xv[j] = i + 128 * j < n2 ? x2[i + 128 * j] : make_float2(0.f, 0.f);
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (i + 128 * j < n2) *reinterpret_cast<float2*>(xs + 2 * (i + 128 * j)) = xv[j];
+    }
+    const uint16_t* w = p.w_in + (size_t)base * A;
+    const int nw = min(own, d - base) * A;
+#pragma unroll 1
+    for (int i = tid; i < own * A; i += 4 * 128) {
+      uint16_t wv[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) wv[j] = i + 128 * j < nw ? w[i + 128 * j] : (uint16_t)0;
+#pragma unroll
+      for (int j = 0; j < 4; ++j)
+        if (i + 128 * j < own * A) ws[i + 128 * j] = __uint_as_float((uint32_t)wv[j] << 16);
+    }
+  }
+  tmark(c, 8);
+  compute_sync();
+  tmark(c, 9);
+  const float* s_a = mod_vec(p, step, p.layer0, 0);
+  const float* b_a = mod_vec(p, step, p.layer0, 1);
+  const int npair = own / 2;
+  const PairRows pa = pair_rows(tid, npair);
+  const int hc = base + 2 * pa.pr;
+  if (pa.active && hc < d) {
+    float* h_a = p.h_a;
+    uint16_t* z_a = p.z_a;
+    const float2 sa = *reinterpret_cast<const float2*>(s_a + hc);
+    const float* w0 = ws + (2 * pa.pr) * A;
+    const float* w1 = w0 + A;
+    if (pa.t0 == 0)
+      *reinterpret_cast<uint32_t*>(z_a + act64_off(kBiasRow, hc)) = pack_bf16(b_a[hc], b_a[hc + 1]);
+#pragma unroll 1
+    for (int t = pa.t0; t < T; t += pa.dt) {
+      const float* xr = xs + t * A;
+      float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
+      int k = 0;
+#pragma unroll 1
+      for (; k + 2 <= A; k += 2) {
+        a0 = fmaf(xr[k], w0[k], a0);
+        a1 = fmaf(xr[k], w1[k], a1);
+        c0 = fmaf(xr[k + 1], w0[k + 1], c0);
+        c1 = fmaf(xr[k + 1], w1[k + 1], c1);
+      }
+      if (k < A) {
+        a0 = fmaf(xr[k], w0[k], a0);
+        a1 = fmaf(xr[k], w1[k], a1);
+      }
+      a0 += c0;
+      a1 += c1;
+      *reinterpret_cast<float2*>(h_a + (size_t)t * d + hc) = make_float2(a0, a1);
+      *reinterpret_cast<uint32_t*>(z_a + act64_off(t, hc)) = pack_bf16(a0 * (1.0f + sa.x), a1 * (1.0f + sa.y));
+      sq[t * npair + pa.pr] = fmaf(a0, a0, a1 * a1);
+    }
+  } else if (pa.active) {
+#pragma unroll 1
+    for (int t = pa.t0; t < T; t += pa.dt) sq[t * npair + pa.pr] = 0.f;
+  }
+  tmark(c, 10);
+  compute_sync();
+  if (tid < T) {
+    float s = 0.f;
+#pragma unroll 1
+    for (int pr = 0; pr < npair; ++pr) s += sq[tid * npair + pr];
+    p.sumsq_a[c.cta * kRows + tid] = s;
+  }
+}
+
+// Final AdaRMSNorm (s_o, b_o) + out-proj + Euler: items (t, a) in order, a
+// contiguous range per warp; the warp keeps y(t) in registers and evaluates
+// up to 4 actions at a time.
+__device__ __noinline__ void phase_outproj(Ctx& c, int step) {
+  if (!c.ok) return;
+  const StepParams& p = *c.p;
+  const int T = p.T, A = p.A, d = p.d, n_ctas = p.n_ctas;
+  const int lane = c.lane;
+  const float eps = p.eps, dt = p.dt;
+  const float* s_o = p.mod + (size_t)step * p.n_mod + (size_t)6 * p.L * d;
+  const float* b_o = s_o + d;
+  const float* h_a = p.h_a;
+  const float* sumsq = p.sumsq_a;
+  const uint16_t* w_out = p.w_out;
+  const float* out_bias = p.out_bias;
+  float* vbuf = p.vbuf;
+  float* x = p.x;
+  const bool update = p.update_x != 0;
+  const int nw = n_ctas * kComputeWarps;
   const int gw = c.cta * kComputeWarps + (c.warp - 2);
-  const int total = p.T * p.A;
+  const int total = T * A;
   const int per = (total + nw - 1) / nw;
   const int i0 = gw * per, i1 = min(total, i0 + per);
   constexpr int MAXV = 32;   // d <= 1024
   float y[MAXV];
-  int cur_t = -1;
-  for (int it = i0; it < i1; ++it) {
-    const int t = it / p.A, a = it % p.A;
-    if (t != cur_t) {
+  int it = i0;
+#pragma unroll 1
+  while (it < i1) {
+    const int t = it / A;
+    const int iend = min(i1, (t + 1) * A);
+    {
       float s = 0.f;
-      for (int q = 0; q < p.n_clusters; ++q) s += p.sumsq_a[q * kRows + t];
-      const float rs = 1.0f / sqrtf(s / (float)p.d + p.eps);
+#pragma unroll 1
+      for (int q = lane; q < n_ctas; q += 32) s += sumsq[q * kRows + t];
+      for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
+      const float rs = 1.0f / sqrtf(s / (float)d + eps);
 #pragma unroll
       for (int i = 0; i < MAXV; ++i) {
-        const int k = c.lane + 32 * i;
-        y[i] = k < p.d ? fmaf(p.h_a[(size_t)t * p.d + k] * rs, 1.0f + s_o[k], b_o[k]) : 0.f;
+        const int k = lane + 32 * i;
+        y[i] = k < d ? fmaf(h_a[(size_t)t * d + k] * rs, 1.0f + s_o[k], b_o[k]) : 0.f;
       }
-      cur_t = t;
     }
-    float dot = 0.f;
-    const uint16_t* w = p.w_out + (size_t)a * p.d;
+    if (it == i0) tmark(c, 8);
+#pragma unroll 1
+    for (; it < iend; it += 2) {
+      float dot0 = 0.f, dot1 = 0.f;
+      const bool two = it + 1 < iend;
+      const uint16_t* w = w_out + (size_t)(it - t * A) * d;
 #pragma unroll
-    for (int i = 0; i < MAXV; ++i) {
-      const int k = c.lane + 32 * i;
-      if (k < p.d) dot = fmaf(y[i], __uint_as_float((uint32_t)w[k] << 16), dot);
+      for (int i = 0; i < MAXV; ++i) {
+        const int k = lane + 32 * i;
+        if (k < d) {
+          dot0 = fmaf(y[i], __uint_as_float((uint32_t)w[k] << 16), dot0);
+          if (two) dot1 = fmaf(y[i], __uint_as_float((uint32_t)w[k + d] << 16), dot1);
+        }
+      }
+      for (int o = 16; o; o >>= 1) {
+        dot0 += __shfl_xor_sync(0xffffffffu, dot0, o);
+        dot1 += __shfl_xor_sync(0xffffffffu, dot1, o);
+      }
+      if (lane < 2 && it + lane < iend) {
+        const int a = it + lane - t * A;
+        const float vv = (lane == 0 ? dot0 : dot1) + (out_bias ? out_bias[a] : 0.f);
+        vbuf[(size_t)t * A + a] = vv;
+        if (update) x[(size_t)t * A + a] = fmaf(dt, vv, x[(size_t)t * A + a]);
+      }
     }
-    for (int o = 16; o; o >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, o);
-    if (c.lane == 0) {
-      const float v = dot + (p.out_bias ? p.out_bias[a] : 0.f);
-      p.vbuf[(size_t)t * p.A + a] = v;
-      if (p.update_x) p.x[(size_t)t * p.A + a] = fmaf(p.dt, v, p.x[(size_t)t * p.A + a]);
-    }
+    it = iend;   // the 2-wide steps may overshoot the token boundary
+    tmark(c, 9);
   }
 }
 
 __device__ void compute_main(Ctx& c) {
   const StepParams& p = *c.p;
+  tmark(c, 0);
   for (int s = p.step0; s < p.step1 && c.ok; ++s) {
     if (p.do_inproj) {
       phase_inproj(c, s);
@@ -894,11 +1085,17 @@ __device__ void compute_main(Ctx& c) {
       grid_sync(c);
       phase_attn(c, l);
       grid_sync(c);
-      phase_o(c, s, l);
+      residual_phase(c, G_O, p.o_act, p.h_a, p.h_b, mod_vec(p, s, l, 2), mod_vec(p, s, l, 3),
+                     mod_vec(p, s, l, 4), p.z_f, p.sumsq_f);
       grid_sync(c);
       phase_gu(c, s, l);
       grid_sync(c);
-      phase_down(c, s, l);
+      {
+        const bool next = l + 1 < p.L;
+        residual_phase(c, G_DOWN, p.u_act, p.h_b, p.h_a, mod_vec(p, s, l, 5),
+                       next ? mod_vec(p, s, l + 1, 0) : nullptr, next ? mod_vec(p, s, l + 1, 1) : nullptr,
+                       next ? p.z_a : nullptr, p.sumsq_a);
+      }
       grid_sync(c);
     }
     if (p.do_outproj) {
@@ -927,10 +1124,10 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
     }
     mbar_init(smem_u32(&ctl->act_full), 1);
     mbar_init(smem_u32(&ctl->mma_done), 1);
-    mbar_init(smem_u32(&ctl->xa), kClusterSize);
-    mbar_init(smem_u32(&ctl->xb), kClusterSize);
+    mbar_init(smem_u32(&ctl->recv), 1);
     mbar_init(smem_u32(&ctl->att), 1);
     mbar_init(smem_u32(&ctl->drain), 1);
+    mbar_init(smem_u32(&ctl->xsync), kClusterSize);
     ctl->abort = 0;
     fence_mbar_init();
   }
@@ -941,7 +1138,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
   tc_fence_before();
   __syncthreads();
   // Every CTA of the cluster must have initialised its barriers before any
-  // remote arrive lands on them.
+  // remote store lands on them.
   cluster_sync_all();
   tc_fence_after();
   const uint32_t tmem = ctl->tmem_slot;
@@ -955,7 +1152,6 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
   } else {
     Ctx c;
     c.p = &p;
-    c.ring = ring;
     c.work = work;
     c.ctl = ctl;
     c.tmem = tmem;
@@ -965,7 +1161,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
     c.tid = threadIdx.x - 64;
     c.warp = warp;
     c.lane = lane;
-    c.gemm_count = c.xa_count = c.xb_count = c.att_count = 0;
+    c.gemm_count = c.recv_count = c.att_count = c.xs_count = 0;
     c.epoch = 0;
     c.P = *p.P_dev;
     c.ok = true;
@@ -974,7 +1170,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
   }
   tc_fence_before();
   __syncthreads();
-  // No CTA may leave while a peer can still read its shared memory.
+  // No CTA may leave while a peer can still store into its shared memory.
   cluster_sync_all();
   if (warp == 1) {
     tc_fence_after();

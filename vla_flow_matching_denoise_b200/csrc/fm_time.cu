@@ -28,34 +28,48 @@ constexpr uint32_t kTChunk = kTTile * 128;   // 16 KB: 128 rows x 64 bf16
 constexpr double kTwoPi = 6.283185307179586476925286766559;
 }  // namespace
 
-// One block per time step: e (fp64 -> fp32 in shared memory), then
-// h1[k, i] = SiLU(sum_j e_j W1[i, j]) for all i, stored bf16 in ACT64 row k.
+// Hidden rows of the time MLP: e_k (fp64 -> fp32) for every step in shared
+// memory, then one warp per hidden unit i: lanes split W1[i, :] (coalesced)
+// and h1[k, i] = SiLU(sum_j e_k[j] W1[i, j]) for all steps k, stored bf16 in
+// ACT64 row k.
 __global__ void time_embed_kernel(const __grid_constant__ TimeParams p) {
-  __shared__ float e[kTimeDim];
-  const int k = blockIdx.x;
-  const double t = 1.0 - (double)k / (double)p.n_steps;
+  extern __shared__ float e_dyn[];   // [n_steps][kTimeDim]
+  float (*e)[kTimeDim] = reinterpret_cast<float (*)[kTimeDim]>(e_dyn);
   const int half = kTimeDim / 2;
-  for (int j = threadIdx.x; j < half; j += blockDim.x) {
+  for (int idx = threadIdx.x; idx < p.n_steps * half; idx += blockDim.x) {
+    const int k = idx / half, j = idx % half;
+    const double t = 1.0 - (double)k / (double)p.n_steps;
     const double period = 4e-3 * pow(4.0 / 4e-3, (double)j / (double)(half - 1));
     const double ang = kTwoPi * t / period;
-    e[j] = (float)sin(ang);
-    e[j + half] = (float)cos(ang);
+    e[k][j] = (float)sin(ang);
+    e[k][j + half] = (float)cos(ang);
   }
   __syncthreads();
-  for (int i = threadIdx.x; i < p.d; i += blockDim.x) {
-    const uint16_t* w = p.w1 + (size_t)i * kTimeDim;
+  const int lane = threadIdx.x & 31;
+  const int i = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (i >= p.d) return;
+  // lane holds W1[i, 8*lane .. 8*lane+7]
+  const uint4 wv = *reinterpret_cast<const uint4*>(p.w1 + (size_t)i * kTimeDim + 8 * lane);
+  const uint32_t wr[4] = {wv.x, wv.y, wv.z, wv.w};
+  float w[8];
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    w[2 * q] = __uint_as_float(wr[q] << 16);
+    w[2 * q + 1] = __uint_as_float(wr[q] & 0xFFFF0000u);
+  }
+  const int kb = i >> 6, c = (i & 63) >> 3;
+  for (int k = 0; k < p.n_steps; ++k) {
     float acc = 0.f;
-#pragma unroll 8
-    for (int j = 0; j < kTimeDim; j += 2) {
-      const uint32_t pair = *reinterpret_cast<const uint32_t*>(w + j);
-      acc = fmaf(e[j], __uint_as_float(pair << 16), acc);
-      acc = fmaf(e[j + 1], __uint_as_float(pair & 0xFFFF0000u), acc);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) acc = fmaf(e[k][8 * lane + q], w[q], acc);
+#pragma unroll
+    for (int o = 16; o; o >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, o);
+    if (lane == 0) {
+      const float h = acc / (1.0f + expf(-acc));
+      uint16_t* row = p.h1_act + (size_t)kb * (kRows * 64) + (size_t)k * 64;
+      __nv_bfloat16 hb = __float2bfloat16_rn(h);
+      row[((c ^ (k & 7)) << 3) + (i & 7)] = *reinterpret_cast<uint16_t*>(&hb);
     }
-    const float h = acc / (1.0f + expf(-acc));
-    const int kb = i >> 6, c = (i & 63) >> 3;
-    uint16_t* row = p.h1_act + (size_t)kb * (kRows * 64) + (size_t)k * 64;
-    __nv_bfloat16 hb = __float2bfloat16_rn(h);
-    row[((c ^ (k & 7)) << 3) + (i & 7)] = *reinterpret_cast<uint16_t*>(&hb);
   }
 }
 
@@ -211,8 +225,11 @@ size_t time_gemm_smem_bytes(int d) {
 }
 
 cudaError_t launch_time(const TimeParams& p, int n_sms, cudaStream_t st) {
-  time_embed_kernel<<<p.n_steps, 256, 0, st>>>(p);
-  cudaError_t e = cudaGetLastError();
+  const size_t esmem = (size_t)p.n_steps * kTimeDim * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(time_embed_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)esmem);
+  if (e != cudaSuccess) return e;
+  time_embed_kernel<<<(p.d + 7) / 8, 256, esmem, st>>>(p);
+  e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t smem = time_gemm_smem_bytes(p.d);
   e = cudaFuncSetAttribute(time_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);

@@ -95,6 +95,9 @@ WORKLOADS: Dict[str, ExpertShape] = {
     "lingbot_fp8_p256_n10": ExpertShape(36, 1024, 16, 2, 128, 4096, 75, 256, 10, fp8=True),
     # 64 independent requests on one GPU.
     "lingbot_b64_p256_n10": ExpertShape(36, 1024, 16, 2, 128, 4096, 75, 256, 10, batch=64),
+    # Four layers of the LingBot-shaped expert: the profiling case (same layer
+    # shape, ~200 MB on the device, weights still larger than L2).
+    "lingbot_l4_p256_n10": ExpertShape(4, 1024, 16, 2, 128, 4096, 75, 256, 10),
 }
 
 
