@@ -208,12 +208,32 @@ fm_status fm_sync(fm_expert *h, void *stream);
 fm_status fm_get_geometry(const fm_expert *h, int *cluster_size, int *n_clusters,
                           int *n_ctas);
 
+/* The time-conditioning rows m_k (as fm_time_modulation) for callers that
+ * cannot allocate device memory: a control loop or runtime whose device memory
+ * is fixed and audited at start-up, or an embedder that gives the library
+ * only buffers it owns.  The pages have no counterpart of this entry point;
+ * it allocates nothing.
+ *   w1: device bf16 bits [d_model, 256]; w2: device bf16 bits [n_mod, d_model]
+ *   (row-major, as in fm_weights); m_out: device fp32 [steps, n_mod].
+ *   Limits: 1 <= steps <= 64, 64 <= d_model <= 1024 (a multiple of 64).  Larger
+ *   sizes return FM_ERR_INVALID_ARG and fm_last_error(NULL) says why.
+ * Its only intermediate, the bf16 hidden activations (64 x 1024 at most, 128
+ * KB), lives in a device array inside the library that every GPU using the
+ * library holds until the process exits.  The first call on a device looks up
+ * that array's address; make that first call before any stream capture.  All
+ * calls share the array and each overwrites the part it reads, so nothing
+ * depends on a previous call; calls that overlap on the GPU (two streams)
+ * race on it.  Stream-ordered; does not synchronise. */
+fm_status fm_time_modulation_noalloc(const uint16_t *w1, const uint16_t *w2, int d_model, int n_mod,
+                                     int steps, float *m_out, void *stream);
+
 /* Release the handle and every device buffer it owns; NULL is a no-op.
  * Returns the number of device bytes released. */
 size_t fm_expert_destroy(fm_expert *h);
 
 /* Text of the last error on this handle ("" if none); NULL handle: the last
- * error of a failed fm_expert_create on this thread. */
+ * error of a failed fm_expert_create or fm_time_modulation_noalloc on this
+ * thread. */
 const char *fm_last_error(const fm_expert *h);
 const char *fm_status_string(fm_status s);
 int fm_abi_version(void);

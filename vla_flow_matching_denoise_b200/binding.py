@@ -27,7 +27,7 @@ STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_NOT_READY", 3: "FM_ERR
 # Every symbol include/fm_expert.h declares.
 EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity", "fm_time_modulation",
            "fm_trace_bytes", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
-           "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases",
+           "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
            "fm_expert_destroy", "fm_last_error", "fm_status_string",
            "fm_abi_version")
 
@@ -85,6 +85,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_sync.argtypes = [vp, vp]
     lib.fm_profile_denoise.argtypes = [vp, ip, ip, ip, vp, vp]
     lib.fm_profile_phases.argtypes = [vp, ip, vp, ctypes.POINTER(sz), vp]
+    lib.fm_time_modulation_noalloc.argtypes = [vp, vp, ip, ip, ip, vp, vp]
     lib.fm_get_geometry.argtypes = [vp, ctypes.POINTER(ip), ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.fm_expert_destroy.argtypes = [vp]
     lib.fm_expert_destroy.restype = sz
@@ -95,7 +96,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_abi_version.restype = ip
     for name in ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity",
                  "fm_time_modulation", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
-                 "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases"):
+                 "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc"):
         getattr(lib, name).restype = ip
     _lib = lib
     return lib

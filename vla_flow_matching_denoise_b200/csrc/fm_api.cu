@@ -23,6 +23,11 @@ namespace {
 
 thread_local std::string g_create_error;
 
+}  // namespace
+
+void fm::set_thread_error(const char* msg) { g_create_error = msg; }
+
+namespace {
 
 struct DevBuf {
   void* p = nullptr;

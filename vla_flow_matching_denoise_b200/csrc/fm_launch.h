@@ -25,4 +25,7 @@ size_t step_smem_bytes();
 cudaError_t step_max_clusters(int* n_clusters);
 cudaError_t launch_step(const StepParams& p, cudaStream_t st);
 
+// Sets the text fm_last_error(NULL) returns on this thread.
+void set_thread_error(const char* msg);
+
 }  // namespace fm
