@@ -90,8 +90,8 @@ struct StepParams {
   uint16_t* qbuf;            // [H_kv][q_rows][hd]: row (h % G) * T + t of group h / G
   uint16_t* kcache;          // [L][B][H_kv][S_max][hd]
   uint16_t* vcache;
-  uint32_t* bar_count;       // grid barrier: one arrival word per CTA, 16-byte aligned,
-                             // zeroed before launch (word = barriers passed)
+  uint32_t* bar_count;       // grid barrier arrival counter, zeroed before launch
+                             // (counts CTA arrivals over all barriers of the launch)
   uint32_t* err;             // error word (non-zero: a bounded wait gave up)
   // schedule of this launch
   int step0, step1;          // modulation rows used

@@ -149,48 +149,28 @@ __device__ void fail(Ctx& c, uint32_t code) {
   c.ok = false;
 }
 
-// Grid barrier among the compute warps of every CTA.  Each CTA publishes the
-// number of barriers it has passed in its own word (a release store, no
-// contended atomic); warp 0 of the compute warps polls all words with vector
-// loads until every CTA has arrived.
+// Grid barrier among the compute warps of every CTA: one release add per CTA
+// on a shared arrival counter (cumulative: the CTA barrier before it orders
+// every compute thread's writes), then one thread polls it with acquire loads
+// until all CTAs of this barrier generation have arrived.
 __device__ void grid_sync(Ctx& c) {
   if (!c.ok) return;
   tmark(c, 4);
   fence_proxy_async_global();
   compute_sync();
-  const uint32_t target = c.epoch + 1;
-  uint32_t* flags = c.p->bar_count;
   if (c.tid == 0) {
-    // cumulative: the CTA barrier above orders every compute thread's writes
-    // before this release
-    fence_acq_rel_gpu();
-    st_release_u32(flags + c.cta, target);
+    const uint32_t target = (c.epoch + 1) * (uint32_t)c.p->n_ctas;
+    uint32_t* count = c.p->bar_count;
+    red_release_add(count, 1u);
     tmark(c, 5);
-  }
-  if (c.warp == 2) {
-    const int n4 = (c.p->n_ctas + 3) / 4;
     const long long t0 = clock64();
-    bool good = true;
-    for (;;) {
-      bool mine = true;
-      for (int i = c.lane; i < n4; i += 32) {
-        const uint4 f = ld_relaxed_v4(flags + 4 * i);
-        const int base = 4 * i, n = c.p->n_ctas;
-        mine = mine && f.x >= target && (base + 1 >= n || f.y >= target) && (base + 2 >= n || f.z >= target) &&
-               (base + 3 >= n || f.w >= target);
-      }
-      if (__all_sync(0xffffffffu, mine)) break;
+    while (ld_acquire_u32(count) < target) {
       if (*(volatile uint32_t*)c.p->err != 0u || clock64() - t0 > c.p->spin_budget) {
-        good = false;
+        fail(c, E_GRID);
         break;
       }
     }
-    if (c.lane == 0) {
-      if (!good) fail(c, E_GRID);
-      fence_acq_rel_gpu();
-      fence_proxy_async_global();
-    }
-    __syncwarp();
+    fence_proxy_async_global();
   }
   compute_sync();
   if (*(volatile int*)&c.ctl->abort) c.ok = false;
