@@ -329,7 +329,8 @@ def main():
                    "chunk": f"{shape.chunk_len}x{shape.action_dim}", "euler_steps": n,
                    "requests_per_gpu": B, "weights": "fp8-e4m3" if shape.fp8 else "bf16",
                    "parallelism": f"replicas x{ws}",
-                   "l2": "inputs larger than L2: 1.25 GB of weights stream per Euler step (L2 126 MB)"},
+                   "l2": f"inputs larger than L2: {loop_bytes(shape, 1, B) / 1e9:.3f} GB of weights and KV "
+                         "stream per Euler step (L2 126 MB)"},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_chunk": ms_e2e / args.steps,
                 "h2d_bytes_per_step": int(x0.nbytes), "d2h_bytes_per_step": int(x0.nbytes)},

@@ -59,9 +59,14 @@ struct fm_expert {
   uint16_t* w_in = nullptr;
   uint16_t* w_out = nullptr;
   float* out_bias = nullptr;
-  // fp8 copies kept for fm_get_fp8_weights
-  std::vector<uint8_t*> fp8_codes;   // [L*7]
-  std::vector<float*> fp8_scale;     // [L*7]
+  // E4M3 weights: row scales by packed channel (read by the kernel) and, for
+  // fm_get_fp8_weights, the packing tables and the scales in source-row order
+  float* wscale = nullptr;           // [L][sc_stride]
+  int sc_stride = 0;
+  int sc_off[4] = {0, 0, 0, 0};
+  std::vector<PackChunk> pack_jobs;
+  std::vector<int32_t> pack_rows;
+  std::vector<float> row_scale;      // [L][rows of QKV + O + GU + DOWN]
   // buffers
   float* mod = nullptr;
   uint16_t* h1_act = nullptr;
@@ -249,10 +254,19 @@ fm_status upload_rows(fm_expert* h, uint16_t* dst, const uint16_t* src, size_t e
   return FM_OK;
 }
 
+// Index of packed channel q of n-group grp of cluster cl in a layer's scale
+// table: the owners' columns in packing order (gate_up: 2 rows per u column).
+int packed_index(const fm_expert* h, int g, int cl, int grp, int q) {
+  const GemmPlan& gp = h->plan[g];
+  return (g == G_GU ? 2 * gp.ch_off[cl] : gp.ch_off[cl]) + grp * gp.ng[cl] + q;
+}
+
 fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   const fm_config& c = h->cfg;
   const int d = c.d_model, F = c.d_ff, qn = c.n_q_heads * c.head_dim,
             kn = c.n_kv_heads * c.head_dim;
+  const bool fp8 = c.wtype == FM_W_FP8_E4M3;
+  const uint64_t row_bytes = fp8 ? 64 : 128;   // one chunk row: 64 weights
   // Per-layer packing jobs (identical for every layer) and CTA spans.
   std::vector<PackChunk> jobs;
   std::vector<int32_t> rows;
@@ -275,14 +289,40 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
         pc.nrows = (uint16_t)ng;
         pc.mat = (uint8_t)g;
         pc.kb = (uint32_t)(ks * gp.nchunk + i);
+        pc.fp8 = fp8 ? 1 : 0;
         jobs.push_back(pc);
-        off += (uint64_t)ng * 128;
+        off += (uint64_t)ng * row_bytes;
       }
     }
   }
   span[h->n_ctas] = (uint32_t)off;
   h->layer_bytes = off;
   if (off > 0xFFFFFFFFull) return set_err(h, FM_ERR_UNSUPPORTED, "layer span too large");
+  // E4M3: packed-channel -> source-row map of each linear's scale table
+  const int mrows[4] = {qn + 2 * kn, d, 2 * F, d};
+  std::vector<int32_t> sc_src[4];
+  if (fp8) {
+    int at = 0;
+    for (int g = 0; g < 4; ++g) {
+      const GemmPlan& gp = h->plan[g];
+      int n = 0;
+      for (int cl = 0; cl < h->n_clusters; ++cl)
+        if (gp.ng[cl] > 0) n = std::max(n, packed_index(h, g, cl, gp.NS - 1, gp.ng[cl] - 1) + 1);
+      n = (n + 3) & ~3;
+      sc_src[g].assign(n, -1);
+      for (int cl = 0; cl < h->n_clusters; ++cl)
+        for (int grp = 0; grp < gp.NS; ++grp)
+          for (int q = 0; q < gp.ng[cl]; ++q) sc_src[g][packed_index(h, g, cl, grp, q)] = source_row(h, g, cl, grp, q);
+      h->sc_off[g] = at;
+      at += n;
+    }
+    h->sc_stride = at;
+    h->pack_jobs = jobs;
+    h->pack_rows = rows;
+    h->row_scale.assign((size_t)c.n_layers * (mrows[0] + mrows[1] + mrows[2] + mrows[3]), 0.f);
+    DALLOC(h->wscale, (size_t)c.n_layers * h->sc_stride * 4);
+  }
+  std::vector<float> sc_host(fp8 ? (size_t)c.n_layers * h->sc_stride : 0, 0.f);
 
   PackChunk* d_jobs = nullptr;
   int32_t* d_rows = nullptr;
@@ -292,7 +332,7 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   DALLOC(h->span_off, span.size() * 4);
   CK(cudaMemcpy(h->span_off, span.data(), span.size() * 4, cudaMemcpyHostToDevice));
   // temporary buffers (freed at the end)
-  void* tmp[6] = {};
+  void* tmp[8] = {};
   const size_t sz_qkv = (size_t)(qn + 2 * kn) * d, sz_o = (size_t)d * qn, sz_gu = (size_t)2 * F * d,
                sz_dn = (size_t)d * F;
   cudaError_t e = cudaSuccess;
@@ -301,7 +341,10 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   if (e == cudaSuccess) e = cudaMalloc(&tmp[2], sz_gu * 2);
   if (e == cudaSuccess) e = cudaMalloc(&tmp[3], sz_dn * 2);
   if (e == cudaSuccess) e = cudaMalloc(&tmp[4], jobs.size() * sizeof(PackChunk) + rows.size() * 4 + 64);
-  if (e == cudaSuccess) e = cudaMalloc(&tmp[5], 4 * sizeof(void*) + 4 * sizeof(int));
+  if (e == cudaSuccess) e = cudaMalloc(&tmp[5], 8 * sizeof(void*) + 4 * sizeof(int));
+  // E4M3: codes of the four linears and their row scales
+  if (e == cudaSuccess && fp8) e = cudaMalloc(&tmp[6], sz_qkv + sz_o + sz_gu + sz_dn);
+  if (e == cudaSuccess && fp8) e = cudaMalloc(&tmp[7], (size_t)(mrows[0] + mrows[1] + mrows[2] + mrows[3]) * 4);
   fm_status st = FM_OK;
   if (e != cudaSuccess) {
     st = set_err(h, FM_ERR_OOM, "packing buffers: %s", cudaGetErrorString(e));
@@ -309,13 +352,24 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
     d_jobs = static_cast<PackChunk*>(tmp[4]);
     d_rows = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(tmp[4]) + jobs.size() * sizeof(PackChunk));
     d_mats = static_cast<uint16_t**>(tmp[5]);
-    d_matk = reinterpret_cast<int*>(static_cast<uint8_t*>(tmp[5]) + 4 * sizeof(void*));
+    d_matk = reinterpret_cast<int*>(static_cast<uint8_t*>(tmp[5]) + 8 * sizeof(void*));
     uint16_t* mats[4] = {static_cast<uint16_t*>(tmp[0]), static_cast<uint16_t*>(tmp[1]),
                          static_cast<uint16_t*>(tmp[2]), static_cast<uint16_t*>(tmp[3])};
     const int matk[4] = {d, qn, d, F};
+    uint8_t* q8[4] = {};
+    float* rs[4] = {};
+    if (fp8) {
+      q8[0] = static_cast<uint8_t*>(tmp[6]);
+      q8[1] = q8[0] + sz_qkv;
+      q8[2] = q8[1] + sz_o;
+      q8[3] = q8[2] + sz_gu;
+      rs[0] = static_cast<float*>(tmp[7]);
+      for (int g = 1; g < 4; ++g) rs[g] = rs[g - 1] + mrows[g - 1];
+    }
     e = cudaMemcpy(d_jobs, jobs.data(), jobs.size() * sizeof(PackChunk), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(d_rows, rows.data(), rows.size() * 4, cudaMemcpyHostToDevice);
-    if (e == cudaSuccess) e = cudaMemcpy(d_mats, mats, sizeof(mats), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && fp8) e = cudaMemcpy(d_mats, q8, sizeof(q8), cudaMemcpyHostToDevice);
+    else if (e == cudaSuccess) e = cudaMemcpy(d_mats, mats, sizeof(mats), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(d_matk, matk, sizeof(matk), cudaMemcpyHostToDevice);
     if (e != cudaSuccess) st = set_err(h, FM_ERR_CUDA, "pack tables: %s", cudaGetErrorString(e));
     for (int l = 0; l < c.n_layers && st == FM_OK; ++l) {
@@ -331,10 +385,33 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
       if (e == cudaSuccess) e = cudaMemcpy(mats[2], lw.w_gate, (size_t)F * d * 2, cudaMemcpyDefault);
       if (e == cudaSuccess) e = cudaMemcpy(mats[2] + (size_t)F * d, lw.w_up, (size_t)F * d * 2, cudaMemcpyDefault);
       if (e == cudaSuccess) e = cudaMemcpy(mats[3], lw.w_down, sz_dn * 2, cudaMemcpyDefault);
-      if (e == cudaSuccess)
+      if (fp8) {
+        // R8: per-row absmax / 448 and E4M3 codes of every linear, then the
+        // codes go into the arena and the scales into the packed-order table
+        for (int g = 0; g < 4 && e == cudaSuccess; ++g) e = launch_fp8_quantize(mats[g], mrows[g], matk[g], rs[g], q8[g], 0);
+        if (e == cudaSuccess)
+          e = launch_pack8(d_jobs, (int)jobs.size(), d_rows, reinterpret_cast<const uint8_t* const*>(d_mats), d_matk,
+                           h->arena + (size_t)l * off, 0);
+        float* lrs = h->row_scale.data() + (size_t)l * (mrows[0] + mrows[1] + mrows[2] + mrows[3]);
+        if (e == cudaSuccess)
+          e = cudaMemcpy(lrs, rs[0], (size_t)(mrows[0] + mrows[1] + mrows[2] + mrows[3]) * 4, cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess) {
+          const float* src = lrs;
+          for (int g = 0; g < 4; ++g) {
+            float* dst = sc_host.data() + (size_t)l * h->sc_stride + h->sc_off[g];
+            for (size_t i = 0; i < sc_src[g].size(); ++i) dst[i] = sc_src[g][i] >= 0 ? src[sc_src[g][i]] : 0.f;
+            src += mrows[g];
+          }
+        }
+      } else if (e == cudaSuccess) {
         e = launch_pack(d_jobs, (int)jobs.size(), d_rows, d_mats, d_matk, h->arena + (size_t)l * off, 0);
+      }
       if (e == cudaSuccess) e = cudaDeviceSynchronize();
       if (e != cudaSuccess) st = set_err(h, FM_ERR_CUDA, "packing layer %d: %s", l, cudaGetErrorString(e));
+    }
+    if (st == FM_OK && fp8) {
+      e = cudaMemcpy(h->wscale, sc_host.data(), sc_host.size() * 4, cudaMemcpyHostToDevice);
+      if (e != cudaSuccess) st = set_err(h, FM_ERR_CUDA, "scale table: %s", cudaGetErrorString(e));
     }
   }
   for (void* p : tmp)
@@ -499,6 +576,10 @@ StepParams base_params(const fm_expert* h) {
   p.vcache = h->vcache;
   p.bar_count = h->bar_count;
   p.err = h->err_word;
+  p.fp8 = c.wtype == FM_W_FP8_E4M3 ? 1 : 0;
+  p.wscale = h->wscale;
+  p.sc_stride = h->sc_stride;
+  for (int g = 0; g < 4; ++g) p.sc_off[g] = h->sc_off[g];
   p.step0 = 0;
   p.step1 = 0;
   p.layer0 = 0;
@@ -634,10 +715,6 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
   h->n_clusters = std::min(std::min(ncl, h->n_sms / kClusterSize), kMaxClusters);
   h->n_ctas = h->n_clusters * kClusterSize;
   if ((st = build_plan(h)) != FM_OK) return bail(st);
-  if (cfg->wtype == FM_W_FP8_E4M3) {
-    set_err(h, FM_ERR_UNSUPPORTED, "FP8 weights are not available in this build yet");
-    return bail(FM_ERR_UNSUPPORTED);
-  }
   if (cudaStreamCreateWithFlags(&h->cap_stream, cudaStreamNonBlocking) != cudaSuccess) {
     set_err(h, FM_ERR_CUDA, "stream creation failed");
     return bail(FM_ERR_CUDA);
@@ -945,9 +1022,35 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
 
 fm_status fm_get_fp8_weights(fm_expert* h, int layer, int which, uint8_t* codes, float* scale) {
   if (!h) return FM_ERR_INVALID_ARG;
-  if (h->cfg.wtype != FM_W_FP8_E4M3) return set_err(h, FM_ERR_INVALID_ARG, "handle holds bf16 weights");
-  (void)layer; (void)which; (void)codes; (void)scale;
-  return set_err(h, FM_ERR_UNSUPPORTED, "not available");
+  const fm_config& c = h->cfg;
+  if (c.wtype != FM_W_FP8_E4M3) return set_err(h, FM_ERR_INVALID_ARG, "handle holds bf16 weights");
+  if (layer < 0 || layer >= c.n_layers || which < 0 || which > 6 || !codes || !scale)
+    return set_err(h, FM_ERR_INVALID_ARG, "layer %d / which %d invalid or NULL buffer", layer, which);
+  const int d = c.d_model, F = c.d_ff, qn = c.n_q_heads * c.head_dim, kn = c.n_kv_heads * c.head_dim;
+  // linear `which` = rows [r0, r0 + rows) of packed matrix g (K columns)
+  static const int kG[7] = {G_QKV, G_QKV, G_QKV, G_O, G_GU, G_GU, G_DOWN};
+  const int g = kG[which];
+  const int r0s[7] = {0, qn, qn + kn, 0, 0, F, 0};
+  const int nrows[7] = {qn, kn, kn, d, F, F, d};
+  const int kdim[4] = {d, qn, d, F};
+  const int mrows[4] = {qn + 2 * kn, d, 2 * F, d};
+  const int r0 = r0s[which], R = nrows[which], K = kdim[g];
+  CK(cudaSetDevice(h->device));
+  std::vector<uint8_t> lay(h->layer_bytes);
+  CK(cudaMemcpy(lay.data(), h->arena + (size_t)layer * h->layer_bytes, h->layer_bytes, cudaMemcpyDeviceToHost));
+  std::memset(codes, 0, (size_t)R * K);
+  for (const PackChunk& pc : h->pack_jobs) {
+    if (pc.mat != g) continue;
+    for (int q = 0; q < pc.nrows; ++q) {
+      const int sr = h->pack_rows[pc.rowidx_off + q];
+      if (sr < r0 || sr >= r0 + R) continue;
+      std::memcpy(codes + (size_t)(sr - r0) * K + (size_t)pc.kb * 64, lay.data() + pc.dst_off + (size_t)q * 64, 64);
+    }
+  }
+  size_t base = (size_t)layer * (mrows[0] + mrows[1] + mrows[2] + mrows[3]);
+  for (int i = 0; i < g; ++i) base += mrows[i];
+  std::memcpy(scale, h->row_scale.data() + base + r0, (size_t)R * 4);
+  return FM_OK;
 }
 
 fm_status fm_profile_denoise(fm_expert* h, int batch, int steps, int iters, float* ms, void* stream) {

@@ -10,6 +10,10 @@
 //  * Packed weights: the same image with rows = output channels: a "chunk" is
 //    R rows x 64 input columns (R * 128 bytes).  The engine lays every CTA's
 //    chunks of one layer out contiguously, in the order the CTA consumes them.
+//    With E4M3 weights a chunk is R rows x 64 one-byte codes, plain row-major
+//    (R * 64 bytes); the kernel widens it to the bf16 image in shared memory.
+//    The per-output-row scales of a layer sit in a table indexed by packed
+//    channel (see StepParams::wscale).
 //  * KV cache: [L][B][H_kv][S_max][hd] bf16, each 256-byte row (hd = 128)
 //    split in 16-byte pieces stored at piece (c ^ (row & 7)); rows 0..P-1 are
 //    the prefix, rows P..P+T-1 the chunk of the current velocity evaluation.
@@ -24,6 +28,8 @@ constexpr int kClusterSize = 8;        // CTAs per cluster (portable maximum)
 constexpr int kMaxClusters = 24;       // 8-CTA clusters a B200 can hold (148 SMs)
 constexpr int kComputeWarps = 4;       // warps 2..5
 constexpr int kThreads = 192;          // producer warp, MMA warp, 4 compute warps
+constexpr int kConvWarps = 2;          // E4M3 -> bf16 widening warps of the step kernel
+constexpr int kStepThreads = kThreads + 32 * kConvWarps;
 constexpr int kRows = 64;              // MMA M: token rows per tile
 constexpr int kMaxT = 50;              // valid token rows (one chunk)
 constexpr int kBiasRow = 50;           // row carrying the AdaRMSNorm shift vector
@@ -66,8 +72,12 @@ struct StepParams {
   int att_blocks;            // 64-row blocks per KV group
   int q_rows;                // padded rows per KV group in the q buffer (multiple of 64)
   // weights
-  const uint8_t* arena;      // packed per-layer weights
+  const uint8_t* arena;      // packed per-layer weights (bf16 image or E4M3 codes)
   uint64_t layer_bytes;      // bytes of one layer in the arena
+  int fp8;                   // 1: the arena holds E4M3 codes, widened in shared memory
+  const float* wscale;       // fp8: [L][sc_stride] fp32 row scales by packed channel; else null
+  int sc_stride;             // floats per layer in wscale
+  int sc_off[4];             // first entry of each linear inside a layer's table
   const uint32_t* span_off;  // [n_ctas + 1]: byte offset of each CTA's span in a layer
   const uint16_t* w_in;      // [d, A] bf16
   const uint16_t* w_out;     // [A, d] bf16

@@ -11,6 +11,8 @@ namespace fm {
 cudaError_t launch_pack(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
                         const uint16_t* const* mats, const int* mat_k, uint8_t* dst,
                         cudaStream_t st);
+cudaError_t launch_pack8(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
+                         const uint8_t* const* mats, const int* mat_k, uint8_t* dst, cudaStream_t st);
 cudaError_t launch_fp8_quantize(const uint16_t* w, int rows, int K, float* scale, uint8_t* q,
                                 cudaStream_t st);
 cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, int Hkv, int hd, int S_max,

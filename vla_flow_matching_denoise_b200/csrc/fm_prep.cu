@@ -29,6 +29,24 @@ __global__ void pack_kernel(const PackChunk* __restrict__ chunks, const int32_t*
   }
 }
 
+// Copies 16-byte pieces of E4M3 code rows (one byte per weight) into a chunk
+// of R rows x 64 codes, row-major, unswizzled.
+__global__ void pack8_kernel(const PackChunk* __restrict__ chunks, const int32_t* __restrict__ rowidx,
+                             const uint8_t* const* __restrict__ mats, const int* __restrict__ mat_k,
+                             uint8_t* __restrict__ dst) {
+  const PackChunk ch = chunks[blockIdx.x];
+  const uint8_t* src = mats[ch.mat];
+  const int K = mat_k[ch.mat];
+  const int pieces = ch.nrows * 4;
+  for (int p = threadIdx.x; p < pieces; p += blockDim.x) {
+    const int row = p >> 2, c = p & 3;
+    const int sr = rowidx[ch.rowidx_off + row];
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (sr >= 0) v = *reinterpret_cast<const uint4*>(src + (size_t)sr * K + (size_t)ch.kb * 64 + c * 16);
+    *reinterpret_cast<uint4*>(dst + ch.dst_off + (size_t)row * 64 + c * 16) = v;
+  }
+}
+
 // Per-row absmax / 448 of a bf16 matrix [rows, K] (R8: s = absmax / 448, 1 for
 // an all-zero row).  One warp per row.
 __global__ void fp8_row_scale_kernel(const uint16_t* __restrict__ w, int rows, int K,
@@ -93,6 +111,13 @@ cudaError_t launch_pack(const PackChunk* chunks, int nchunks, const int32_t* row
                         cudaStream_t st) {
   if (nchunks == 0) return cudaSuccess;
   pack_kernel<<<nchunks, 256, 0, st>>>(chunks, rowidx, mats, mat_k, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack8(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
+                         const uint8_t* const* mats, const int* mat_k, uint8_t* dst, cudaStream_t st) {
+  if (nchunks == 0) return cudaSuccess;
+  pack8_kernel<<<nchunks, 256, 0, st>>>(chunks, rowidx, mats, mat_k, dst);
   return cudaGetLastError();
 }
 

@@ -32,6 +32,12 @@
 //    rows of that group's heads) on one cluster, keys split over its 8 CTAs,
 //    mma.sync with an online softmax, partials pushed to the row owners for
 //    the log-sum-exp combine.
+//  * E4M3 weights ("LingBot-VLA on Thor (sm_110)", §2: FP8 weight path):
+//    the ring receives one-byte codes in the upper half of each chunk's slot;
+//    two extra warps widen them in place to the bf16 image (exact: every E4M3
+//    value is a bf16 value), so the tensor cores still run bf16 x bf16 with
+//    bf16 activations.  The per-output-row scale multiplies the reduced fp32
+//    sum in the epilogue.
 #include <cuda_bf16.h>
 #include <cstddef>
 #include <cstdint>
@@ -47,6 +53,7 @@ namespace {
 struct Ctrl {
   uint64_t full[kRingSlots];
   uint64_t empty[kRingSlots];
+  uint64_t conv[kRingSlots];   // E4M3 weights: chunk widened to bf16
   uint64_t act_full;
   uint64_t mma_done;
   uint64_t recv;      // split-K / attention partials pushed by the cluster
@@ -71,6 +78,7 @@ enum : uint32_t {
   E_RECV = 1u << 3,
   E_MMA_DONE = 1u << 4,
   E_ATT = 1u << 7,
+  E_CONV = 1u << 8,
 };
 
 __device__ __forceinline__ bool wait_ab(uint32_t bar, uint32_t parity, long long budget,
@@ -187,6 +195,9 @@ __device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* 
     nch[g] = ng > 0 ? (uint32_t)p.g[g].nchunk : 0u;
     bytes[g] = (uint32_t)ng * 128u;
   }
+  // E4M3: a chunk's codes (half its bf16 size) land in the upper half of its
+  // slot and are widened in place
+  const uint32_t shift = p.fp8 ? 1u : 0u;
   uint32_t st[kRingSlots], en[kRingSlots];
   uint32_t head = 0, tail = 0, pos = 0;
   const uint32_t span0 = p.span_off[cta];
@@ -220,9 +231,10 @@ __device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* 
           en[slot] = at + sz;
           if (p.tlog != nullptr && (int)head < p.tlog_chunks)
             p.tlog[(size_t)cta * p.tlog_stride + p.tlog_chunk_off + p.tlog_chunks + head] = gtimer();
-          mbar_arrive_expect_tx(smem_u32(&ctl->full[slot]), sz);
-          bulk_g2s(smem_u32(ring + at), src, sz, smem_u32(&ctl->full[slot]), pol);
-          src += sz;
+          const uint32_t csz = sz >> shift;
+          mbar_arrive_expect_tx(smem_u32(&ctl->full[slot]), csz);
+          bulk_g2s(smem_u32(ring + at + (sz - csz)), src, csz, smem_u32(&ctl->full[slot]), pol);
+          src += csz;
           ++head;
         }
       }
@@ -235,6 +247,71 @@ __device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* 
   // Every issued copy must land before the CTA exits.
   for (uint32_t q = tail; q < head; ++q)
     mbar_wait(smem_u32(&ctl->full[q % kRingSlots]), (q / kRingSlots) & 1, p.spin_budget);
+}
+
+// ------------------------------------------------------------ widening warps
+// E4M3 -> bf16, in place: chunk rows of 64 codes sit in the upper half of the
+// slot; row r becomes the 128-byte swizzled bf16 row r.  Every thread loads
+// all of its pieces before any thread stores (named barrier), so no store can
+// overwrite codes not yet read.  ctid: 0 .. 32 * kConvWarps - 1.
+__device__ __noinline__ void converter(const StepParams& p, uint8_t* ring, Ctrl* ctl, int cluster, int ctid) {
+  constexpr int kCT = 32 * kConvWarps;
+  constexpr int kMaxPieces = 256 * 4 / kCT;   // 16-byte code pieces per thread (ng <= 256)
+  uint32_t nch[4], bytes[4];
+  for (int g = 0; g < 4; ++g) {
+    const int ng = p.g[g].ng[cluster];
+    nch[g] = ng > 0 ? (uint32_t)p.g[g].nchunk : 0u;
+    bytes[g] = (uint32_t)ng * 128u;
+  }
+  uint32_t it = 0, pos = 0;
+  bool good = true;
+  for (int s = p.step0; s < p.step1 && good; ++s) {
+    for (int l = p.layer0; l < p.layer1 && good; ++l) {
+      for (int g = 0; g < 4 && good; ++g) {
+        const int npieces = (int)(bytes[g] >> 5);   // ng rows x 4 pieces
+        for (uint32_t c = 0; c < nch[g]; ++c, ++it) {
+          const uint32_t at = ring_place(pos, bytes[g]);
+          const uint32_t slot = it % kRingSlots;
+          if (!wait_ab(smem_u32(&ctl->full[slot]), (it / kRingSlots) & 1, p.spin_budget, &ctl->abort)) {
+            good = false;
+            break;
+          }
+          uint8_t* base = ring + at;
+          const uint8_t* codes = base + (bytes[g] >> 1);
+          uint4 v[kMaxPieces];
+#pragma unroll
+          for (int j = 0; j < kMaxPieces; ++j) {
+            const int i = ctid + kCT * j;
+            if (i < npieces) v[j] = *reinterpret_cast<const uint4*>(codes + 16 * i);
+          }
+          named_bar_sync(2, kCT);
+#pragma unroll
+          for (int j = 0; j < kMaxPieces; ++j) {
+            const int i = ctid + kCT * j;
+            if (i >= npieces) break;
+            const int r = i >> 2, q = i & 3;   // row, 16-code quarter -> bf16 pieces 2q, 2q + 1
+            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+            uint32_t o[8];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              o[2 * k] = e4m3x2_to_bf16x2((uint16_t)(w[k] & 0xFFFFu));
+              o[2 * k + 1] = e4m3x2_to_bf16x2((uint16_t)(w[k] >> 16));
+            }
+            uint8_t* row = base + (r >> 3) * 1024 + (r & 7) * 128;
+            *reinterpret_cast<uint4*>(row + (((2 * q) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+          }
+          // generic-proxy stores must be visible to the tensor cores' reads
+          fence_proxy_async_smem();
+          mbar_arrive(smem_u32(&ctl->conv[slot]));
+        }
+      }
+    }
+  }
+  if (!good && !ctl->abort) {
+    atomicOr(p.err, E_CONV);
+    ctl->abort = 1;
+  }
 }
 
 // ------------------------------------------------------------ MMA warp
@@ -267,8 +344,8 @@ __device__ __noinline__ void mma_issuer(const StepParams& p, uint8_t* ring, uint
         for (uint32_t c = 0; c < nch[g]; ++c, ++it) {
           const uint32_t at = ring_place(pos, bytes[g]);
           const uint32_t slot = it % kRingSlots;
-          if (!wait_ab(smem_u32(&ctl->full[slot]), (it / kRingSlots) & 1, p.spin_budget,
-                       &ctl->abort)) {
+          if (!wait_ab(smem_u32(p.fp8 ? &ctl->conv[slot] : &ctl->full[slot]), (it / kRingSlots) & 1,
+                       p.spin_budget, &ctl->abort)) {
             good = false;
             break;
           }
@@ -316,6 +393,7 @@ struct GemmView {
   int ownp;      // row stride (floats) of the staging / receive blocks, multiple of 4
   int nchunk;
   int base;      // first owned packed channel (gate_up: first owned u column)
+  int pbase;     // index of the first owned column in the layer's scale table
   uint32_t recv_off;   // byte offset of the receive buffer in the work region
 };
 
@@ -331,10 +409,19 @@ __device__ __forceinline__ GemmView gemm_view(const Ctx& c, int g) {
   v.nchunk = gp.nchunk;
   v.base = (g == G_GU) ? gp.ch_off[c.cluster] + v.grp * (v.ng / 2) + v.ks * (v.own / 2)
                        : gp.ch_off[c.cluster] + v.grp * v.ng + v.ks * v.own;
+  v.pbase = (g == G_GU) ? 2 * gp.ch_off[c.cluster] + v.grp * v.ng + v.ks * v.own : v.base;
   const uint32_t a_bytes = (uint32_t)v.nchunk * 8192u;
   const uint32_t s_bytes = (uint32_t)(v.KS * kRecvRows * v.ownp * 4);
   v.recv_off = ((a_bytes > s_bytes ? a_bytes : s_bytes) + 15u) & ~15u;
   return v;
+}
+
+// Row scales of two adjacent owned columns (E4M3 weights); 1 for bf16, where
+// the product is exact and leaves the result unchanged.
+__device__ __forceinline__ float2 wscale2(const Ctx& c, int g, int l, int idx) {
+  const StepParams& p = *c.p;
+  if (p.wscale == nullptr) return make_float2(1.f, 1.f);
+  return *reinterpret_cast<const float2*>(p.wscale + (size_t)l * p.sc_stride + p.sc_off[g] + idx);
 }
 
 // Starts GEMM g: arms the receive barrier for the partials the cluster will
@@ -526,6 +613,7 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
 #pragma unroll 1
     for (int t = pa.t0, k = 0; t < T; t += pa.dt, ++k) aux[k * 128] = rope[t * half];
   }
+  const float2 sc = act ? wscale2(c, G_QKV, l, v.pbase + 2 * pa.pr) : make_float2(1.f, 1.f);
   push_partials(c, v);
   if (!c.ok || !act) return;
   const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
@@ -536,7 +624,7 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
   for (int t = pa.t0, k = 0; t < T; t += pa.dt, ++k) {
     const float2 a = recv_sum2(rb, v.KS, v.ownp, t, 2 * pa.pr);
     const float rs = rstd[t];
-    const float y0 = fmaf(rs, a.x, bsh.x), y1 = fmaf(rs, a.y, bsh.y);
+    const float y0 = fmaf(rs, a.x, bsh.x) * sc.x, y1 = fmaf(rs, a.y, bsh.y) * sc.y;
     const int rr = row_off + t;
     uint16_t* rowp = dst + (size_t)rr * hd;
     if (kind < 2) {
@@ -808,7 +896,7 @@ __device__ __noinline__ void phase_attn(Ctx& c, int l) {
 // o_proj / down: gated residual on the owned columns, two threads per row t
 // (each half of the owned column pairs); z for the next linear, row sum of
 // squares.  Operands of the epilogue are fetched before the MMAs finish.
-__device__ __noinline__ void residual_phase(Ctx& c, int g, const uint16_t* act, const float* h_old,
+__device__ __noinline__ void residual_phase(Ctx& c, int g, int l, const uint16_t* act, const float* h_old,
                                             float* h_new, const float* gate, const float* sc,
                                             const float* shift, uint16_t* z, float* sumsq) {
   if (!c.ok) return;
@@ -829,6 +917,10 @@ __device__ __noinline__ void residual_phase(Ctx& c, int g, const uint16_t* act, 
     ho[k] = gt[k] = sv[k] = make_float2(0.f, 0.f);
     if (k < np) {
       gt[k] = *reinterpret_cast<const float2*>(gate + hc);
+      // gate x row scale of the linear (exactly the gate for bf16 weights)
+      const float2 ws = wscale2(c, g, l, v.pbase + 2 * (p0 + k));
+      gt[k].x *= ws.x;
+      gt[k].y *= ws.y;
       if (t < T) ho[k] = *reinterpret_cast<const float2*>(h_old + (size_t)t * d + hc);
       if (z != nullptr) sv[k] = *reinterpret_cast<const float2*>((t == kBiasRow ? shift : sc) + hc);
     }
@@ -876,6 +968,7 @@ __device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
   const float* rstd = c.ctl->rstd;
   uint16_t* u_act = p.u_act;
   const int lg = 2 * pa.pr, lu = uown + 2 * pa.pr;
+  const float2 sg = wscale2(c, G_GU, l, v.pbase + lg), su = wscale2(c, G_GU, l, v.pbase + lu);
   const float2 bg = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lg);
   const float2 bu = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lu);
   tmark(c, 8);
@@ -884,8 +977,8 @@ __device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
     const float2 ag = recv_sum2(rb, v.KS, v.ownp, t, lg);
     const float2 au = recv_sum2(rb, v.KS, v.ownp, t, lu);
     const float rs = rstd[t];
-    const float g0 = fmaf(rs, ag.x, bg.x), g1 = fmaf(rs, ag.y, bg.y);
-    const float u0 = fmaf(rs, au.x, bu.x), u1 = fmaf(rs, au.y, bu.y);
+    const float g0 = fmaf(rs, ag.x, bg.x) * sg.x, g1 = fmaf(rs, ag.y, bg.y) * sg.y;
+    const float u0 = fmaf(rs, au.x, bu.x) * su.x, u1 = fmaf(rs, au.y, bu.y) * su.y;
     const float v0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
     const float v1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
     *reinterpret_cast<uint32_t*>(u_act + act64_off(t, uc)) = pack_bf16(v0, v1);
@@ -1065,14 +1158,14 @@ __device__ void compute_main(Ctx& c) {
       grid_sync(c);
       phase_attn(c, l);
       grid_sync(c);
-      residual_phase(c, G_O, p.o_act, p.h_a, p.h_b, mod_vec(p, s, l, 2), mod_vec(p, s, l, 3),
+      residual_phase(c, G_O, l, p.o_act, p.h_a, p.h_b, mod_vec(p, s, l, 2), mod_vec(p, s, l, 3),
                      mod_vec(p, s, l, 4), p.z_f, p.sumsq_f);
       grid_sync(c);
       phase_gu(c, s, l);
       grid_sync(c);
       {
         const bool next = l + 1 < p.L;
-        residual_phase(c, G_DOWN, p.u_act, p.h_b, p.h_a, mod_vec(p, s, l, 5),
+        residual_phase(c, G_DOWN, l, p.u_act, p.h_b, p.h_a, mod_vec(p, s, l, 5),
                        next ? mod_vec(p, s, l + 1, 0) : nullptr, next ? mod_vec(p, s, l + 1, 1) : nullptr,
                        next ? p.z_a : nullptr, p.sumsq_a);
       }
@@ -1087,7 +1180,7 @@ __device__ void compute_main(Ctx& c) {
 
 }  // namespace
 
-__global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant__ StepParams p) {
+__global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_constant__ StepParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
@@ -1101,6 +1194,7 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
     for (int s = 0; s < kRingSlots; ++s) {
       mbar_init(smem_u32(&ctl->full[s]), 1);
       mbar_init(smem_u32(&ctl->empty[s]), 1);
+      mbar_init(smem_u32(&ctl->conv[s]), 32 * kConvWarps);
     }
     mbar_init(smem_u32(&ctl->act_full), 1);
     mbar_init(smem_u32(&ctl->mma_done), 1);
@@ -1129,6 +1223,8 @@ __global__ void __launch_bounds__(kThreads, 1) step_kernel(const __grid_constant
   } else if (warp == 1) {
     if (lane == 0) mma_issuer(p, ring, work, ctl, tmem, cluster);
     __syncwarp();
+  } else if (warp >= 2 + kComputeWarps) {
+    if (p.fp8) converter(p, ring, ctl, cluster, threadIdx.x - 32 * (2 + kComputeWarps));
   } else {
     Ctx c;
     c.p = &p;
@@ -1171,7 +1267,7 @@ cudaError_t step_max_clusters(int* n_clusters) {
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(kClusterSize * 32, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kStepThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
@@ -1186,7 +1282,7 @@ cudaError_t launch_step(const StepParams& p, cudaStream_t st) {
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.gridDim = dim3(p.n_ctas, 1, 1);
-  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.blockDim = dim3(kStepThreads, 1, 1);
   cfg.dynamicSmemBytes = kSmemBytes;
   cfg.stream = st;
   cfg.attrs = attr;
