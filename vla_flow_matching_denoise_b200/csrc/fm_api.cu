@@ -67,6 +67,18 @@ struct fm_expert {
   std::vector<PackChunk> pack_jobs;
   std::vector<int32_t> pack_rows;
   std::vector<float> row_scale;      // [L][rows of QKV + O + GU + DOWN]
+  // batched path (B >= 2 requests advance together, M = B * T rows)
+  bool batched = false;
+  uint8_t* barena = nullptr;         // per layer: [N/BN][K/64] chunks of each linear
+  uint64_t blayer_bytes = 0;
+  uint64_t boff[4] = {0, 0, 0, 0};
+  int Mp = 0;                        // padded rows of the batched activations
+  uint16_t* bz_a = nullptr;          // ACT128 [Mp/128][d/64]
+  uint16_t* bz_f = nullptr;
+  uint16_t* bo = nullptr;            // ACT128 [Mp/128][Hq*hd/64]
+  uint16_t* bu = nullptr;            // ACT128 [Mp/128][F/64]
+  float* bh = nullptr;               // [Mp][d]
+  uint16_t* bq = nullptr;            // [B_cap][Hkv][q_rows][hd]
   // buffers
   float* mod = nullptr;
   uint16_t* h1_act = nullptr;
@@ -323,6 +335,40 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
     DALLOC(h->wscale, (size_t)c.n_layers * h->sc_stride * 4);
   }
   std::vector<float> sc_host(fp8 ? (size_t)c.n_layers * h->sc_stride : 0, 0.f);
+  // Batched-path packing: each linear as [N/BN][K/64] chunks of BN rows
+  // (gate_up tile j: gate rows 128 j .. then up rows 128 j ..).
+  std::vector<PackChunk> bjobs;
+  std::vector<int32_t> brows;
+  if (h->batched) {
+    const int Ns[4] = {qn + 2 * kn, d, 2 * F, d};
+    const int Ks[4] = {d, qn, d, F};
+    const int epi[4] = {BE_QKV, BE_RESID, BE_SWIGLU, BE_RESID};
+    uint64_t boff = 0;
+    for (int g = 0; g < 4; ++g) {
+      const int bn = bgemm_bn(epi[g], Ns[g]), nkb = Ks[g] / 64;
+      h->boff[g] = boff;
+      for (int nt = 0; nt < Ns[g] / bn; ++nt) {
+        const uint32_t roff = (uint32_t)brows.size();
+        for (int q = 0; q < bn; ++q) {
+          int r = nt * bn + q;
+          if (g == G_GU) r = q < bn / 2 ? nt * (bn / 2) + q : F + nt * (bn / 2) + (q - bn / 2);
+          brows.push_back(r);
+        }
+        for (int kb = 0; kb < nkb; ++kb) {
+          PackChunk pc{};
+          pc.dst_off = boff + ((uint64_t)nt * nkb + kb) * bn * 128;
+          pc.rowidx_off = roff;
+          pc.nrows = (uint16_t)bn;
+          pc.mat = (uint8_t)g;
+          pc.kb = (uint32_t)kb;
+          bjobs.push_back(pc);
+        }
+      }
+      boff += (uint64_t)Ns[g] * Ks[g] * 2;
+    }
+    h->blayer_bytes = boff;
+    DALLOC(h->barena, (size_t)c.n_layers * boff);
+  }
 
   PackChunk* d_jobs = nullptr;
   int32_t* d_rows = nullptr;
@@ -332,7 +378,7 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   DALLOC(h->span_off, span.size() * 4);
   CK(cudaMemcpy(h->span_off, span.data(), span.size() * 4, cudaMemcpyHostToDevice));
   // temporary buffers (freed at the end)
-  void* tmp[8] = {};
+  void* tmp[9] = {};
   const size_t sz_qkv = (size_t)(qn + 2 * kn) * d, sz_o = (size_t)d * qn, sz_gu = (size_t)2 * F * d,
                sz_dn = (size_t)d * F;
   cudaError_t e = cudaSuccess;
@@ -345,6 +391,10 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   // E4M3: codes of the four linears and their row scales
   if (e == cudaSuccess && fp8) e = cudaMalloc(&tmp[6], sz_qkv + sz_o + sz_gu + sz_dn);
   if (e == cudaSuccess && fp8) e = cudaMalloc(&tmp[7], (size_t)(mrows[0] + mrows[1] + mrows[2] + mrows[3]) * 4);
+  if (e == cudaSuccess && h->batched)
+    e = cudaMalloc(&tmp[8], bjobs.size() * sizeof(PackChunk) + brows.size() * 4 + 64);
+  PackChunk* d_bjobs = nullptr;
+  int32_t* d_brows = nullptr;
   fm_status st = FM_OK;
   if (e != cudaSuccess) {
     st = set_err(h, FM_ERR_OOM, "packing buffers: %s", cudaGetErrorString(e));
@@ -368,6 +418,12 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
     }
     e = cudaMemcpy(d_jobs, jobs.data(), jobs.size() * sizeof(PackChunk), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(d_rows, rows.data(), rows.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess && h->batched) {
+      d_bjobs = static_cast<PackChunk*>(tmp[8]);
+      d_brows = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(tmp[8]) + bjobs.size() * sizeof(PackChunk));
+      e = cudaMemcpy(d_bjobs, bjobs.data(), bjobs.size() * sizeof(PackChunk), cudaMemcpyHostToDevice);
+      if (e == cudaSuccess) e = cudaMemcpy(d_brows, brows.data(), brows.size() * 4, cudaMemcpyHostToDevice);
+    }
     if (e == cudaSuccess && fp8) e = cudaMemcpy(d_mats, q8, sizeof(q8), cudaMemcpyHostToDevice);
     else if (e == cudaSuccess) e = cudaMemcpy(d_mats, mats, sizeof(mats), cudaMemcpyHostToDevice);
     if (e == cudaSuccess) e = cudaMemcpy(d_matk, matk, sizeof(matk), cudaMemcpyHostToDevice);
@@ -405,6 +461,9 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
         }
       } else if (e == cudaSuccess) {
         e = launch_pack(d_jobs, (int)jobs.size(), d_rows, d_mats, d_matk, h->arena + (size_t)l * off, 0);
+        if (e == cudaSuccess && h->batched)
+          e = launch_pack(d_bjobs, (int)bjobs.size(), d_brows, d_mats, d_matk,
+                          h->barena + (size_t)l * h->blayer_bytes, 0);
       }
       if (e == cudaSuccess) e = cudaDeviceSynchronize();
       if (e != cudaSuccess) st = set_err(h, FM_ERR_CUDA, "packing layer %d: %s", l, cudaGetErrorString(e));
@@ -611,8 +670,126 @@ TimeParams time_params(const fm_expert* h, int steps) {
   return t;
 }
 
+// Batched path: Euler steps step0 .. step1 - 1 of a `steps`-step schedule for
+// `batch` requests together (x in h->x, velocities to h->vbuf; x updated when
+// `update`).  The modulation rows must already be in h->mod.
+cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int steps, bool update,
+                            cudaStream_t st) {
+  const fm_config& c = h->cfg;
+  const int T = c.chunk_len, d = c.d_model, M = batch * T, L = c.n_layers;
+  const int qn = c.n_q_heads * c.head_dim, kn = c.n_kv_heads * c.head_dim, F = c.d_ff;
+  const int Mp = (M + kBM - 1) / kBM * kBM;
+  const size_t lay = (size_t)c.max_batch * c.n_kv_heads * h->S_max * c.head_dim;
+  BRowParams r{};
+  r.M = M;
+  r.T = T;
+  r.A = c.action_dim;
+  r.d = d;
+  r.eps = c.rms_eps;
+  r.dt = -1.0f / (float)steps;
+  r.x = h->x;
+  r.x_out = update ? h->x : nullptr;
+  r.v_out = h->vbuf;
+  r.w_in = h->w_in;
+  r.w_out = h->w_out;
+  r.out_bias = h->out_bias;
+  r.h = h->bh;
+  BGemmParams g{};
+  g.M = M;
+  g.Mp = Mp;
+  g.h = h->bh;
+  g.u_act = h->bu;
+  g.F = F;
+  g.qbuf = h->bq;
+  g.rope = h->rope;
+  g.P_dev = h->P_dev;
+  g.T = T;
+  g.Hq = c.n_q_heads;
+  g.Hkv = c.n_kv_heads;
+  g.hd = c.head_dim;
+  g.S_max = h->S_max;
+  g.q_rows = h->q_rows;
+  g.err = h->err_word;
+  g.spin_budget = 4000000000LL;
+  BAttnParams a{};
+  a.qbuf = h->bq;
+  a.o_act = h->bo;
+  a.P_dev = h->P_dev;
+  a.B = batch;
+  a.T = T;
+  a.Hq = c.n_q_heads;
+  a.Hkv = c.n_kv_heads;
+  a.hd = c.head_dim;
+  a.S_max = h->S_max;
+  a.q_rows = h->q_rows;
+  a.qblocks = (c.n_q_heads / c.n_kv_heads * T + 63) / 64;
+  a.err = h->err_word;
+  a.spin_budget = 4000000000LL;
+  cudaError_t e = cudaSuccess;
+  for (int s = step0; s < step1 && e == cudaSuccess; ++s) {
+    const float* mrow = h->mod + (size_t)s * h->n_mod;
+    r.s = mrow;
+    r.b = mrow + d;
+    r.z = h->bz_a;
+    e = launch_binproj(r, st);
+    for (int l = 0; l < L && e == cudaSuccess; ++l) {
+      const float* lm = mrow + (size_t)6 * l * d;
+      const uint8_t* wl = h->barena + (size_t)l * h->blayer_bytes;
+      // QKV + RoPE -> q, cache rows P .. P + T - 1
+      g.A = reinterpret_cast<const uint8_t*>(h->bz_a);
+      g.W = wl + h->boff[G_QKV];
+      g.K = d;
+      g.N = qn + 2 * kn;
+      g.kc = h->kcache + l * lay;
+      g.vc = h->vcache + l * lay;
+      e = launch_bgemm(g, BE_QKV, h->n_sms, st);
+      a.kc = h->kcache + l * lay;
+      a.vc = h->vcache + l * lay;
+      if (e == cudaSuccess) e = launch_battn(a, st);
+      // o_proj + gated residual, then the FFN norm
+      g.A = reinterpret_cast<const uint8_t*>(h->bo);
+      g.W = wl + h->boff[G_O];
+      g.K = qn;
+      g.N = d;
+      g.gate = lm + 2 * d;
+      if (e == cudaSuccess) e = launch_bgemm(g, BE_RESID, h->n_sms, st);
+      r.s = lm + 3 * d;
+      r.b = lm + 4 * d;
+      r.z = h->bz_f;
+      if (e == cudaSuccess) e = launch_bnorm(r, st);
+      // gate_up + SwiGLU, down + gated residual
+      g.A = reinterpret_cast<const uint8_t*>(h->bz_f);
+      g.W = wl + h->boff[G_GU];
+      g.K = d;
+      g.N = 2 * F;
+      if (e == cudaSuccess) e = launch_bgemm(g, BE_SWIGLU, h->n_sms, st);
+      g.A = reinterpret_cast<const uint8_t*>(h->bu);
+      g.W = wl + h->boff[G_DOWN];
+      g.K = F;
+      g.N = d;
+      g.gate = lm + 5 * d;
+      if (e == cudaSuccess) e = launch_bgemm(g, BE_RESID, h->n_sms, st);
+      if (l + 1 < L && e == cudaSuccess) {
+        r.s = lm + 6 * d;
+        r.b = lm + 7 * d;
+        r.z = h->bz_a;
+        e = launch_bnorm(r, st);
+      }
+    }
+    r.s = mrow + (size_t)6 * L * d;
+    r.b = r.s + d;
+    if (e == cudaSuccess) e = launch_boutproj(r, st);
+  }
+  return e;
+}
+
 // Enqueues one full denoise of `batch` requests (x already in h->x).
 cudaError_t enqueue_denoise(fm_expert* h, int batch, int steps, cudaStream_t st) {
+  if (batch >= 2 && h->batched) {
+    cudaError_t e = launch_time(time_params(h, steps), h->n_sms, st);
+    if (e != cudaSuccess) return e;
+    return enqueue_batched(h, batch, 0, steps, steps, true, st);
+  }
   cudaError_t e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
   if (e != cudaSuccess) return e;
   e = launch_time(time_params(h, steps), h->n_sms, st);
@@ -719,6 +896,14 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
     set_err(h, FM_ERR_CUDA, "stream creation failed");
     return bail(FM_ERR_CUDA);
   }
+  {
+    // the batched path needs whole 128-column weight tiles, the in-proj's
+    // 256-column thread mapping and at most 1024 residual columns
+    const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+    h->batched = c.wtype == FM_W_BF16 && c.max_batch >= 2 && c.d_model % 256 == 0 && c.d_model <= 1024 &&
+                 c.d_ff % 128 == 0 && qkv % 128 == 0 && (c.n_q_heads * c.head_dim) % 64 == 0 &&
+                 (c.head_dim == 64 || c.head_dim == 128);
+  }
   if ((st = pack_weights(h, w)) != FM_OK) return bail(st);
 
   const size_t T = c.chunk_len, A = c.action_dim, d = c.d_model;
@@ -748,6 +933,16 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
   ALLOC_OR_BAIL(h->vcache, kv);
   ALLOC_OR_BAIL(h->bar_count, (size_t)(h->n_ctas + 4) * 4);
   ALLOC_OR_BAIL(h->err_word, 4);
+  if (h->batched) {
+    h->Mp = (int)((B * T + kBM - 1) / kBM * kBM);
+    const size_t Mp = (size_t)h->Mp;
+    ALLOC_OR_BAIL(h->bz_a, Mp * d * 2);
+    ALLOC_OR_BAIL(h->bz_f, Mp * d * 2);
+    ALLOC_OR_BAIL(h->bo, Mp * c.n_q_heads * c.head_dim * 2);
+    ALLOC_OR_BAIL(h->bu, Mp * c.d_ff * 2);
+    ALLOC_OR_BAIL(h->bh, Mp * d * 4);
+    ALLOC_OR_BAIL(h->bq, B * c.n_kv_heads * h->q_rows * c.head_dim * 2);
+  }
 #undef ALLOC_OR_BAIL
   if (cudaDeviceSynchronize() != cudaSuccess) {
     set_err(h, FM_ERR_CUDA, "set-up failed: %s", cudaGetErrorString(cudaGetLastError()));
@@ -900,16 +1095,20 @@ fm_status fm_velocity(fm_expert* h, const float* x, int batch, int step_index, i
   if (s != FM_OK) return s;
   const fm_config& c = h->cfg;
   const size_t xs = (size_t)c.chunk_len * c.action_dim;
-  for (int b = 0; b < batch; ++b) {
-    StepParams p = base_params(h);
-    p.b = b;
-    p.x = h->x + b * xs;
-    p.vbuf = h->vbuf + b * xs;
-    p.step0 = step_index;
-    p.step1 = step_index + 1;
-    p.update_x = 0;
-    CK(cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st));
-    CK(launch_step(p, st));
+  if (batch >= 2 && h->batched) {
+    CK(enqueue_batched(h, batch, step_index, step_index + 1, steps, false, st));
+  } else {
+    for (int b = 0; b < batch; ++b) {
+      StepParams p = base_params(h);
+      p.b = b;
+      p.x = h->x + b * xs;
+      p.vbuf = h->vbuf + b * xs;
+      p.step0 = step_index;
+      p.step1 = step_index + 1;
+      p.update_x = 0;
+      CK(cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st));
+      CK(launch_step(p, st));
+    }
   }
   CK(cudaMemcpyAsync(v_out, h->vbuf, (size_t)batch * xs * 4, cudaMemcpyDefault, st));
   if (!is_device_ptr(v_out)) {
@@ -1072,7 +1271,8 @@ fm_status fm_profile_denoise(fm_expert* h, int batch, int steps, int iters, floa
     cudaError_t e = cudaEventRecord(ev[0], st);
     if (e == cudaSuccess) e = launch_time(time_params(h, steps), h->n_sms, st);
     if (e == cudaSuccess) e = cudaEventRecord(ev[1], st);
-    for (int b = 0; b < batch && e == cudaSuccess; ++b) {
+    if (e == cudaSuccess && batch >= 2 && h->batched) e = enqueue_batched(h, batch, 0, steps, steps, true, st);
+    for (int b = 0; b < batch && e == cudaSuccess && !(batch >= 2 && h->batched); ++b) {
       StepParams p = base_params(h);
       p.b = b;
       p.x = h->x + b * xs;

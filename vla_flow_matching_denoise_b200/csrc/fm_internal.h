@@ -117,6 +117,64 @@ struct StepParams {
   int tlog_chunks;           // chunk slots per section
 };
 
+// ---------------------------------------------------------------- batched path
+// Layout "ACT128": a bf16 activation matrix of Mp rows (Mp a multiple of 128;
+// row m = b * T + t for request b, token t) stored as [Mp/128][K/64] blocks of
+// 128 rows x 128 bytes (16 KB), 16-byte pieces swizzled by (row & 7): the
+// image tcgen05.mma reads for an M = 128 operand.  Packed batched weights:
+// [N/BN][K/64] chunks of BN rows x 64 columns in the same swizzled image.
+constexpr int kBM = 128;               // rows per batched GEMM tile
+constexpr int kBRing = 192 * 1024;     // batched GEMM operand ring
+
+enum BEpi { BE_QKV = 0, BE_RESID = 1, BE_SWIGLU = 2 };
+
+struct BGemmParams {
+  const uint8_t* A;          // ACT128 [Mp/128][K/64]
+  const uint8_t* W;          // packed [N/BN][K/64] chunks of BN x 64
+  int K, N, M, Mp;           // reduction, output channels, valid rows (B*T), padded rows
+  // BE_RESID: h[m][n] += gate[n] * D[m][n]   (fp32, row stride N)
+  float* h;
+  const float* gate;
+  // BE_SWIGLU: tile j holds gate rows 128j.. then up rows 128j..; u = SiLU(g) up
+  uint16_t* u_act;           // ACT128 [Mp/128][F/64]
+  int F;
+  // BE_QKV: RoPE on q, k; q -> qbuf [B][Hkv][q_rows][hd]; k, v -> cache rows P + t
+  uint16_t* qbuf;
+  uint16_t* kc;              // this layer's K cache [B_cap][Hkv][S_max][hd]
+  uint16_t* vc;
+  const float* rope;         // [T][hd/2] (cos, sin)
+  const int* P_dev;
+  int T, Hq, Hkv, hd, S_max, q_rows;
+  uint32_t* err;
+  long long spin_budget;
+};
+
+struct BRowParams {          // in-proj, AdaRMSNorm, out-proj + Euler (row kernels)
+  int M, T, A, d;
+  float eps, dt;
+  const float* x;            // [M][A] (in-proj input)
+  float* x_out;              // [M][A] updated in place by out-proj (x += dt v), or null
+  float* v_out;              // [M][A] velocity
+  const uint16_t* w_in;      // [d][A]
+  const uint16_t* w_out;     // [A][d]
+  const float* out_bias;     // [A] or null
+  float* h;                  // [Mp][d] fp32 residual
+  const float* s;            // norm scale and shift [d]
+  const float* b;
+  uint16_t* z;               // ACT128 [Mp/128][d/64]
+};
+
+struct BAttnParams {
+  const uint16_t* qbuf;      // [B][Hkv][q_rows][hd]
+  const uint16_t* kc;        // this layer's cache [B_cap][Hkv][S_max][hd]
+  const uint16_t* vc;
+  uint16_t* o_act;           // ACT128 [Mp/128][Hq*hd/64]
+  const int* P_dev;
+  int B, T, Hq, Hkv, hd, S_max, q_rows, qblocks;
+  uint32_t* err;
+  long long spin_budget;
+};
+
 struct TimeParams {
   int n_steps, d, n_mod;
   const uint16_t* w1;        // [d, 256] bf16

@@ -27,6 +27,14 @@ size_t step_smem_bytes();
 cudaError_t step_max_clusters(int* n_clusters);
 cudaError_t launch_step(const StepParams& p, cudaStream_t st);
 
+// Batched path (B requests per step, M = B * T rows).
+int bgemm_bn(int epi, int N);   // weight tile width the GEMM uses for this epilogue
+cudaError_t launch_bgemm(const BGemmParams& p, int epi, int n_sms, cudaStream_t st);
+cudaError_t launch_binproj(const BRowParams& p, cudaStream_t st);
+cudaError_t launch_bnorm(const BRowParams& p, cudaStream_t st);
+cudaError_t launch_boutproj(const BRowParams& p, cudaStream_t st);
+cudaError_t launch_battn(const BAttnParams& p, cudaStream_t st);
+
 // Sets the text fm_last_error(NULL) returns on this thread.
 void set_thread_error(const char* msg);
 

@@ -19,10 +19,12 @@
 //    cluster) and, inside a cluster, over its 8 CTAs by K and n-groups.  Warp
 //    1 issues tcgen05.mma with M = 64 token rows (50 valid + the shift row +
 //    padding), N = the CTA's channels, accumulating fp32 in TMEM.
-//  * Split-K partials go straight from TMEM registers to the CTA that owns
-//    the output columns: st.async into its receive buffer completes bytes on
-//    its mbarrier, so the owner waits once and reduces from local shared
-//    memory in a fixed order (results are bit-reproducible).
+//  * Split-K partials leave TMEM through tcgen05.ld, are staged in shared
+//    memory as one block per owner of output columns, and each block goes to
+//    its owner with one bulk copy shared::cta -> shared::cluster that
+//    completes bytes on the owner's mbarrier; the owner waits once and reduces
+//    its KS slots from local shared memory in a fixed order (results are
+//    bit-reproducible).
 //  * AdaRMSNorm is folded into the linears: the owner of a residual column
 //    writes z = bf16(h (1 + s)) and, in row 50, the shift b; the consumer
 //    linear's epilogue applies rstd(row) to rows 0..49 and adds row 50
@@ -524,16 +526,18 @@ __device__ __noinline__ void load_rstd(const Ctx& c, const float* sumsq) {
   Ctrl* const ctl = c.ctl;
   const float4* src = reinterpret_cast<const float4*>(sumsq);
   const int nf4 = n * (kRows / 4);
+  // every load in flight at once (one L2 round trip), then added in CTA order
+  constexpr int kMaxF = kMaxClusters * kClusterSize * (kRows / 4) / 128;
+  float4 x[kMaxF];
+#pragma unroll
+  for (int j = 0; j < kMaxF; ++j) {
+    const int f = tid + 128 * j;
+    x[j] = f < nf4 ? src[f] : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
   float4 a = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 1
-  for (int f = tid; f < nf4; f += 4 * 128) {
-    float4 x[4];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) x[j] = f + 128 * j < nf4 ? src[f + 128 * j] : make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      a.x += x[j].x; a.y += x[j].y; a.z += x[j].z; a.w += x[j].w;
-    }
+  for (int j = 0; j < kMaxF; ++j) {
+    a.x += x[j].x; a.y += x[j].y; a.z += x[j].z; a.w += x[j].w;
   }
   *reinterpret_cast<float4*>(&ctl->red[tid >> 4][4 * (tid & 15)]) = a;
   compute_sync();
