@@ -352,7 +352,7 @@ def main():
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_chunk": ms_e2e / args.steps,
                 "h2d_bytes_per_step": int(x0.nbytes), "d2h_bytes_per_step": int(x0.nbytes)},
-        "gpu_launches": args.steps * ((2 + n * (7 * shape.n_layers + 1)) if batched else (2 + B)),
+        "gpu_launches": args.steps * ((2 + n * (7 * shape.n_layers + 2)) if batched else (2 + B)),
         "roofline": ({"bound": "tensor", "achieved": lf / (ms_loop / 1000.0) / 1e12, "peak": tflops_sus,
                       "unit": "TFLOP/s", "frac": lf / (ms_loop / 1000.0) / 1e12 / tflops_sus,
                       "traffic": traffic, "peak_kind": peak_kind + " sustained bf16",

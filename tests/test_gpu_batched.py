@@ -31,9 +31,14 @@ def _request(kp, vp, b):
     return [k[b:b + 1] for k in kp], [v[b:b + 1] for v in vp]
 
 
-@pytest.mark.parametrize("B,P", [(2, 64), (3, 37), (5, 0)])
-def test_batched_tiny_matches_oracle_per_request(B, P):
-    s = dataclasses.replace(synth.WORKLOADS["tiny"], batch=B, prefix_len=P)
+# a narrow expert with LingBot's head and FFN widths (K of o_proj 2048, of
+# down 4096; 256-wide QKV tiles)
+WIDE = synth.ExpertShape(2, 256, 16, 2, 128, 4096, 75, 64, 10)
+
+
+@pytest.mark.parametrize("base,B,P", [("tiny", 2, 64), ("tiny", 3, 37), ("tiny", 5, 0), ("wide", 3, 64)])
+def test_batched_tiny_matches_oracle_per_request(base, B, P):
+    s = dataclasses.replace(WIDE if base == "wide" else synth.WORKLOADS["tiny"], batch=B, prefix_len=P)
     raw = synth.make_weights(s)
     W = O.Weights(raw)
     kp, vp = synth.make_prefix(s, seed=B)

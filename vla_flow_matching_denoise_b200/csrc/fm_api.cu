@@ -77,7 +77,8 @@ struct fm_expert {
   uint16_t* bz_f = nullptr;
   uint16_t* bo = nullptr;            // ACT128 [Mp/128][Hq*hd/64]
   uint16_t* bu = nullptr;            // ACT128 [Mp/128][F/64]
-  float* bh = nullptr;               // [Mp][d]
+  float* bh = nullptr;               // [Mp][d] residual
+  float* bdelta = nullptr;           // [Mp][d] gated branch of o_proj / down
   uint16_t* bq = nullptr;            // [B_cap][Hkv][q_rows][hd]
   // buffers
   float* mod = nullptr;
@@ -694,10 +695,11 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
   r.w_out = h->w_out;
   r.out_bias = h->out_bias;
   r.h = h->bh;
+  r.delta = h->bdelta;
   BGemmParams g{};
   g.M = M;
   g.Mp = Mp;
-  g.h = h->bh;
+  g.h = h->bdelta;
   g.u_act = h->bu;
   g.F = F;
   g.qbuf = h->bq;
@@ -756,7 +758,7 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       r.s = lm + 3 * d;
       r.b = lm + 4 * d;
       r.z = h->bz_f;
-      if (e == cudaSuccess) e = launch_bnorm(r, st);
+      if (e == cudaSuccess) e = launch_bresnorm(r, st);
       // gate_up + SwiGLU, down + gated residual
       g.A = reinterpret_cast<const uint8_t*>(h->bz_f);
       g.W = wl + h->boff[G_GU];
@@ -769,12 +771,12 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       g.N = d;
       g.gate = lm + 5 * d;
       if (e == cudaSuccess) e = launch_bgemm(g, BE_RESID, h->n_sms, st);
-      if (l + 1 < L && e == cudaSuccess) {
-        r.s = lm + 6 * d;
-        r.b = lm + 7 * d;
-        r.z = h->bz_a;
-        e = launch_bnorm(r, st);
-      }
+      // h += gated down branch; the next layer's attention norm (none after
+      // the last layer: the out-proj kernel applies the final norm)
+      r.s = lm + 6 * d;
+      r.b = lm + 7 * d;
+      r.z = l + 1 < L ? h->bz_a : nullptr;
+      if (e == cudaSuccess) e = launch_bresnorm(r, st);
     }
     r.s = mrow + (size_t)6 * L * d;
     r.b = r.s + d;
@@ -941,6 +943,7 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
     ALLOC_OR_BAIL(h->bo, Mp * c.n_q_heads * c.head_dim * 2);
     ALLOC_OR_BAIL(h->bu, Mp * c.d_ff * 2);
     ALLOC_OR_BAIL(h->bh, Mp * d * 4);
+    ALLOC_OR_BAIL(h->bdelta, Mp * d * 4);
     ALLOC_OR_BAIL(h->bq, B * c.n_kv_heads * h->q_rows * c.head_dim * 2);
   }
 #undef ALLOC_OR_BAIL

@@ -60,6 +60,8 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __e
 // Thread = one accumulator row (TMEM lane); `ta` is the TMEM address of column
 // 0 of this tile for the thread's lane quarter.
 
+// Gated residual branch: delta[m][n] = gate[n] * D[m][n] (fp32, stores only;
+// the row kernel that follows adds it to h and normalises).
 template <int BN>
 __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt) {
 #pragma unroll 1
@@ -69,17 +71,12 @@ __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int
     tmem_ld_wait();
     if (!valid) continue;
     const int n0 = nt * BN + cb * 16;
-    float4* hp = reinterpret_cast<float4*>(p.h + (size_t)m * p.N + n0);
+    float4* dp = reinterpret_cast<float4*>(p.h + (size_t)m * p.N + n0);
     const float4* gp = reinterpret_cast<const float4*>(p.gate + n0);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
-      float4 hv = hp[q];
       const float4 g = gp[q];
-      hv.x = fmaf(g.x, v[4 * q], hv.x);
-      hv.y = fmaf(g.y, v[4 * q + 1], hv.y);
-      hv.z = fmaf(g.z, v[4 * q + 2], hv.z);
-      hv.w = fmaf(g.w, v[4 * q + 3], hv.w);
-      hp[q] = hv;
+      dp[q] = make_float4(g.x * v[4 * q], g.y * v[4 * q + 1], g.z * v[4 * q + 2], g.w * v[4 * q + 3]);
     }
   }
 }
@@ -143,11 +140,14 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
         tmem_ld_wait();
         if (!valid) continue;
         float ol[16], oh[16];
+        const float4* r4 = reinterpret_cast<const float4*>(rope + c);   // (cos, sin) pairs, 128 B
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float2 r = rope[c + i];
-          ol[i] = lo[i] * r.x - hi[i] * r.y;
-          oh[i] = hi[i] * r.x + lo[i] * r.y;
+        for (int i = 0; i < 8; ++i) {
+          const float4 r = r4[i];
+          ol[2 * i] = lo[2 * i] * r.x - hi[2 * i] * r.y;
+          oh[2 * i] = hi[2 * i] * r.x + lo[2 * i] * r.y;
+          ol[2 * i + 1] = lo[2 * i + 1] * r.z - hi[2 * i + 1] * r.w;
+          oh[2 * i + 1] = hi[2 * i + 1] * r.z + lo[2 * i + 1] * r.w;
         }
         store_row16(rowp, row, c, ol);
         store_row16(rowp, row, half + c, oh);
@@ -181,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkb = p.K / 64;
   const int MT = p.Mp / kBM, NT = p.N / BN;
-  const int ntiles = MT * NT;
+  const int ntiles = MT * NT;   // m-tile fastest
   const long long budget = p.spin_budget;
 
   if (threadIdx.x == 0) {
@@ -371,21 +371,26 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
   }
 }
 
-// AdaRMSNorm: one warp per row, z = bf16(h rstd (1 + s) + b) in ACT128.
-__global__ void __launch_bounds__(256) bnorm_kernel(const __grid_constant__ BRowParams p) {
+// Gated residual + AdaRMSNorm, one warp per row: h += delta, then (unless z
+// is null) z = bf16(h rstd (1 + s) + b) in ACT128.
+__global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ BRowParams p) {
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= p.M) return;
   const int d = p.d, n4 = d / 128;   // float4 per lane
-  const float4* hr = reinterpret_cast<const float4*>(p.h + (size_t)m * d);
+  float4* hr = reinterpret_cast<float4*>(p.h + (size_t)m * d);
   float4 v[8];
   float s = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     if (i >= n4) break;
-    v[i] = hr[lane + 32 * i];
+    const float4 br = reinterpret_cast<const float4*>(p.delta + (size_t)m * d)[lane + 32 * i];
+    const float4 a = hr[lane + 32 * i];
+    v[i] = make_float4(a.x + br.x, a.y + br.y, a.z + br.z, a.w + br.w);
+    hr[lane + 32 * i] = v[i];
     s = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, fmaf(v[i].w, v[i].w, s))));
   }
+  if (p.z == nullptr) return;
 #pragma unroll
   for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   const float rs = 1.0f / sqrtf(s / (float)d + p.eps);
@@ -458,19 +463,23 @@ __global__ void __launch_bounds__(256) boutproj_kernel(const __grid_constant__ B
 
 // ------------------------------------------------------------------ attention
 // One CTA per (request b, KV group g, block of 64 of the group's G*T query
-// rows); 4 warps x 16 rows; keys in tiles of 64 (double-buffered bulk copies),
-// QK^T and PV with mma.sync m16n8k16, online softmax in base 2.
+// rows); 4 warps x 16 rows.  Each warp keeps its q rows as mma.sync A
+// fragments in registers (loaded once from global), and walks the keys in
+// tiles of 64 (K and V double-buffered in shared memory by bulk copy):
+// S = q K^T for the 64 keys (m16n8k16), one online-softmax update per tile
+// (base 2), then P V with P taken straight from the S accumulators.
+constexpr int kAttnKeys = 64;
 template <int HD>
-__global__ void __launch_bounds__(128) battn_kernel(const __grid_constant__ BAttnParams p) {
+__global__ void __launch_bounds__(128, 3) battn_kernel(const __grid_constant__ BAttnParams p) {
   constexpr int KSTEPS = HD / 16;
-  constexpr int DT = HD / 8;
-  constexpr int TILE = 64 * HD * 2;     // bytes of a 64-row tile
+  constexpr int DT = HD / 8;                      // 8-column tiles of the output
+  constexpr int NT = kAttnKeys / 8;               // 8-key tiles of S
+  constexpr int TILE = kAttnKeys * HD * 2;        // bytes of one K or V tile
   extern __shared__ uint8_t sm_raw[];
   uint8_t* sm = align1024(sm_raw);
-  uint8_t* qs = sm;
-  uint8_t* kbuf = sm + TILE;            // [2] K tiles
-  uint8_t* vbuf = kbuf + 2 * TILE;      // [2] V tiles
-  uint64_t* bars = reinterpret_cast<uint64_t*>(vbuf + 2 * TILE);   // [3]: q, tile 0, tile 1
+  uint8_t* kbuf = sm;                             // [2] K tiles
+  uint8_t* vbuf = sm + 2 * TILE;                  // [2] V tiles
+  uint64_t* bars = reinterpret_cast<uint64_t*>(vbuf + 2 * TILE);   // [2] tile barriers
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int qb = blockIdx.x % p.qblocks;
   const int g = (blockIdx.x / p.qblocks) % p.Hkv;
@@ -484,43 +493,49 @@ __global__ void __launch_bounds__(128) battn_kernel(const __grid_constant__ BAtt
   const size_t kvoff = (((size_t)b * p.Hkv + g) * p.S_max) * HD;
   const uint16_t* kg = p.kc + kvoff;
   const uint16_t* vg = p.vc + kvoff;
-  const uint16_t* qg = p.qbuf + (((size_t)b * p.Hkv + g) * p.q_rows + row0) * HD;
-  const int ntile = (S + 63) / 64;
+  const int ntile = (S + kAttnKeys - 1) / kAttnKeys;
   if (tid == 0) {
-    for (int i = 0; i < 3; ++i) mbar_init(smem_u32(&bars[i]), 1);
+    mbar_init(smem_u32(&bars[0]), 1);
+    mbar_init(smem_u32(&bars[1]), 1);
     fence_mbar_init();
   }
   __syncthreads();
   const uint64_t pol = policy_evict_last();
   auto issue = [&](int it) {
-    const int kb = it * 64, nk = min(64, S - kb);
-    const uint32_t bar = smem_u32(&bars[1 + (it & 1)]);
+    const int kb = it * kAttnKeys, nk = min(kAttnKeys, S - kb);
+    const uint32_t bar = smem_u32(&bars[it & 1]);
     mbar_arrive_expect_tx(bar, 2u * (uint32_t)nk * HD * 2u);
     bulk_g2s(smem_u32(kbuf + (it & 1) * TILE), kg + (size_t)kb * HD, (uint32_t)nk * HD * 2, bar, pol);
     bulk_g2s(smem_u32(vbuf + (it & 1) * TILE), vg + (size_t)kb * HD, (uint32_t)nk * HD * 2, bar, pol);
   };
   if (tid == 0) {
-    mbar_arrive_expect_tx(smem_u32(&bars[0]), 64u * HD * 2u);
-    bulk_g2s(smem_u32(qs), qg, 64u * HD * 2u, smem_u32(&bars[0]), pol);   // q_rows padding keeps this in bounds
     issue(0);
     if (ntile > 1) issue(1);
   }
-  const long long budget = p.spin_budget;
-  if (!mbar_wait(smem_u32(&bars[0]), 0, budget)) {
-    atomicOr(p.err, 0x1000u);
-    return;
-  }
+  // q fragments (rows r0 + gid, r0 + gid + 8; columns 16 kk + 2 tig (+8))
+  const int gid = lane >> 2, tig = lane & 3;
   const int r0 = 16 * warp;
+  uint32_t qa[KSTEPS][4];
+  {
+    const uint16_t* qg = p.qbuf + (((size_t)b * p.Hkv + g) * p.q_rows) * HD;
+    const int Ra = row0 + r0 + gid, Rb = Ra + 8;   // rows of the group block (q_rows padding is zero)
+    const uint16_t* qra = qg + (size_t)Ra * HD;
+    const uint16_t* qrb = qg + (size_t)Rb * HD;
+#pragma unroll
+    for (int kk = 0; kk < KSTEPS; ++kk) {
+      const int e0 = 16 * kk + 2 * tig;
+      qa[kk][0] = *reinterpret_cast<const uint32_t*>(qra + ((((e0 >> 3)) ^ (Ra & 7)) << 3) + (e0 & 7));
+      qa[kk][1] = *reinterpret_cast<const uint32_t*>(qrb + ((((e0 >> 3)) ^ (Rb & 7)) << 3) + (e0 & 7));
+      qa[kk][2] = *reinterpret_cast<const uint32_t*>(qra + ((((e0 >> 3) + 1) ^ (Ra & 7)) << 3) + (e0 & 7));
+      qa[kk][3] = *reinterpret_cast<const uint32_t*>(qrb + ((((e0 >> 3) + 1) ^ (Rb & 7)) << 3) + (e0 & 7));
+    }
+  }
+  const long long budget = p.spin_budget;
   const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
   float m_r[2] = {-INFINITY, -INFINITY}, l_r[2] = {0.f, 0.f};
   float o[DT][4];
 #pragma unroll
   for (int i = 0; i < DT; ++i) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-  const uint32_t qa = smem_u32(qs);
-  const int qrow = r0 + (lane & 15);
-  const uint32_t q_lane = qa + qrow * HD * 2;
-  const int q_sw = (row0 + qrow) & 7;
-  const int q_pc = lane >> 4;
   const int kkey = (lane & 7) + ((lane >> 4) << 3);
   const int k_pc = (lane >> 3) & 1;
   const int vkey = (lane & 7) + (((lane >> 3) & 1) << 3);
@@ -528,89 +543,90 @@ __global__ void __launch_bounds__(128) battn_kernel(const __grid_constant__ BAtt
   bool good = true;
 #pragma unroll 1
   for (int it = 0; it < ntile; ++it) {
-    const int kb = it * 64, nk = min(64, S - kb);
-    if (!mbar_wait(smem_u32(&bars[1 + (it & 1)]), (it >> 1) & 1, budget)) {
+    const int kb = it * kAttnKeys, nk = min(kAttnKeys, S - kb);
+    if (!mbar_wait(smem_u32(&bars[it & 1]), (it >> 1) & 1, budget)) {
       atomicOr(p.err, 0x2000u);
       good = false;
       break;
     }
     uint8_t* ks_ = kbuf + (it & 1) * TILE;
     uint8_t* vs_ = vbuf + (it & 1) * TILE;
-    const int nk16 = (nk + 15) & ~15;
-    if (nk16 > nk) {
+    if (nk < kAttnKeys) {
       // zero V rows past the last key so no stale shared memory meets a zero weight
       uint4* zr = reinterpret_cast<uint4*>(vs_ + (size_t)nk * HD * 2);
-      for (int i = tid; i < (nk16 - nk) * HD * 2 / 16; i += 128) zr[i] = make_uint4(0u, 0u, 0u, 0u);
+      for (int i = tid; i < (kAttnKeys - nk) * HD * 2 / 16; i += 128) zr[i] = make_uint4(0u, 0u, 0u, 0u);
       __syncthreads();
     }
     const uint32_t ka = smem_u32(ks_), va = smem_u32(vs_);
-#pragma unroll 1
-    for (int kt = 0; kt < nk; kt += 16) {
-      float s[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      const uint32_t k_lane = ka + (kt + kkey) * HD * 2;
-      const int k_sw = (kt + kkey) & 7;    // kb is a multiple of 64: absolute row & 7
-#pragma unroll 2
-      for (int kk = 0; kk < KSTEPS; ++kk) {
-        uint32_t a0, a1, a2, a3, b0, b1, b2, b3;
-        ldsm_x4(q_lane + (((2 * kk + q_pc) ^ q_sw) << 4), a0, a1, a2, a3);
-        ldsm_x4(k_lane + (((2 * kk + k_pc) ^ k_sw) << 4), b0, b1, b2, b3);
-        mma16816(s[0], a0, a1, a2, a3, b0, b1);
-        mma16816(s[1], a0, a1, a2, a3, b2, b3);
-      }
-      float mx[2] = {-INFINITY, -INFINITY};
+    // S = q K^T over the 64 keys of the tile (kb is a multiple of 64, so a
+    // key's swizzle row is its index inside the tile)
+    float sc[NT][4];
 #pragma unroll
-      for (int t2 = 0; t2 < 2; ++t2) {
+    for (int j = 0; j < NT; ++j) sc[j][0] = sc[j][1] = sc[j][2] = sc[j][3] = 0.f;
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const int key = kt + 8 * t2 + 2 * (lane & 3) + (e & 1);
-          s[t2][e] = key < nk ? s[t2][e] * sl2 : -INFINITY;
-          mx[e >> 1] = fmaxf(mx[e >> 1], s[t2][e]);
-        }
-      }
+    for (int kk = 0; kk < KSTEPS; ++kk) {
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 1));
-        mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 2));
+      for (int j2 = 0; j2 < NT / 2; ++j2) {
+        const int key = 16 * j2 + kkey;
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(ka + key * HD * 2 + (((2 * kk + k_pc) ^ (key & 7)) << 4), b0, b1, b2, b3);
+        mma16816(sc[2 * j2], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b0, b1);
+        mma16816(sc[2 * j2 + 1], qa[kk][0], qa[kk][1], qa[kk][2], qa[kk][3], b2, b3);
       }
-      float corr[2], mnew[2];
+    }
+    float mx[2] = {-INFINITY, -INFINITY};
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        mnew[h2] = fmaxf(m_r[h2], mx[h2]);
-        corr[h2] = (m_r[h2] == -INFINITY) ? 0.f : exp2f(m_r[h2] - mnew[h2]);
-        m_r[h2] = mnew[h2];
-      }
-      float ls[2] = {0.f, 0.f};
-      uint32_t pa[4];
+    for (int j = 0; j < NT; ++j) {
 #pragma unroll
-      for (int t2 = 0; t2 < 2; ++t2) {
-        const float p0 = exp2f(s[t2][0] - mnew[0]), p1 = exp2f(s[t2][1] - mnew[0]);
-        const float p2 = exp2f(s[t2][2] - mnew[1]), p3 = exp2f(s[t2][3] - mnew[1]);
-        ls[0] += p0 + p1;
-        ls[1] += p2 + p3;
-        pa[2 * t2] = pack2_bf16(p0, p1);
-        pa[2 * t2 + 1] = pack2_bf16(p2, p3);
+      for (int e = 0; e < 4; ++e) {
+        const int key = 8 * j + 2 * tig + (e & 1);
+        sc[j][e] = key < nk ? sc[j][e] * sl2 : -INFINITY;
+        mx[e >> 1] = fmaxf(mx[e >> 1], sc[j][e]);
       }
+    }
+    float corr[2], mnew[2], ls[2] = {0.f, 0.f};
 #pragma unroll
-      for (int h2 = 0; h2 < 2; ++h2) {
-        ls[h2] += __shfl_xor_sync(0xffffffffu, ls[h2], 1);
-        ls[h2] += __shfl_xor_sync(0xffffffffu, ls[h2], 2);
-        l_r[h2] = l_r[h2] * corr[h2] + ls[h2];
-      }
+    for (int h2 = 0; h2 < 2; ++h2) {
+      mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 1));
+      mx[h2] = fmaxf(mx[h2], __shfl_xor_sync(0xffffffffu, mx[h2], 2));
+      mnew[h2] = fmaxf(m_r[h2], mx[h2]);
+      corr[h2] = (m_r[h2] == -INFINITY) ? 0.f : exp2f(m_r[h2] - mnew[h2]);
+      m_r[h2] = mnew[h2];
+    }
+    uint32_t pa[NT][2];
 #pragma unroll
-      for (int i = 0; i < DT; ++i) {
-        o[i][0] *= corr[0];
-        o[i][1] *= corr[0];
-        o[i][2] *= corr[1];
-        o[i][3] *= corr[1];
-      }
-      const uint32_t v_lane = va + (kt + vkey) * HD * 2;
-      const int v_sw = (kt + vkey) & 7;
+    for (int j = 0; j < NT; ++j) {
+      const float p0 = exp2f(sc[j][0] - mnew[0]), p1 = exp2f(sc[j][1] - mnew[0]);
+      const float p2 = exp2f(sc[j][2] - mnew[1]), p3 = exp2f(sc[j][3] - mnew[1]);
+      ls[0] += p0 + p1;
+      ls[1] += p2 + p3;
+      pa[j][0] = pack2_bf16(p0, p1);
+      pa[j][1] = pack2_bf16(p2, p3);
+    }
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      ls[h2] += __shfl_xor_sync(0xffffffffu, ls[h2], 1);
+      ls[h2] += __shfl_xor_sync(0xffffffffu, ls[h2], 2);
+      l_r[h2] = l_r[h2] * corr[h2] + ls[h2];
+    }
+#pragma unroll
+    for (int i = 0; i < DT; ++i) {
+      o[i][0] *= corr[0];
+      o[i][1] *= corr[0];
+      o[i][2] *= corr[1];
+      o[i][3] *= corr[1];
+    }
+    // O += P V, 16 keys at a time (A fragment = the S accumulators of two 8-key tiles)
+#pragma unroll
+    for (int j2 = 0; j2 < NT / 2; ++j2) {
+      const int key = 16 * j2 + vkey;
+      const uint32_t v_lane = va + key * HD * 2;
 #pragma unroll
       for (int i = 0; i < DT; i += 2) {
         uint32_t b0, b1, b2, b3;
-        ldsm_x4_t(v_lane + (((i + v_pc) ^ v_sw) << 4), b0, b1, b2, b3);
-        mma16816(o[i], pa[0], pa[1], pa[2], pa[3], b0, b1);
-        mma16816(o[i + 1], pa[0], pa[1], pa[2], pa[3], b2, b3);
+        ldsm_x4_t(v_lane + (((i + v_pc) ^ (key & 7)) << 4), b0, b1, b2, b3);
+        mma16816(o[i], pa[2 * j2][0], pa[2 * j2][1], pa[2 * j2 + 1][0], pa[2 * j2 + 1][1], b0, b1);
+        mma16816(o[i + 1], pa[2 * j2][0], pa[2 * j2][1], pa[2 * j2 + 1][0], pa[2 * j2 + 1][1], b2, b3);
       }
     }
     // the buffer is refilled with tile it + 2 once every warp is done with it
@@ -621,10 +637,10 @@ __global__ void __launch_bounds__(128) battn_kernel(const __grid_constant__ BAtt
     }
   }
   if (!good) return;
-  // normalise and store o rows: query row R = row0 + r -> head g*G + R / T, token R % T
+  // normalise and store o rows: query row R -> head g*G + R / T, token R % T
 #pragma unroll
   for (int h2 = 0; h2 < 2; ++h2) {
-    const int R = row0 + r0 + (lane >> 2) + 8 * h2;
+    const int R = row0 + r0 + gid + 8 * h2;
     if (R - row0 >= nrows) continue;
     const float inv = 1.0f / l_r[h2];
     const int head = g * G + R / T, t = R % T;
@@ -632,7 +648,7 @@ __global__ void __launch_bounds__(128) battn_kernel(const __grid_constant__ BAtt
     const int K = p.Hq * HD;
 #pragma unroll
     for (int i = 0; i < DT; ++i) {
-      const int c = head * HD + 8 * i + 2 * (lane & 3);
+      const int c = head * HD + 8 * i + 2 * tig;
       *reinterpret_cast<uint32_t*>(p.o_act + act128_off(m, c, K)) =
           pack2_bf16(o[i][2 * h2] * inv, o[i][2 * h2 + 1] * inv);
     }
@@ -671,8 +687,8 @@ cudaError_t launch_binproj(const BRowParams& p, cudaStream_t st) {
   return cudaGetLastError();
 }
 
-cudaError_t launch_bnorm(const BRowParams& p, cudaStream_t st) {
-  bnorm_kernel<<<(p.M + 7) / 8, 256, 0, st>>>(p);
+cudaError_t launch_bresnorm(const BRowParams& p, cudaStream_t st) {
+  bresnorm_kernel<<<(p.M + 7) / 8, 256, 0, st>>>(p);
   return cudaGetLastError();
 }
 
@@ -685,7 +701,7 @@ cudaError_t launch_boutproj(const BRowParams& p, cudaStream_t st) {
 }
 
 cudaError_t launch_battn(const BAttnParams& p, cudaStream_t st) {
-  const size_t smem = 1024 + (size_t)5 * 64 * p.hd * 2 + 64;
+  const size_t smem = 1024 + (size_t)4 * kAttnKeys * p.hd * 2 + 64;
   const int grid = p.B * p.Hkv * p.qblocks;
   cudaError_t e;
   if (p.hd == 128) {

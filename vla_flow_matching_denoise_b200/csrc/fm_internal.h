@@ -132,7 +132,7 @@ struct BGemmParams {
   const uint8_t* A;          // ACT128 [Mp/128][K/64]
   const uint8_t* W;          // packed [N/BN][K/64] chunks of BN x 64
   int K, N, M, Mp;           // reduction, output channels, valid rows (B*T), padded rows
-  // BE_RESID: h[m][n] += gate[n] * D[m][n]   (fp32, row stride N)
+  // BE_RESID: h[m][n] = gate[n] * D[m][n]   (fp32 residual branch, row stride N)
   float* h;
   const float* gate;
   // BE_SWIGLU: tile j holds gate rows 128j.. then up rows 128j..; u = SiLU(g) up
@@ -159,6 +159,7 @@ struct BRowParams {          // in-proj, AdaRMSNorm, out-proj + Euler (row kerne
   const uint16_t* w_out;     // [A][d]
   const float* out_bias;     // [A] or null
   float* h;                  // [Mp][d] fp32 residual
+  const float* delta;        // [Mp][d] fp32 gated branch added to h (residual + norm kernel)
   const float* s;            // norm scale and shift [d]
   const float* b;
   uint16_t* z;               // ACT128 [Mp/128][d/64]

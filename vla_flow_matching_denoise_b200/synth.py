@@ -98,6 +98,8 @@ WORKLOADS: Dict[str, ExpertShape] = {
     # Four layers of the LingBot-shaped expert: the profiling case (same layer
     # shape, ~200 MB on the device, weights still larger than L2).
     "lingbot_l4_p256_n10": ExpertShape(4, 1024, 16, 2, 128, 4096, 75, 256, 10),
+    # The same four layers with 64 requests: the profiling case of the batched path.
+    "lingbot_l4_b64_p256_n10": ExpertShape(4, 1024, 16, 2, 128, 4096, 75, 256, 10, batch=64),
 }
 
 
