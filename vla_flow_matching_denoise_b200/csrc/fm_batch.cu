@@ -21,6 +21,7 @@
 #include <cuda_bf16.h>
 #include <cstddef>
 #include <cstdint>
+#include <utility>
 
 #include "fm_internal.h"
 #include "fm_launch.h"
@@ -204,10 +205,24 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  grid_dep_launch();
 
   if (warp == 0) {
     if (lane == 0) {
       const uint64_t pol = policy_evict_last();   // A and W are both re-read by other CTAs
+      // The weights do not depend on the previous kernel: the first stages'
+      // weight chunks are requested before waiting for it.
+      int npre = 0;
+      if ((int)blockIdx.x < ntiles) {
+        npre = nkb < C::kStages ? nkb : C::kStages;
+        const uint8_t* w0 = p.W + (size_t)((int)blockIdx.x / MT) * nkb * C::kW;
+        for (int j = 0; j < npre; ++j) {
+          mbar_expect_tx(smem_u32(&full[j]), C::kW);
+          bulk_g2s(smem_u32(ring + (size_t)j * C::kStage + C::kA), w0 + (size_t)j * C::kW, C::kW,
+                   smem_u32(&full[j]), pol);
+        }
+      }
+      grid_dep_wait();
       uint32_t it = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x) {
@@ -222,9 +237,14 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
             break;
           }
           uint8_t* dst = ring + (size_t)s * C::kStage;
-          mbar_arrive_expect_tx(smem_u32(&full[s]), C::kStage);
-          bulk_g2s(smem_u32(dst), a_src + (size_t)kb * C::kA, C::kA, smem_u32(&full[s]), pol);
-          bulk_g2s(smem_u32(dst + C::kA), w_src + (size_t)kb * C::kW, C::kW, smem_u32(&full[s]), pol);
+          if ((int)it < npre) {
+            mbar_arrive_expect_tx(smem_u32(&full[s]), C::kA);
+            bulk_g2s(smem_u32(dst), a_src + (size_t)kb * C::kA, C::kA, smem_u32(&full[s]), pol);
+          } else {
+            mbar_arrive_expect_tx(smem_u32(&full[s]), C::kStage);
+            bulk_g2s(smem_u32(dst), a_src + (size_t)kb * C::kA, C::kA, smem_u32(&full[s]), pol);
+            bulk_g2s(smem_u32(dst + C::kA), w_src + (size_t)kb * C::kW, C::kW, smem_u32(&full[s]), pol);
+          }
         }
       }
       // every issued copy must land before the CTA may exit
@@ -268,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
       mbar_wait(smem_u32(drain), 0, budget);
     }
   } else {
+    grid_dep_wait();                             // outputs and epilogue operands follow the previous kernel
     const int q4 = warp & 3;                     // TMEM lane quarter this warp may read
     const int row = 32 * q4 + lane;
     const int P = (EPI == BE_QKV) ? *p.P_dev : 0;
@@ -308,6 +329,8 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
   __shared__ float xs[kRowsIn][128];
   __shared__ float red[8][kRowsIn];
   __shared__ float rstd[kRowsIn];
+  grid_dep_launch();
+  grid_dep_wait();
   const int m0 = blockIdx.x * kRowsIn;
   const int tid = threadIdx.x, A = p.A, d = p.d;
   for (int i = tid; i < kRowsIn * A; i += 256) {
@@ -374,6 +397,8 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
 // Gated residual + AdaRMSNorm, one warp per row: h += delta, then (unless z
 // is null) z = bf16(h rstd (1 + s) + b) in ACT128.
 __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ BRowParams p) {
+  grid_dep_launch();
+  grid_dep_wait();
   const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (m >= p.M) return;
@@ -412,6 +437,8 @@ __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ B
 // 16 row sums reduced by shuffles.
 __global__ void __launch_bounds__(256) boutproj_kernel(const __grid_constant__ BRowParams p) {
   extern __shared__ float ys[];   // [kRowsIn][d]
+  grid_dep_launch();
+  grid_dep_wait();
   const int m0 = blockIdx.x * kRowsIn;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = p.d, A = p.A;
@@ -481,6 +508,8 @@ __global__ void __launch_bounds__(128, 3) battn_kernel(const __grid_constant__ B
   uint8_t* vbuf = sm + 2 * TILE;                  // [2] V tiles
   uint64_t* bars = reinterpret_cast<uint64_t*>(vbuf + 2 * TILE);   // [2] tile barriers
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  grid_dep_launch();
+  grid_dep_wait();
   const int qb = blockIdx.x % p.qblocks;
   const int g = (blockIdx.x / p.qblocks) % p.Hkv;
   const int b = blockIdx.x / (p.qblocks * p.Hkv);
@@ -655,6 +684,25 @@ __global__ void __launch_bounds__(128, 3) battn_kernel(const __grid_constant__ B
   }
 }
 
+// Launch with programmatic stream serialization: the kernel may start while
+// the previous one in the stream finishes (it waits with griddepcontrol.wait
+// before touching what that kernel writes).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(Params...), int grid, int block, size_t smem, cudaStream_t st,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(block, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <int BN, int EPI>
 cudaError_t launch_bgemm_t(const BGemmParams& p, int n_sms, cudaStream_t st) {
   using C = BCfg<BN>;
@@ -663,8 +711,7 @@ cudaError_t launch_bgemm_t(const BGemmParams& p, int n_sms, cudaStream_t st) {
   if (e != cudaSuccess) return e;
   const int ntiles = (p.Mp / kBM) * (p.N / BN);
   const int grid = ntiles < n_sms ? ntiles : n_sms;
-  bgemm_kernel<BN, EPI><<<grid, kThreads, C::kSmem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(bgemm_kernel<BN, EPI>, grid, kThreads, C::kSmem, st, p);
 }
 
 }  // namespace
@@ -683,21 +730,18 @@ cudaError_t launch_bgemm(const BGemmParams& p, int epi, int n_sms, cudaStream_t 
 }
 
 cudaError_t launch_binproj(const BRowParams& p, cudaStream_t st) {
-  binproj_kernel<<<(p.M + kRowsIn - 1) / kRowsIn, 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(binproj_kernel, (p.M + kRowsIn - 1) / kRowsIn, 256, 0, st, p);
 }
 
 cudaError_t launch_bresnorm(const BRowParams& p, cudaStream_t st) {
-  bresnorm_kernel<<<(p.M + 7) / 8, 256, 0, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(bresnorm_kernel, (p.M + 7) / 8, 256, 0, st, p);
 }
 
 cudaError_t launch_boutproj(const BRowParams& p, cudaStream_t st) {
   const size_t smem = (size_t)kRowsIn * p.d * sizeof(float);
   cudaError_t e = cudaFuncSetAttribute(boutproj_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  boutproj_kernel<<<(p.M + kRowsIn - 1) / kRowsIn, 256, smem, st>>>(p);
-  return cudaGetLastError();
+  return launch_pdl(boutproj_kernel, (p.M + kRowsIn - 1) / kRowsIn, 256, smem, st, p);
 }
 
 cudaError_t launch_battn(const BAttnParams& p, cudaStream_t st) {
@@ -707,13 +751,13 @@ cudaError_t launch_battn(const BAttnParams& p, cudaStream_t st) {
   if (p.hd == 128) {
     e = cudaFuncSetAttribute(battn_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    battn_kernel<128><<<grid, 128, smem, st>>>(p);
+    e = launch_pdl(battn_kernel<128>, grid, 128, smem, st, p);
   } else {
     e = cudaFuncSetAttribute(battn_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    battn_kernel<64><<<grid, 128, smem, st>>>(p);
+    e = launch_pdl(battn_kernel<64>, grid, 128, smem, st, p);
   }
-  return cudaGetLastError();
+  return e;
 }
 
 }  // namespace fm

@@ -453,6 +453,7 @@ __device__ __noinline__ void push_partials(Ctx& c, const GemmView& v) {
   Ctrl* const ctl = c.ctl;
   const long long budget = c.p->spin_budget;
   const int tid = c.tid;
+  tmark(c, 12);
   if (!wait_ab(smem_u32(&ctl->mma_done), c.gemm_count & 1, budget, &ctl->abort)) {
     fail(c, E_MMA_DONE);
     return;
@@ -474,6 +475,7 @@ __device__ __noinline__ void push_partials(Ctx& c, const GemmView& v) {
     for (int i = 0; i < 4; ++i)
       if (i < nb) tmem_ld16(tb + cb + 16 * i, x[i]);
     tmem_ld_wait();
+    if (cb == 0) tmark(c, 13);
     if (valid) {
       int o = cb / own, lc = cb - o * own;
       float* rowp = stg + (o * kRecvRows + row) * ownp;
@@ -590,6 +592,7 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
   const GemmView v = gemm_view(c, G_QKV);
   if (v.ng == 0) return;
   gemm_begin(c, v, p.z_a);
+  tmark(c, 11);
   load_rstd(c, p.sumsq_a);
   const int T = p.T, hd = p.hd, half = hd / 2, G = p.Hq / p.Hkv;
   const int qn = p.Hq * hd, kn = p.Hkv * hd, N = p.g[G_QKV].N;
@@ -907,6 +910,7 @@ __device__ __noinline__ void residual_phase(Ctx& c, int g, int l, const uint16_t
   const GemmView v = gemm_view(c, g);
   if (v.ng == 0) return;
   gemm_begin(c, v, act);
+  tmark(c, 11);
   const int T = c.p->T, d = c.p->d;
   const int tid = c.tid;
   const int t = tid >> 1, hf = tid & 1;
@@ -960,6 +964,7 @@ __device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
   const GemmView v = gemm_view(c, G_GU);
   if (v.ng == 0) return;
   gemm_begin(c, v, p.z_f);
+  tmark(c, 11);
   load_rstd(c, p.sumsq_f);
   push_partials(c, v);
   if (!c.ok) return;
