@@ -203,7 +203,9 @@ def cpu_baseline(shape: synth.ExpertShape, n_sample: int, seed: int = 0):
             "sample": r.sample_text(n_sample, el)}
 
 
-def dist_setup(gpus: int):
+def dist_setup(gpus: int, backend: str = "nccl"):
+    """One process per GPU (torchrun sets RANK / WORLD_SIZE / LOCAL_RANK /
+    MASTER_*).  Returns (world size, rank, local rank, torch.distributed or None)."""
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
@@ -211,9 +213,31 @@ def dist_setup(gpus: int):
     if ws > 1:
         import torch.distributed as dist
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
         pg = dist
     return ws, rank, local, pg
+
+
+def max_over_ranks(value: float, pg, device) -> float:
+    """The largest of the ranks' values (every rank gets it)."""
+    if pg is None:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_inputs(shape: synth.ExpertShape, rank: int):
+    """Each rank's own requests: prefix K/V and x0 seeded by the rank (the
+    weights are the same on every rank)."""
+    kp, vp = synth.make_prefix(shape, seed=rank)
+    return kp, vp, synth.make_x0(shape, seed=rank)
+
+
+def job_value(ws: int, batch: int, steps: int, calls: int, ms_total: float) -> float:
+    """Euler steps per second of the whole job: every rank's requests count."""
+    return ws * batch * steps * calls / (ms_total / 1000.0)
 
 
 def run_reference(args, shape):
@@ -263,8 +287,7 @@ def main():
 
     B, n = shape.batch, shape.steps
     raw = synth.make_weights(shape, seed=0)
-    kp, vp = synth.make_prefix(shape, seed=rank)
-    x0 = synth.make_x0(shape, seed=rank)
+    kp, vp, x0 = rank_inputs(shape, rank)
     e = Expert(shape, raw, device=local)
     del raw
     e.set_prefix(kp, vp, B, shape.prefix_len)
@@ -294,14 +317,9 @@ def main():
             e.denoise(x_dev, n, out=out_dev)
         ev1.record(stream)
         barrier()
-    ms_total = ev0.elapsed_time(ev1)
-    if pg is not None:
-        t = torch.tensor([ms_total], device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_total = float(t.item())
+    ms_total = max_over_ranks(ev0.elapsed_time(ev1), pg, "cuda")
     ms_call = ms_total / args.steps
-    euler_total = ws * B * n * args.steps
-    value = euler_total / (ms_total / 1000.0)
+    value = job_value(ws, B, n, args.steps, ms_total)
 
     # end to end through the public API with pinned host buffers
     xh = torch.from_numpy(x0).pin_memory()
@@ -314,12 +332,8 @@ def main():
         e.denoise(xh, n, out=oh)
     ev1.record(stream)
     barrier()
-    ms_e2e = ev0.elapsed_time(ev1)
-    if pg is not None:
-        t = torch.tensor([ms_e2e], device="cuda")
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms_e2e = float(t.item())
-    e2e_value = euler_total / (ms_e2e / 1000.0)
+    ms_e2e = max_over_ranks(ev0.elapsed_time(ev1), pg, "cuda")
+    e2e_value = job_value(ws, B, n, args.steps, ms_e2e)
 
     # the loop kernel alone (event-timed, outside the graph)
     ms_time_mlp, ms_loop = e.profile(B, n, max(3, min(args.steps, 10)))
@@ -335,6 +349,8 @@ def main():
     e.close()
 
     if rank != 0:
+        if pg is not None:
+            pg.destroy_process_group()
         return
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
