@@ -52,6 +52,18 @@ namespace fm {
 
 namespace {
 
+// This CTA's share of one linear.
+struct GemmView {
+  int ng;        // channels of its n-group (0: idle cluster)
+  int KS, ks, grp;
+  int own;       // owned output columns
+  int ownp;      // row stride (floats) of the staging / receive blocks, multiple of 4
+  int nchunk;
+  int base;      // first owned packed channel (gate_up: first owned u column)
+  int pbase;     // index of the first owned column in the layer's scale table
+  uint32_t recv_off;   // byte offset of the receive buffer in the work region
+};
+
 struct Ctrl {
   uint64_t full[kRingSlots];
   uint64_t empty[kRingSlots];
@@ -66,6 +78,7 @@ struct Ctrl {
   int abort;
   alignas(16) float rstd[kRows];
   alignas(16) float red[8][kRows];   // written with float4 stores
+  GemmView views[4];                 // this CTA's share of each linear (fixed per launch)
 };
 static_assert(offsetof(Ctrl, red) % 16 == 0 && offsetof(Ctrl, rstd) % 16 == 0, "vector alignment");
 
@@ -386,37 +399,30 @@ __device__ __forceinline__ const float* mod_vec(const StepParams& p, int step, i
 
 constexpr int kMaxPairs = 4;    // owned column pairs per residual thread (checked by the planner)
 constexpr int kAuxBytes = 8 * 1024;   // end of the work region: per-thread epilogue operands
+constexpr int kAuxRows = kAuxBytes / (128 * 8);   // float2 rows per compute thread
 
-// This CTA's share of one linear.
-struct GemmView {
-  int ng;        // channels of its n-group (0: idle cluster)
-  int KS, ks, grp;
-  int own;       // owned output columns
-  int ownp;      // row stride (floats) of the staging / receive blocks, multiple of 4
-  int nchunk;
-  int base;      // first owned packed channel (gate_up: first owned u column)
-  int pbase;     // index of the first owned column in the layer's scale table
-  uint32_t recv_off;   // byte offset of the receive buffer in the work region
-};
-
-__device__ __forceinline__ GemmView gemm_view(const Ctx& c, int g) {
-  const GemmPlan& gp = c.p->g[g];
+// Computed once per launch into shared memory (make_views); the phases read
+// it from there instead of re-deriving it from the launch parameters.
+__device__ GemmView compute_view(const StepParams& p, int g, int cluster, int rank) {
+  const GemmPlan& gp = p.g[g];
   GemmView v;
-  v.ng = gp.ng[c.cluster];
+  v.ng = gp.ng[cluster];
   v.KS = gp.KS;
-  v.ks = c.rank % gp.KS;
-  v.grp = c.rank / gp.KS;
+  v.ks = rank % gp.KS;
+  v.grp = rank / gp.KS;
   v.own = v.ng / gp.KS;
   v.ownp = (v.own + 3) & ~3;
   v.nchunk = gp.nchunk;
-  v.base = (g == G_GU) ? gp.ch_off[c.cluster] + v.grp * (v.ng / 2) + v.ks * (v.own / 2)
-                       : gp.ch_off[c.cluster] + v.grp * v.ng + v.ks * v.own;
-  v.pbase = (g == G_GU) ? 2 * gp.ch_off[c.cluster] + v.grp * v.ng + v.ks * v.own : v.base;
+  v.base = (g == G_GU) ? gp.ch_off[cluster] + v.grp * (v.ng / 2) + v.ks * (v.own / 2)
+                       : gp.ch_off[cluster] + v.grp * v.ng + v.ks * v.own;
+  v.pbase = (g == G_GU) ? 2 * gp.ch_off[cluster] + v.grp * v.ng + v.ks * v.own : v.base;
   const uint32_t a_bytes = (uint32_t)v.nchunk * 8192u;
   const uint32_t s_bytes = (uint32_t)(v.KS * kRecvRows * v.ownp * 4);
   v.recv_off = ((a_bytes > s_bytes ? a_bytes : s_bytes) + 15u) & ~15u;
   return v;
 }
+
+__device__ __forceinline__ GemmView gemm_view(const Ctx& c, int g) { return c.ctl->views[g]; }
 
 // Row scales of two adjacent owned columns (E4M3 weights); 1 for bf16, where
 // the product is exact and leaves the result unchanged.
@@ -462,35 +468,44 @@ __device__ __noinline__ void push_partials(Ctx& c, const GemmView& v) {
   tc_fence_after();
   tmark(c, 1);
   const int ng = v.ng, own = v.own, ownp = v.ownp;
+  // M = 64 accumulator: rows 16 sp .. 16 sp + 15 sit in TMEM lanes 32 sp ..
+  // 32 sp + 15 of this warp's quarter; 16x256b loads spread them over all 32
+  // threads (rows r_lo, r_lo + 8; column pairs 2 (lane % 4) + 8 j).
   const int sp = c.warp & 3;
-  const int row = 16 * sp + c.lane;
-  const bool valid = c.lane < 16 && row < kRecvRows;
+  const int r_lo = 16 * sp + (c.lane >> 2), r_hi = r_lo + 8;
+  const bool ok_lo = r_lo < kRecvRows, ok_hi = r_hi < kRecvRows;
+  const int cq = 2 * (c.lane & 3);
   const uint32_t tb = c.tmem + ((uint32_t)(32 * sp) << 16);
   float* const stg = reinterpret_cast<float*>(c.work);
+  // this thread's columns are cq, cq + 8, ...: their owner block and column
+  // inside it advance incrementally (owners hold an even number of columns,
+  // so a column pair never straddles two owners)
+  float* blk = stg;
+  int lc = cq;
+  while (lc >= own) {
+    lc -= own;
+    blk += kRecvRows * ownp;
+  }
+  blk += lc;
 #pragma unroll 1
   for (int cb = 0; cb < ng; cb += 64) {
-    float x[4][16];
-    const int nb = min(4, (ng - cb) >> 4);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      if (i < nb) tmem_ld16(tb + cb + 16 * i, x[i]);
+    float x[2][16];
+    tmem_ld_16x256b_x4(tb + cb, x[0]);
+    if (cb + 32 < ng) tmem_ld_16x256b_x4(tb + cb + 32, x[1]);
     tmem_ld_wait();
     if (cb == 0) tmark(c, 13);
-    if (valid) {
-      int o = cb / own, lc = cb - o * own;
-      float* rowp = stg + (o * kRecvRows + row) * ownp;
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (i >= nb) break;
+    for (int h = 0; h < 2; ++h) {
 #pragma unroll
-        for (int q = 0; q < 8; ++q) {
-          if (lc >= own) {
-            ++o;
-            lc -= own;
-            rowp += kRecvRows * ownp;
-          }
-          *reinterpret_cast<float2*>(rowp + lc) = make_float2(x[i][2 * q], x[i][2 * q + 1]);
-          lc += 2;
+      for (int j = 0; j < 4; ++j) {
+        if (cb + 32 * h + 8 * j >= ng) break;
+        if (ok_lo) *reinterpret_cast<float2*>(blk + r_lo * ownp) = make_float2(x[h][4 * j], x[h][4 * j + 1]);
+        if (ok_hi) *reinterpret_cast<float2*>(blk + r_hi * ownp) = make_float2(x[h][4 * j + 2], x[h][4 * j + 3]);
+        lc += 8;
+        blk += 8;
+        while (lc >= own) {
+          lc -= own;
+          blk += kRecvRows * ownp - own;
         }
       }
     }
@@ -613,12 +628,20 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
     dst = (kind == 1 ? p.kcache : p.vcache) + (((size_t)l * p.B_cap + p.b) * p.Hkv + head) * p.S_max * hd;
     row_off = P;
   }
-  // stage the rotation of every row of this thread
+  // stage the rotation of every row of this thread (all loads in flight at
+  // once; the planner keeps the rows per thread within kAuxRows)
   float2* aux = reinterpret_cast<float2*>(c.work + kWorkBytes - kAuxBytes) + c.tid;
   if (act && kind < 2) {
     const float2* rope = reinterpret_cast<const float2*>(p.rope) + ri;
-#pragma unroll 1
-    for (int t = pa.t0, k = 0; t < T; t += pa.dt, ++k) aux[k * 128] = rope[t * half];
+    float2 rv[kAuxRows];
+#pragma unroll
+    for (int k = 0; k < kAuxRows; ++k) {
+      const int t = pa.t0 + k * pa.dt;
+      if (t < T) rv[k] = rope[t * half];
+    }
+#pragma unroll
+    for (int k = 0; k < kAuxRows; ++k)
+      if (pa.t0 + k * pa.dt < T) aux[k * 128] = rv[k];
   }
   const float2 sc = act ? wscale2(c, G_QKV, l, v.pbase + 2 * pa.pr) : make_float2(1.f, 1.f);
   push_partials(c, v);
@@ -1212,6 +1235,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_cons
     mbar_init(smem_u32(&ctl->drain), 1);
     mbar_init(smem_u32(&ctl->xsync), kClusterSize);
     ctl->abort = 0;
+    for (int g = 0; g < 4; ++g) ctl->views[g] = compute_view(p, g, cluster, (int)cluster_rank());
     fence_mbar_init();
   }
   if (warp == 1) {
