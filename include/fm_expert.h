@@ -137,6 +137,21 @@ fm_status fm_expert_create(const fm_config *cfg, const fm_weights *w, int device
 fm_status fm_set_prefix(fm_expert *h, const uint16_t *const *k, const uint16_t *const *v,
                         int batch, int prefix_len, void *stream);
 
+/* As fm_set_prefix, with a prefix length per request: k[l], v[l] point to
+ * bf16 bits [batch, p_pad, H_kv, hd] (host or device) in which request b
+ * holds prefix_lens[b] valid rows (0 <= prefix_lens[b] <= p_pad <=
+ * max_prefix; the remaining rows are padding and are never read).  Request
+ * b then attends to its P_b prefix keys plus the chunk, and its chunk tokens
+ * take RoPE positions P_b .. P_b+T-1.  prefix_lens is a host array of `batch`
+ * ints; the lengths are stored on the device, so a graph captured for this
+ * (batch, steps) serves any lengths without recapture ("LingBot-VLA v2
+ * Examples", Configuration / CUDA Graph: different language padding masks
+ * reuse the same denoising graph; "api.py", state_prompt_mode "fixed": one
+ * graph at the padded length masked by a device-side valid length).
+ * FM_ERR_INVALID_ARG for a length outside [0, p_pad] or p_pad > max_prefix. */
+fm_status fm_set_prefix_varlen(fm_expert *h, const uint16_t *const *k, const uint16_t *const *v,
+                               int batch, const int *prefix_lens, int p_pad, void *stream);
+
 /* Denoise `batch` chunks: x0 and out are fp32 [batch, T, A], host or device
  * (independently); out may alias x0.  Runs the time MLP once, then `steps`
  * Euler steps from t = 1 to t = 0 ("LingBot-VLA on Thor (sm_110)", §1: the

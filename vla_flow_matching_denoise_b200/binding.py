@@ -25,7 +25,7 @@ STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_NOT_READY", 3: "FM_ERR
           4: "FM_ERR_CUDA", 5: "FM_ERR_TIMEOUT", 6: "FM_ERR_UNSUPPORTED"}
 
 # Every symbol include/fm_expert.h declares.
-EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity", "fm_time_modulation",
+EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_set_prefix_varlen", "fm_denoise", "fm_velocity", "fm_time_modulation",
            "fm_trace_bytes", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
            "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
            "fm_expert_destroy", "fm_last_error", "fm_status_string",
@@ -86,6 +86,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_profile_denoise.argtypes = [vp, ip, ip, ip, vp, vp]
     lib.fm_profile_phases.argtypes = [vp, ip, vp, ctypes.POINTER(sz), vp]
     lib.fm_time_modulation_noalloc.argtypes = [vp, vp, ip, ip, ip, vp, vp]
+    lib.fm_set_prefix_varlen.argtypes = [vp, vp, vp, ip, vp, ip, vp]
     lib.fm_get_geometry.argtypes = [vp, ctypes.POINTER(ip), ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.fm_expert_destroy.argtypes = [vp]
     lib.fm_expert_destroy.restype = sz
@@ -96,7 +97,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_abi_version.restype = ip
     for name in ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity",
                  "fm_time_modulation", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
-                 "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc"):
+                 "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
+                 "fm_set_prefix_varlen"):
         getattr(lib, name).restype = ip
     _lib = lib
     return lib
@@ -190,6 +192,16 @@ class Expert:
         kp = (ctypes.c_void_p * L)(*[_ptr(x) for x in k])
         vp = (ctypes.c_void_p * L)(*[_ptr(x) for x in v])
         self._check("fm_set_prefix", self.lib.fm_set_prefix(self.h, kp, vp, batch, prefix_len, _stream(stream)))
+
+    def set_prefix_varlen(self, k: Sequence, v: Sequence, batch: int, prefix_lens: Sequence[int], p_pad: int,
+                          stream=None):
+        """k[l], v[l]: [batch, p_pad, H_kv, hd] bf16 bits; request b uses its first prefix_lens[b] rows."""
+        L = self.shape.n_layers
+        kp = (ctypes.c_void_p * L)(*[_ptr(x) for x in k])
+        vp = (ctypes.c_void_p * L)(*[_ptr(x) for x in v])
+        lens = (ctypes.c_int * batch)(*[int(x) for x in prefix_lens])
+        self._check("fm_set_prefix_varlen", self.lib.fm_set_prefix_varlen(self.h, kp, vp, batch, lens, p_pad,
+                                                                           _stream(stream)))
 
     def denoise(self, x0, steps: int, out=None, stream=None):
         """x0: fp32 [B, T, A] numpy (host) or torch (device).  Returns `out`."""

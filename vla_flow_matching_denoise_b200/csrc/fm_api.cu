@@ -102,7 +102,7 @@ struct fm_expert {
   uint32_t* err_word = nullptr;
   int S_max = 0;
   int prefix_batch = 0;   // batch of the last fm_set_prefix (0 = none)
-  int prefix_len = 0;
+  std::vector<int> prefix_lens;   // per request, host copy of P_dev
   std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
   std::map<std::pair<int, int>, cudaGraph_t> graph_defs;
 };
@@ -917,8 +917,8 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
   } while (0)
   ALLOC_OR_BAIL(h->mod, (size_t)c.max_steps * h->n_mod * 4);
   ALLOC_OR_BAIL(h->h1_act, (size_t)kRows * d * 2);
-  ALLOC_OR_BAIL(h->rope, T * c.head_dim * 4);
-  ALLOC_OR_BAIL(h->P_dev, 4);
+  ALLOC_OR_BAIL(h->rope, B * T * c.head_dim * 4);
+  ALLOC_OR_BAIL(h->P_dev, B * 4);
   ALLOC_OR_BAIL(h->x, B * T * A * 4);
   ALLOC_OR_BAIL(h->vbuf, B * T * A * 4);
   ALLOC_OR_BAIL(h->h_a, T * d * 4);
@@ -955,27 +955,27 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
   return FM_OK;
 }
 
-fm_status fm_set_prefix(fm_expert* h, const uint16_t* const* k, const uint16_t* const* v, int batch,
-                        int prefix_len, void* stream) {
-  if (!h) return FM_ERR_INVALID_ARG;
+namespace {
+
+// Copies the prefix K/V of `batch` requests (k[l], v[l]: [B, p_pad, H_kv, hd],
+// request b valid for its first lens[b] rows) into the cache and stores the
+// lengths and the chunk's RoPE table on the device.
+fm_status set_prefix_impl(fm_expert* h, const uint16_t* const* k, const uint16_t* const* v, int batch,
+                          int p_pad, const std::vector<int>& lens, cudaStream_t st) {
   const fm_config& c = h->cfg;
-  if (batch < 1 || batch > c.max_batch)
-    return set_err(h, FM_ERR_INVALID_ARG, "batch %d outside [1, %d]", batch, c.max_batch);
-  if (prefix_len < 0 || prefix_len > c.max_prefix)
-    return set_err(h, FM_ERR_INVALID_ARG, "prefix_len %d outside [0, %d]", prefix_len, c.max_prefix);
-  if (prefix_len > 0 && (!k || !v)) return set_err(h, FM_ERR_INVALID_ARG, "k or v is NULL");
   CK(cudaSetDevice(h->device));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const size_t per = (size_t)batch * prefix_len * c.n_kv_heads * c.head_dim;
+  const size_t per = (size_t)batch * p_pad * c.n_kv_heads * c.head_dim;
   const size_t lay = (size_t)c.max_batch * c.n_kv_heads * h->S_max * c.head_dim;
   void* tmp = nullptr;
-  if (prefix_len > 0) {
+  if (p_pad > 0) {
     for (int l = 0; l < c.n_layers; ++l)
       if (!k[l] || !v[l]) return set_err(h, FM_ERR_INVALID_ARG, "prefix pointer of layer %d is NULL", l);
     CK(cudaMalloc(&tmp, per * 2 * 2));
   }
+  // lengths first: the copy kernels read them
+  CK(cudaMemcpyAsync(h->P_dev, lens.data(), (size_t)batch * 4, cudaMemcpyHostToDevice, st));
   fm_status out = FM_OK;
-  for (int l = 0; l < c.n_layers && prefix_len > 0; ++l) {
+  for (int l = 0; l < c.n_layers && p_pad > 0; ++l) {
     const uint16_t* srcs[2] = {k[l], v[l]};
     uint16_t* dsts[2] = {h->kcache + l * lay, h->vcache + l * lay};
     for (int i = 0; i < 2; ++i) {
@@ -986,7 +986,7 @@ fm_status fm_set_prefix(fm_expert* h, const uint16_t* const* k, const uint16_t* 
         if (e != cudaSuccess) { out = set_err(h, FM_ERR_CUDA, "prefix upload: %s", cudaGetErrorString(e)); break; }
         src = t;
       }
-      cudaError_t e = launch_kv_copy(src, batch, prefix_len, c.n_kv_heads, c.head_dim, h->S_max, dsts[i], st);
+      cudaError_t e = launch_kv_copy(src, batch, p_pad, h->P_dev, c.n_kv_heads, c.head_dim, h->S_max, dsts[i], st);
       if (e != cudaSuccess) { out = set_err(h, FM_ERR_CUDA, "kv copy: %s", cudaGetErrorString(e)); break; }
     }
     if (out != FM_OK) break;
@@ -998,12 +998,43 @@ fm_status fm_set_prefix(fm_expert* h, const uint16_t* const* k, const uint16_t* 
   }
   if (tmp) cudaFree(tmp);
   if (out != FM_OK) return out;
-  CK(cudaMemcpyAsync(h->P_dev, &prefix_len, 4, cudaMemcpyHostToDevice, st));
-  CK(launch_rope_table(c.chunk_len, c.head_dim, prefix_len, (double)c.rope_base, h->rope, st));
+  CK(launch_rope_table(batch, c.chunk_len, c.head_dim, h->P_dev, (double)c.rope_base, h->rope, st));
   CK(cudaStreamSynchronize(st));
   h->prefix_batch = batch;
-  h->prefix_len = prefix_len;
+  h->prefix_lens = lens;
   return FM_OK;
+}
+
+}  // namespace
+
+fm_status fm_set_prefix(fm_expert* h, const uint16_t* const* k, const uint16_t* const* v, int batch,
+                        int prefix_len, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (batch < 1 || batch > c.max_batch)
+    return set_err(h, FM_ERR_INVALID_ARG, "batch %d outside [1, %d]", batch, c.max_batch);
+  if (prefix_len < 0 || prefix_len > c.max_prefix)
+    return set_err(h, FM_ERR_INVALID_ARG, "prefix_len %d outside [0, %d]", prefix_len, c.max_prefix);
+  if (prefix_len > 0 && (!k || !v)) return set_err(h, FM_ERR_INVALID_ARG, "k or v is NULL");
+  return set_prefix_impl(h, k, v, batch, prefix_len, std::vector<int>(batch, prefix_len),
+                         static_cast<cudaStream_t>(stream));
+}
+
+fm_status fm_set_prefix_varlen(fm_expert* h, const uint16_t* const* k, const uint16_t* const* v, int batch,
+                               const int* prefix_lens, int p_pad, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (batch < 1 || batch > c.max_batch)
+    return set_err(h, FM_ERR_INVALID_ARG, "batch %d outside [1, %d]", batch, c.max_batch);
+  if (!prefix_lens) return set_err(h, FM_ERR_INVALID_ARG, "prefix_lens is NULL");
+  if (p_pad < 0 || p_pad > c.max_prefix)
+    return set_err(h, FM_ERR_INVALID_ARG, "p_pad %d outside [0, %d]", p_pad, c.max_prefix);
+  std::vector<int> lens(prefix_lens, prefix_lens + batch);
+  for (int b = 0; b < batch; ++b)
+    if (lens[b] < 0 || lens[b] > p_pad)
+      return set_err(h, FM_ERR_INVALID_ARG, "prefix_lens[%d] = %d outside [0, p_pad = %d]", b, lens[b], p_pad);
+  if (p_pad > 0 && (!k || !v)) return set_err(h, FM_ERR_INVALID_ARG, "k or v is NULL");
+  return set_prefix_impl(h, k, v, batch, p_pad, lens, static_cast<cudaStream_t>(stream));
 }
 
 static fm_status get_graph(fm_expert* h, int batch, int steps, cudaGraphExec_t* out) {
@@ -1198,7 +1229,7 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
         CK(cudaMemcpy(kvh.data(), cache + (size_t)g * h->S_max * hd, kvh.size() * 2, cudaMemcpyDeviceToHost));
         for (int t = 0; t < T; ++t)
           for (int e = 0; e < hd; ++e) {
-            const int row = h->prefix_len + t;
+            const int row = h->prefix_lens[0] + t;
             out[(size_t)t * kn + g * hd + e] = swz_get(kvh, (size_t)row * hd, row, e);
           }
       }

@@ -113,11 +113,12 @@ __device__ __forceinline__ void store_row16(uint16_t* rowp, int row, int e0, con
 }
 
 template <int BN>
-__device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt, int P) {
+__device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt) {
   const int hd = p.hd, half = hd / 2;
   const int qn = p.Hq * hd, kn = p.Hkv * hd, G = p.Hq / p.Hkv;
   const int b = valid ? m / p.T : 0, t = valid ? m % p.T : 0;
-  const float2* rope = reinterpret_cast<const float2*>(p.rope) + (size_t)t * half;
+  const int P = p.P_dev[b];   // this request's prefix length: chunk rows and RoPE positions follow it
+  const float2* rope = reinterpret_cast<const float2*>(p.rope) + ((size_t)b * p.T + t) * half;
 #pragma unroll 1
   for (int ho = 0; ho < BN; ho += hd) {
     const int col0 = nt * BN + ho;
@@ -291,7 +292,6 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
     grid_dep_wait();                             // outputs and epilogue operands follow the previous kernel
     const int q4 = warp & 3;                     // TMEM lane quarter this warp may read
     const int row = 32 * q4 + lane;
-    const int P = (EPI == BE_QKV) ? *p.P_dev : 0;
     uint32_t local = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
       const uint32_t acc = local & 1;
@@ -306,7 +306,7 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
       const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + acc * BN;
       if (EPI == BE_RESID) epi_resid<BN>(p, ta, m, valid, nt);
       else if (EPI == BE_SWIGLU) epi_swiglu<BN>(p, ta, m, valid, nt);
-      else epi_qkv<BN>(p, ta, m, valid, nt, P);
+      else epi_qkv<BN>(p, ta, m, valid, nt);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
@@ -514,7 +514,7 @@ __global__ void __launch_bounds__(128, 3) battn_kernel(const __grid_constant__ B
   const int g = (blockIdx.x / p.qblocks) % p.Hkv;
   const int b = blockIdx.x / (p.qblocks * p.Hkv);
   const int G = p.Hq / p.Hkv, T = p.T;
-  const int P = *p.P_dev;
+  const int P = p.P_dev[b];
   const int S = P + T;
   const int row0 = qb * 64;
   const int nrows = min(64, G * T - row0);

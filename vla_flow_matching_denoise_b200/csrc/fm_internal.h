@@ -64,7 +64,7 @@ struct StepParams {
   int L, d, Hq, Hkv, hd, F, A, T, S_max;
   int B_cap;                 // request slots in the KV cache
   int b;                     // request handled by this launch
-  const int* P_dev;          // prefix length, read on the device (no recapture on change)
+  const int* P_dev;          // [B_cap] prefix length per request, read on the device (no recapture on change)
   float eps;
   int n_clusters, n_ctas;
   GemmPlan g[4];
@@ -85,7 +85,7 @@ struct StepParams {
   // per-call tables
   const float* mod;          // [steps][n_mod] fp32 modulation rows
   int n_mod;
-  const float* rope;         // [T][hd/2][2] cos, sin for positions P .. P+T-1
+  const float* rope;         // [B_cap][T][hd/2][2] cos, sin for positions P_b .. P_b+T-1
   // buffers
   float* x;                  // [T, A]
   float* vbuf;               // [T, A]
@@ -142,8 +142,8 @@ struct BGemmParams {
   uint16_t* qbuf;
   uint16_t* kc;              // this layer's K cache [B_cap][Hkv][S_max][hd]
   uint16_t* vc;
-  const float* rope;         // [T][hd/2] (cos, sin)
-  const int* P_dev;
+  const float* rope;         // [B_cap][T][hd/2] (cos, sin) at positions P_b + t
+  const int* P_dev;          // [B_cap] prefix length per request
   int T, Hq, Hkv, hd, S_max, q_rows;
   uint32_t* err;
   long long spin_budget;
@@ -170,7 +170,7 @@ struct BAttnParams {
   const uint16_t* kc;        // this layer's cache [B_cap][Hkv][S_max][hd]
   const uint16_t* vc;
   uint16_t* o_act;           // ACT128 [Mp/128][Hq*hd/64]
-  const int* P_dev;
+  const int* P_dev;          // [B_cap] prefix length per request
   int B, T, Hq, Hkv, hd, S_max, q_rows, qblocks;
   uint32_t* err;
   long long spin_budget;

@@ -15,9 +15,9 @@ cudaError_t launch_pack8(const PackChunk* chunks, int nchunks, const int32_t* ro
                          const uint8_t* const* mats, const int* mat_k, uint8_t* dst, cudaStream_t st);
 cudaError_t launch_fp8_quantize(const uint16_t* w, int rows, int K, float* scale, uint8_t* q,
                                 cudaStream_t st);
-cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, int Hkv, int hd, int S_max,
+cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, const int* lens, int Hkv, int hd, int S_max,
                            uint16_t* cache, cudaStream_t st);
-cudaError_t launch_rope_table(int T, int hd, int P, double base, float* tab, cudaStream_t st);
+cudaError_t launch_rope_table(int B, int T, int hd, const int* P, double base, float* tab, cudaStream_t st);
 
 size_t time_gemm_smem_bytes(int d);
 cudaError_t launch_time(const TimeParams& p, int n_sms, cudaStream_t st);

@@ -75,10 +75,11 @@ __global__ void fp8_quantize_kernel(const uint16_t* __restrict__ w, const float*
   }
 }
 
-// Prefix K or V of one layer: src [B, P, H_kv, hd] -> cache [B_cap][H_kv][S_max][hd]
-// with 16-byte pieces swizzled by (row & 7).
-__global__ void kv_copy_kernel(const uint16_t* __restrict__ src, int B, int P, int Hkv, int hd,
-                               int S_max, uint16_t* __restrict__ cache) {
+// Prefix K or V of one layer: src [B, P_pad, H_kv, hd] -> cache
+// [B_cap][H_kv][S_max][hd] with 16-byte pieces swizzled by (row & 7).  Only
+// the first lens[b] rows of request b are copied (the rest is padding).
+__global__ void kv_copy_kernel(const uint16_t* __restrict__ src, int B, int P, const int* __restrict__ lens,
+                               int Hkv, int hd, int S_max, uint16_t* __restrict__ cache) {
   const int pieces = hd / 8;
   const size_t total = (size_t)B * P * Hkv * pieces;
   for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total;
@@ -88,20 +89,23 @@ __global__ void kv_copy_kernel(const uint16_t* __restrict__ src, int B, int P, i
     const int g = (int)(r % Hkv); r /= Hkv;
     const int s = (int)(r % P);
     const int b = (int)(r / P);
+    if (s >= lens[b]) continue;
     const uint4 v = *reinterpret_cast<const uint4*>(src + (((size_t)b * P + s) * Hkv + g) * hd + c * 8);
     uint16_t* row = cache + (((size_t)b * Hkv + g) * S_max + s) * hd;
     *reinterpret_cast<uint4*>(row + ((c ^ (s & 7)) << 3)) = v;
   }
 }
 
-// cos / sin of pos * base^(-2i/hd) for pos = P + t, in double, stored fp32.
-__global__ void rope_table_kernel(int T, int hd, int P, double base, float* __restrict__ tab) {
+// cos / sin of pos * base^(-2i/hd) for pos = P_b + t of every request b, in
+// double, stored fp32: tab [B][T][hd/2][2].
+__global__ void rope_table_kernel(int B, int T, int hd, const int* __restrict__ P, double base,
+                                  float* __restrict__ tab) {
   const int half = hd / 2;
   const int i = blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= T * half) return;
-  const int t = i / half, j = i % half;
+  if (i >= B * T * half) return;
+  const int b = i / (T * half), t = (i / half) % T, j = i % half;
   const double theta = pow(base, -2.0 * j / hd);
-  const double ang = (double)(P + t) * theta;
+  const double ang = (double)(P[b] + t) * theta;
   tab[2 * i] = (float)cos(ang);
   tab[2 * i + 1] = (float)sin(ang);
 }
@@ -128,16 +132,16 @@ cudaError_t launch_fp8_quantize(const uint16_t* w, int rows, int K, float* scale
   return cudaGetLastError();
 }
 
-cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, int Hkv, int hd, int S_max,
+cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, const int* lens, int Hkv, int hd, int S_max,
                            uint16_t* cache, cudaStream_t st) {
   if ((size_t)B * P == 0) return cudaSuccess;
-  kv_copy_kernel<<<512, 256, 0, st>>>(src, B, P, Hkv, hd, S_max, cache);
+  kv_copy_kernel<<<512, 256, 0, st>>>(src, B, P, lens, Hkv, hd, S_max, cache);
   return cudaGetLastError();
 }
 
-cudaError_t launch_rope_table(int T, int hd, int P, double base, float* tab, cudaStream_t st) {
-  const int n = T * hd / 2;
-  rope_table_kernel<<<(n + 127) / 128, 128, 0, st>>>(T, hd, P, base, tab);
+cudaError_t launch_rope_table(int B, int T, int hd, const int* P, double base, float* tab, cudaStream_t st) {
+  const int n = B * T * hd / 2;
+  rope_table_kernel<<<(n + 127) / 128, 128, 0, st>>>(B, T, hd, P, base, tab);
   return cudaGetLastError();
 }
 

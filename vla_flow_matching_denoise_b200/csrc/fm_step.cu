@@ -452,9 +452,10 @@ __device__ __noinline__ void gemm_begin(const Ctx& c, const GemmView& v, const u
 
 // Waits for the MMAs, stages rows 0..50 of the fp32 partial sums as one
 // contiguous block per owner ([owner][row][ownp]) and sends block o to owner
-// o's receive slot `ks` with one bulk copy each.  Returns once this CTA's own
-// receive buffer is complete.
-__device__ __noinline__ void push_partials(Ctx& c, const GemmView& v) {
+// o's receive slot `ks` with one bulk copy each.  push_wait then waits until
+// this CTA's own receive buffer is complete; work that does not need the
+// partials goes between the two.
+__device__ __noinline__ void push_send(Ctx& c, const GemmView& v) {
   if (!c.ok) return;
   Ctrl* const ctl = c.ctl;
   const long long budget = c.p->spin_budget;
@@ -487,18 +488,22 @@ __device__ __noinline__ void push_partials(Ctx& c, const GemmView& v) {
     blk += kRecvRows * ownp;
   }
   blk += lc;
+  // up to 128 columns are requested before one wait, so the TMEM read
+  // latency is paid once per 128 columns
+  constexpr int kBatch = 4;   // loads of 32 columns per wait
 #pragma unroll 1
-  for (int cb = 0; cb < ng; cb += 64) {
-    float x[2][16];
-    tmem_ld_16x256b_x4(tb + cb, x[0]);
-    if (cb + 32 < ng) tmem_ld_16x256b_x4(tb + cb + 32, x[1]);
-    tmem_ld_wait();
-    if (cb == 0) tmark(c, 13);
+  for (int c0 = 0; c0 < ng; c0 += 32 * kBatch) {
+    float x[kBatch][16];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
+    for (int h = 0; h < kBatch; ++h)
+      if (c0 + 32 * h < ng) tmem_ld_16x256b_x4(tb + c0 + 32 * h, x[h]);
+    tmem_ld_wait();
+    if (c0 == 0) tmark(c, 13);
+#pragma unroll
+    for (int h = 0; h < kBatch; ++h) {
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        if (cb + 32 * h + 8 * j >= ng) break;
+        if (c0 + 32 * h + 8 * j >= ng) break;
         if (ok_lo) *reinterpret_cast<float2*>(blk + r_lo * ownp) = make_float2(x[h][4 * j], x[h][4 * j + 1]);
         if (ok_hi) *reinterpret_cast<float2*>(blk + r_hi * ownp) = make_float2(x[h][4 * j + 2], x[h][4 * j + 3]);
         lc += 8;
@@ -525,7 +530,11 @@ __device__ __noinline__ void push_partials(Ctx& c, const GemmView& v) {
                    blk, map_shared_rank(bar_local, dst));
   }
   tmark(c, 2);
-  if (!wait_ab(bar_local, c.recv_count & 1, budget, &ctl->abort)) {
+}
+
+__device__ __noinline__ void push_wait(Ctx& c) {
+  if (!c.ok) return;
+  if (!wait_ab(smem_u32(&c.ctl->recv), c.recv_count & 1, c.p->spin_budget, &c.ctl->abort)) {
     fail(c, E_RECV);
     return;
   }
@@ -628,11 +637,14 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
     dst = (kind == 1 ? p.kcache : p.vcache) + (((size_t)l * p.B_cap + p.b) * p.Hkv + head) * p.S_max * hd;
     row_off = P;
   }
-  // stage the rotation of every row of this thread (all loads in flight at
-  // once; the planner keeps the rows per thread within kAuxRows)
+  const float2 sc = act ? wscale2(c, G_QKV, l, v.pbase + 2 * pa.pr) : make_float2(1.f, 1.f);
+  push_send(c, v);
+  // stage the rotation of every row of this thread while the partials are in
+  // flight (all loads at once; the planner keeps the rows per thread within
+  // kAuxRows)
   float2* aux = reinterpret_cast<float2*>(c.work + kWorkBytes - kAuxBytes) + c.tid;
   if (act && kind < 2) {
-    const float2* rope = reinterpret_cast<const float2*>(p.rope) + ri;
+    const float2* rope = reinterpret_cast<const float2*>(p.rope) + (size_t)p.b * T * half + ri;
     float2 rv[kAuxRows];
 #pragma unroll
     for (int k = 0; k < kAuxRows; ++k) {
@@ -643,8 +655,7 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
     for (int k = 0; k < kAuxRows; ++k)
       if (pa.t0 + k * pa.dt < T) aux[k * 128] = rv[k];
   }
-  const float2 sc = act ? wscale2(c, G_QKV, l, v.pbase + 2 * pa.pr) : make_float2(1.f, 1.f);
-  push_partials(c, v);
+  push_wait(c);
   if (!c.ok || !act) return;
   const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
   const float* rstd = c.ctl->rstd;
@@ -956,7 +967,8 @@ __device__ __noinline__ void residual_phase(Ctx& c, int g, int l, const uint16_t
       if (z != nullptr) sv[k] = *reinterpret_cast<const float2*>((t == kBiasRow ? shift : sc) + hc);
     }
   }
-  push_partials(c, v);
+  push_send(c, v);
+  push_wait(c);
   if (!c.ok) return;
   const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
   float sq = 0.f;
@@ -989,7 +1001,8 @@ __device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
   gemm_begin(c, v, p.z_f);
   tmark(c, 11);
   load_rstd(c, p.sumsq_f);
-  push_partials(c, v);
+  push_send(c, v);
+  push_wait(c);
   if (!c.ok) return;
   const int T = p.T, F = p.F;
   const int uown = v.own / 2;
@@ -1272,7 +1285,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_cons
     c.lane = lane;
     c.gemm_count = c.recv_count = c.att_count = c.xs_count = 0;
     c.epoch = 0;
-    c.P = *p.P_dev;
+    c.P = p.P_dev[p.b];
     c.ok = true;
     compute_main(c);
     if (!c.ok) ctl->abort = 1;
