@@ -152,6 +152,38 @@ fm_status fm_set_prefix(fm_expert *h, const uint16_t *const *k, const uint16_t *
 fm_status fm_set_prefix_varlen(fm_expert *h, const uint16_t *const *k, const uint16_t *const *v,
                                int batch, const int *prefix_lens, int p_pad, void *stream);
 
+/* Per-layer prefix K/V projection weights of the vision-language backbone
+ * that fills the cache the expert attends to: bf16 bits [H_kv*hd, d_prefix]
+ * each, [out, in], host or device. */
+typedef struct fm_prefix_weights {
+  const uint16_t *wk;
+  const uint16_t *wv;
+} fm_prefix_weights;
+
+/* Load the prefix cache builder: w[l] for every layer l (copied and packed;
+ * the caller may free them on return).  d_prefix: the backbone's hidden
+ * width, a positive multiple of 64.  Call once per handle; allocates the
+ * builder's device buffers (sized for max_batch x max_prefix rows).
+ * FM_ERR_UNSUPPORTED when 2 * H_kv * hd is not a multiple of 128. */
+fm_status fm_set_prefix_builder(fm_expert *h, const fm_prefix_weights *w, int d_prefix);
+
+/* Build the prefix cache on the device from each layer's prefix hidden
+ * states ("LingBot-VLA v2 Examples", Configuration / CUDA Graph: the 36-layer
+ * KV-cache construction runs once per request, before the fixed-shape
+ * denoising steps): for layer l and request b,
+ *   K = RoPE(x Wk^T) at positions 0 .. P-1,  V = x Wv^T   (bf16 in the cache)
+ * with x = hidden[l][b] ([prefix_len, d_prefix] bf16 bits; hidden[l] is
+ * [batch, prefix_len, d_prefix], host or device).  It replaces fm_set_prefix
+ * for this batch (every request gets P = prefix_len) and runs as tensor-core
+ * GEMMs with a RoPE epilogue writing straight into the cache.
+ * Synchronises `stream`.  FM_ERR_NOT_READY without fm_set_prefix_builder. */
+fm_status fm_build_prefix(fm_expert *h, const uint16_t *const *hidden, int batch, int prefix_len,
+                          void *stream);
+
+/* Test hook: the cached prefix rows of `request` at `layer`, bf16 bits
+ * [P_b, H_kv, hd] into host buffers k and v (K as stored, i.e. rotated). */
+fm_status fm_get_prefix_kv(fm_expert *h, int layer, int request, uint16_t *k, uint16_t *v);
+
 /* Denoise `batch` chunks: x0 and out are fp32 [batch, T, A], host or device
  * (independently); out may alias x0.  Runs the time MLP once, then `steps`
  * Euler steps from t = 1 to t = 0 ("LingBot-VLA on Thor (sm_110)", §1: the

@@ -38,6 +38,8 @@ The pages print no formula, so the conventions below are the plainest readings
      only to build a constant velocity field in tests.
   R8 FP8 weights: per output row c, s_c = absmax_c / 448 (fp32), q = E4M3
      nearest-even of (w / s_c) in fp32, saturated at 448; w' = q * s_c.
+  R9 prefix cache rows: K = RoPE(x Wk^T) at positions 0 .. P-1, V = x Wv^T
+     from each layer's prefix hidden states x, stored as bf16.
 
 Every function below is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, hand values, brute force or independent library routines.
@@ -260,6 +262,31 @@ def denoise(x0: np.ndarray, n: int, raw_weights: Dict, k_prefix, v_prefix, shape
         if velocities is not None:
             velocities.append(rec)
     return out
+
+
+# ----------------------------------------------------------------------------
+# prefix K/V construction (R9)
+# ----------------------------------------------------------------------------
+def prefix_kv(x: np.ndarray, wk: np.ndarray, wv: np.ndarray, n_kv_heads: int, base: float):
+    """R9: one layer's prefix cache rows from that layer's prefix hidden states
+    ("LingBot-VLA v2 Examples", Configuration / CUDA Graph: the 36-layer
+    KV-cache construction runs once per request before the denoise steps).
+
+    x: [P, d_prefix]; wk, wv: [H_kv * hd, d_prefix].  K = RoPE(x Wk^T) at
+    positions 0 .. P-1 (R4), V = x Wv^T; both [P, H_kv, hd].
+    """
+    P = x.shape[0]
+    hd = wk.shape[0] // n_kv_heads
+    k = (x @ wk.T).reshape(P, n_kv_heads, hd)
+    v = (x @ wv.T).reshape(P, n_kv_heads, hd)
+    return rope(k, np.arange(P), base), v
+
+
+def bf16_round_bits(x: np.ndarray) -> np.ndarray:
+    """Nearest-even bf16 bit patterns of float64 values (via their fp32
+    rounding, as a kernel storing an fp32 result as bf16 does)."""
+    u = np.ascontiguousarray(x, dtype=np.float32).view(np.uint32)
+    return ((u + (((u >> np.uint32(16)) & np.uint32(1)) + np.uint32(0x7FFF))) >> np.uint32(16)).astype(np.uint16)
 
 
 # ----------------------------------------------------------------------------

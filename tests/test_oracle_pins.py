@@ -376,3 +376,42 @@ def test_fp8_rows_scale_and_roundtrip():
     deq = O.fp8_dequantize_rows(codes, scale)
     err = np.abs(deq - wf.astype(np.float64))
     assert np.all(err <= np.abs(wf) * 2 ** -4 + 2 ** -9 * scale[:, None] + 1e-12)
+
+
+# --------------------------------------------------------------------------- prefix K/V (R9)
+def test_prefix_kv_one_hot_rows_pick_weight_columns_then_rotate():
+    # x row p = e_j: K row p = RoPE(Wk[:, j]) at position p, V row p = Wv[:, j]
+    rng = np.random.default_rng(21)
+    Hkv, hd, dp = 2, 8, 5
+    wk = rng.standard_normal((Hkv * hd, dp)); wv = rng.standard_normal((Hkv * hd, dp))
+    x = np.zeros((3, dp)); x[0, 4] = 1.0; x[1, 0] = 1.0; x[2, 2] = 1.0
+    k, v = O.prefix_kv(x, wk, wv, Hkv, 1e4)
+    for p, j in enumerate((4, 0, 2)):
+        assert np.allclose(v[p].reshape(-1), wv[:, j], atol=1e-15)
+        col = wk[:, j].reshape(1, Hkv, hd)
+        assert np.allclose(k[p], O.rope(col, np.array([p]), 1e4)[0], atol=1e-14)
+    # position 0 is not rotated
+    assert np.allclose(k[0].reshape(-1), wk[:, 4], atol=1e-15)
+
+
+def test_prefix_kv_brute_force_small():
+    rng = np.random.default_rng(22)
+    Hkv, hd, dp, P = 1, 4, 3, 4
+    wk = rng.standard_normal((hd, dp)); wv = rng.standard_normal((hd, dp)); x = rng.standard_normal((P, dp))
+    k, v = O.prefix_kv(x, wk, wv, Hkv, 100.0)
+    for p in range(P):
+        for e in range(hd):
+            assert abs(v[p, 0, e] - sum(x[p, i] * wv[e, i] for i in range(dp))) < 1e-13
+        raw = [sum(x[p, i] * wk[e, i] for i in range(dp)) for e in range(hd)]
+        for j in range(hd // 2):
+            a = p * 100.0 ** (-2.0 * j / hd)
+            assert abs(k[p, 0, j] - (raw[j] * math.cos(a) - raw[j + 2] * math.sin(a))) < 1e-13
+            assert abs(k[p, 0, j + 2] - (raw[j + 2] * math.cos(a) + raw[j] * math.sin(a))) < 1e-13
+
+
+def test_bf16_round_bits_ties_to_even_and_exact_values():
+    vals = np.array([1.0, 1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -2.5, 0.0])
+    bits = O.bf16_round_bits(vals)
+    # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: ties to even (1.0);
+    # 1 + 3 * 2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6: ties to even (1 + 2^-6)
+    assert list(O.decode_bf16(bits)) == [1.0, 1.0, 1.0 + 2.0 ** -6, -2.5, 0.0]

@@ -25,7 +25,8 @@ STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_NOT_READY", 3: "FM_ERR
           4: "FM_ERR_CUDA", 5: "FM_ERR_TIMEOUT", 6: "FM_ERR_UNSUPPORTED"}
 
 # Every symbol include/fm_expert.h declares.
-EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_set_prefix_varlen", "fm_denoise", "fm_velocity", "fm_time_modulation",
+EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_set_prefix_varlen", "fm_set_prefix_builder",
+           "fm_build_prefix", "fm_get_prefix_kv", "fm_denoise", "fm_velocity", "fm_time_modulation",
            "fm_trace_bytes", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
            "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
            "fm_expert_destroy", "fm_last_error", "fm_status_string",
@@ -87,6 +88,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_profile_phases.argtypes = [vp, ip, vp, ctypes.POINTER(sz), vp]
     lib.fm_time_modulation_noalloc.argtypes = [vp, vp, ip, ip, ip, vp, vp]
     lib.fm_set_prefix_varlen.argtypes = [vp, vp, vp, ip, vp, ip, vp]
+    lib.fm_set_prefix_builder.argtypes = [vp, vp, ip]
+    lib.fm_build_prefix.argtypes = [vp, vp, ip, ip, vp]
+    lib.fm_get_prefix_kv.argtypes = [vp, ip, ip, vp, vp]
     lib.fm_get_geometry.argtypes = [vp, ctypes.POINTER(ip), ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.fm_expert_destroy.argtypes = [vp]
     lib.fm_expert_destroy.restype = sz
@@ -98,7 +102,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity",
                  "fm_time_modulation", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
                  "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
-                 "fm_set_prefix_varlen"):
+                 "fm_set_prefix_varlen", "fm_set_prefix_builder", "fm_build_prefix", "fm_get_prefix_kv"):
         getattr(lib, name).restype = ip
     _lib = lib
     return lib
@@ -202,6 +206,29 @@ class Expert:
         lens = (ctypes.c_int * batch)(*[int(x) for x in prefix_lens])
         self._check("fm_set_prefix_varlen", self.lib.fm_set_prefix_varlen(self.h, kp, vp, batch, lens, p_pad,
                                                                            _stream(stream)))
+
+    def set_prefix_builder(self, weights: Sequence, d_prefix: int):
+        """weights[l] = (wk, wv): bf16 bits [H_kv * hd, d_prefix] each."""
+        L = self.shape.n_layers
+
+        class PW(ctypes.Structure):
+            _fields_ = [("wk", ctypes.c_void_p), ("wv", ctypes.c_void_p)]
+        arr = (PW * L)(*[PW(_ptr(wk), _ptr(wv)) for wk, wv in weights])
+        self._keep_builder = weights
+        self._check("fm_set_prefix_builder", self.lib.fm_set_prefix_builder(self.h, arr, d_prefix))
+
+    def build_prefix(self, hidden: Sequence, batch: int, prefix_len: int, stream=None):
+        """hidden[l]: [batch, prefix_len, d_prefix] bf16 bits (numpy or torch)."""
+        L = self.shape.n_layers
+        hp = (ctypes.c_void_p * L)(*[_ptr(x) for x in hidden])
+        self._check("fm_build_prefix", self.lib.fm_build_prefix(self.h, hp, batch, prefix_len, _stream(stream)))
+
+    def get_prefix_kv(self, layer: int, request: int, prefix_len: int):
+        s = self.shape
+        k = np.empty((prefix_len, s.n_kv_heads, s.head_dim), dtype=np.uint16)
+        v = np.empty_like(k)
+        self._check("fm_get_prefix_kv", self.lib.fm_get_prefix_kv(self.h, layer, request, _ptr(k), _ptr(v)))
+        return k, v
 
     def denoise(self, x0, steps: int, out=None, stream=None):
         """x0: fp32 [B, T, A] numpy (host) or torch (device).  Returns `out`."""

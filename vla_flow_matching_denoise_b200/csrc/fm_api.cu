@@ -80,6 +80,14 @@ struct fm_expert {
   float* bh = nullptr;               // [Mp][d] residual
   float* bdelta = nullptr;           // [Mp][d] gated branch of o_proj / down
   uint16_t* bq = nullptr;            // [B_cap][Hkv][q_rows][hd]
+  // prefix cache builder (fm_set_prefix_builder / fm_build_prefix)
+  int pre_d = 0;                     // backbone hidden width (0: no builder weights)
+  uint8_t* pre_arena = nullptr;      // per layer: [Wk; Wv] in [N/BN][d/64] chunks
+  uint64_t pre_layer_bytes = 0;
+  uint16_t* pre_stage = nullptr;     // ACT128 hidden states of one layer
+  uint16_t* pre_rows = nullptr;      // device copy of a host layer input
+  float* pre_rope = nullptr;         // [max_prefix][hd/2][2] at positions 0 .. max_prefix-1
+  int* pre_zero = nullptr;           // one 0: the position offset of the prefix table
   // buffers
   float* mod = nullptr;
   uint16_t* h1_act = nullptr;
@@ -704,6 +712,7 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
   g.F = F;
   g.qbuf = h->bq;
   g.rope = h->rope;
+  g.rope_stride_b = T;
   g.P_dev = h->P_dev;
   g.T = T;
   g.Hq = c.n_q_heads;
@@ -1250,6 +1259,154 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
   }
   if ((s = run(c.n_layers, c.n_layers, 0, 1)) != FM_OK) return s;
   CK(cudaMemcpy(out, h->vbuf, (size_t)T * c.action_dim * 4, cudaMemcpyDeviceToHost));
+  return FM_OK;
+}
+
+fm_status fm_set_prefix_builder(fm_expert* h, const fm_prefix_weights* w, int d_prefix) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (!w) return set_err(h, FM_ERR_INVALID_ARG, "weights are NULL");
+  if (d_prefix < 64 || d_prefix % 64 != 0)
+    return set_err(h, FM_ERR_INVALID_ARG, "d_prefix %d must be a positive multiple of 64", d_prefix);
+  if (h->pre_d != 0) return set_err(h, FM_ERR_INVALID_ARG, "the prefix builder is already loaded");
+  const int kn = c.n_kv_heads * c.head_dim, N = 2 * kn;
+  if (N % 128 != 0 || (c.head_dim != 64 && c.head_dim != 128))
+    return set_err(h, FM_ERR_UNSUPPORTED, "prefix builder needs 2 H_kv hd a multiple of 128, hd 64 or 128");
+  CK(cudaSetDevice(h->device));
+  const int bn = bgemm_bn(BE_QKV, N), nkb = d_prefix / 64;
+  std::vector<PackChunk> jobs;
+  std::vector<int32_t> rows;
+  for (int nt = 0; nt < N / bn; ++nt) {
+    const uint32_t roff = (uint32_t)rows.size();
+    for (int q = 0; q < bn; ++q) rows.push_back(nt * bn + q);
+    for (int kb = 0; kb < nkb; ++kb) {
+      PackChunk pc{};
+      pc.dst_off = ((uint64_t)nt * nkb + kb) * bn * 128;
+      pc.rowidx_off = roff;
+      pc.nrows = (uint16_t)bn;
+      pc.mat = 0;
+      pc.kb = (uint32_t)kb;
+      jobs.push_back(pc);
+    }
+  }
+  h->pre_layer_bytes = (uint64_t)N * d_prefix * 2;
+  const size_t Mp = (size_t)((c.max_batch * std::max(c.max_prefix, 1) + kBM - 1) / kBM * kBM);
+  DALLOC(h->pre_arena, (size_t)c.n_layers * h->pre_layer_bytes);
+  DALLOC(h->pre_stage, Mp * d_prefix * 2);
+  DALLOC(h->pre_rows, (size_t)c.max_batch * std::max(c.max_prefix, 1) * d_prefix * 2);
+  DALLOC(h->pre_rope, (size_t)std::max(c.max_prefix, 1) * c.head_dim * 4);
+  DALLOC(h->pre_zero, 4);   // zero-filled: positions start at 0
+  void* tmp = nullptr;
+  void* tab = nullptr;
+  cudaError_t e = cudaMalloc(&tmp, (size_t)N * d_prefix * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&tab, jobs.size() * sizeof(PackChunk) + rows.size() * 4 + 2 * sizeof(void*) + 64);
+  fm_status st = FM_OK;
+  if (e != cudaSuccess) st = set_err(h, FM_ERR_OOM, "prefix builder staging: %s", cudaGetErrorString(e));
+  PackChunk* d_jobs = static_cast<PackChunk*>(tab);
+  int32_t* d_rows = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(tab) + jobs.size() * sizeof(PackChunk));
+  uint8_t* tail = reinterpret_cast<uint8_t*>(d_rows) + rows.size() * 4;
+  tail = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(tail) + 15) & ~uintptr_t(15));
+  uint16_t** d_mats = reinterpret_cast<uint16_t**>(tail);
+  int* d_matk = reinterpret_cast<int*>(tail + sizeof(void*));
+  if (st == FM_OK) {
+    uint16_t* mp = static_cast<uint16_t*>(tmp);
+    e = cudaMemcpy(d_jobs, jobs.data(), jobs.size() * sizeof(PackChunk), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(d_rows, rows.data(), rows.size() * 4, cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(d_mats, &mp, sizeof(void*), cudaMemcpyHostToDevice);
+    if (e == cudaSuccess) e = cudaMemcpy(d_matk, &d_prefix, sizeof(int), cudaMemcpyHostToDevice);
+    for (int l = 0; l < c.n_layers && e == cudaSuccess; ++l) {
+      if (!w[l].wk || !w[l].wv) {
+        st = set_err(h, FM_ERR_INVALID_ARG, "prefix builder layer %d has a NULL weight", l);
+        break;
+      }
+      e = cudaMemcpy(mp, w[l].wk, (size_t)kn * d_prefix * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess) e = cudaMemcpy(mp + (size_t)kn * d_prefix, w[l].wv, (size_t)kn * d_prefix * 2, cudaMemcpyDefault);
+      if (e == cudaSuccess)
+        e = launch_pack(d_jobs, (int)jobs.size(), d_rows, d_mats, d_matk, h->pre_arena + (size_t)l * h->pre_layer_bytes, 0);
+    }
+    if (e == cudaSuccess)
+      e = launch_rope_table(1, std::max(c.max_prefix, 1), c.head_dim, h->pre_zero, (double)c.rope_base, h->pre_rope, 0);
+    if (e == cudaSuccess) e = cudaDeviceSynchronize();
+    if (e != cudaSuccess && st == FM_OK) st = set_err(h, FM_ERR_CUDA, "prefix builder packing: %s", cudaGetErrorString(e));
+  }
+  if (tmp) cudaFree(tmp);
+  if (tab) cudaFree(tab);
+  if (st == FM_OK) h->pre_d = d_prefix;
+  return st;
+}
+
+fm_status fm_build_prefix(fm_expert* h, const uint16_t* const* hidden, int batch, int prefix_len, void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (h->pre_d == 0) return set_err(h, FM_ERR_NOT_READY, "fm_set_prefix_builder was not called");
+  if (batch < 1 || batch > c.max_batch)
+    return set_err(h, FM_ERR_INVALID_ARG, "batch %d outside [1, %d]", batch, c.max_batch);
+  if (prefix_len < 0 || prefix_len > c.max_prefix)
+    return set_err(h, FM_ERR_INVALID_ARG, "prefix_len %d outside [0, %d]", prefix_len, c.max_prefix);
+  if (prefix_len > 0 && !hidden) return set_err(h, FM_ERR_INVALID_ARG, "hidden is NULL");
+  CK(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int d = h->pre_d, kn = c.n_kv_heads * c.head_dim, L = c.n_layers;
+  const int M = batch * prefix_len, Mp = (M + kBM - 1) / kBM * kBM;
+  const size_t lay = (size_t)c.max_batch * c.n_kv_heads * h->S_max * c.head_dim;
+  std::vector<int> lens(batch, prefix_len);
+  CK(cudaMemcpyAsync(h->P_dev, lens.data(), (size_t)batch * 4, cudaMemcpyHostToDevice, st));
+  BGemmParams g{};
+  g.M = M;
+  g.Mp = Mp;
+  g.K = d;
+  g.N = 2 * kn;
+  g.T = prefix_len;            // rows m = b * P + p
+  g.Hq = 0;                    // no query heads: columns are K heads then V heads
+  g.Hkv = c.n_kv_heads;
+  g.hd = c.head_dim;
+  g.S_max = h->S_max;
+  g.rope = h->pre_rope;
+  g.rope_stride_b = 0;         // positions 0 .. P-1 for every request
+  g.P_dev = nullptr;           // cache rows start at 0
+  g.err = h->err_word;
+  g.spin_budget = 4000000000LL;
+  for (int l = 0; l < L && M > 0; ++l) {
+    if (!hidden[l]) return set_err(h, FM_ERR_INVALID_ARG, "hidden states of layer %d are NULL", l);
+    const uint16_t* src = hidden[l];
+    if (!is_device_ptr(src)) {
+      CK(cudaMemcpyAsync(h->pre_rows, src, (size_t)M * d * 2, cudaMemcpyHostToDevice, st));
+      src = h->pre_rows;
+    }
+    CK(launch_rows_to_act128(src, M, Mp, d, h->pre_stage, st));
+    g.A = reinterpret_cast<const uint8_t*>(h->pre_stage);
+    g.W = h->pre_arena + (size_t)l * h->pre_layer_bytes;
+    g.kc = h->kcache + l * lay;
+    g.vc = h->vcache + l * lay;
+    CK(launch_bgemm(g, BE_QKV, h->n_sms, st));
+  }
+  CK(launch_rope_table(batch, c.chunk_len, c.head_dim, h->P_dev, (double)c.rope_base, h->rope, st));
+  CK(cudaStreamSynchronize(st));
+  h->prefix_batch = batch;
+  h->prefix_lens = lens;
+  return check_err_word(h);
+}
+
+fm_status fm_get_prefix_kv(fm_expert* h, int layer, int request, uint16_t* k, uint16_t* v) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (layer < 0 || layer >= c.n_layers || request < 0 || request >= h->prefix_batch || !k || !v)
+    return set_err(h, FM_ERR_INVALID_ARG, "layer %d / request %d invalid or NULL buffer", layer, request);
+  CK(cudaSetDevice(h->device));
+  const int P = h->prefix_lens[request], hd = c.head_dim, Hkv = c.n_kv_heads;
+  const size_t lay = (size_t)c.max_batch * Hkv * h->S_max * hd;
+  std::vector<uint16_t> buf((size_t)h->S_max * hd);
+  for (int which = 0; which < 2; ++which) {
+    uint16_t* out = which == 0 ? k : v;
+    const uint16_t* cache = (which == 0 ? h->kcache : h->vcache) + layer * lay;
+    for (int g = 0; g < Hkv; ++g) {
+      CK(cudaMemcpy(buf.data(), cache + (((size_t)request * Hkv + g) * h->S_max) * hd, (size_t)P * hd * 2,
+                    cudaMemcpyDeviceToHost));
+      for (int p = 0; p < P; ++p)
+        for (int e = 0; e < hd; ++e)
+          out[((size_t)p * Hkv + g) * hd + e] = buf[(size_t)p * hd + ((((e >> 3) ^ (p & 7))) << 3) + (e & 7)];
+    }
+  }
   return FM_OK;
 }
 

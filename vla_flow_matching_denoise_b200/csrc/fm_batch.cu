@@ -117,8 +117,9 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
   const int hd = p.hd, half = hd / 2;
   const int qn = p.Hq * hd, kn = p.Hkv * hd, G = p.Hq / p.Hkv;
   const int b = valid ? m / p.T : 0, t = valid ? m % p.T : 0;
-  const int P = p.P_dev[b];   // this request's prefix length: chunk rows and RoPE positions follow it
-  const float2* rope = reinterpret_cast<const float2*>(p.rope) + ((size_t)b * p.T + t) * half;
+  // chunk: rows and RoPE positions follow this request's prefix length
+  const int P = p.P_dev != nullptr ? p.P_dev[b] : 0;
+  const float2* rope = reinterpret_cast<const float2*>(p.rope) + ((size_t)b * p.rope_stride_b + t) * half;
 #pragma unroll 1
   for (int ho = 0; ho < BN; ho += hd) {
     const int col0 = nt * BN + ho;
@@ -126,7 +127,7 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
     const int head = (kind == 0 ? col0 : kind == 1 ? col0 - qn : col0 - qn - kn) / hd;
     uint16_t* rowp;
     int row;
-    if (kind == 0) {
+    if (kind == 0) {   // (only when Hq > 0)
       row = (head % G) * p.T + t;
       rowp = p.qbuf + (((size_t)b * p.Hkv + head / G) * p.q_rows + row) * hd;
     } else {
@@ -730,6 +731,23 @@ cudaError_t launch_bgemm(const BGemmParams& p, int epi, int n_sms, cudaStream_t 
     return bn == 256 ? launch_bgemm_t<256, BE_RESID>(p, n_sms, st) : launch_bgemm_t<128, BE_RESID>(p, n_sms, st);
   if (epi == BE_SWIGLU) return launch_bgemm_t<256, BE_SWIGLU>(p, n_sms, st);
   return bn == 256 ? launch_bgemm_t<256, BE_QKV>(p, n_sms, st) : launch_bgemm_t<128, BE_QKV>(p, n_sms, st);
+}
+
+// Row-major bf16 [M][K] -> ACT128 [Mp/128][K/64]; rows M .. Mp-1 are zero.
+__global__ void rows_to_act128_kernel(const uint16_t* __restrict__ src, int M, int Mp, int K,
+                                      uint16_t* __restrict__ dst) {
+  const int pieces = K / 8;
+  const size_t total = (size_t)Mp * pieces;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < total; i += (size_t)gridDim.x * blockDim.x) {
+    const int m = (int)(i / pieces), c = (int)(i % pieces) * 8;
+    const uint4 v = m < M ? *reinterpret_cast<const uint4*>(src + (size_t)m * K + c) : make_uint4(0u, 0u, 0u, 0u);
+    *reinterpret_cast<uint4*>(dst + act128_off(m, c, K)) = v;
+  }
+}
+
+cudaError_t launch_rows_to_act128(const uint16_t* src, int M, int Mp, int K, uint16_t* dst, cudaStream_t st) {
+  rows_to_act128_kernel<<<1024, 256, 0, st>>>(src, M, Mp, K, dst);
+  return cudaGetLastError();
 }
 
 cudaError_t launch_binproj(const BRowParams& p, cudaStream_t st) {

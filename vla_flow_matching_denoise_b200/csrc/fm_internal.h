@@ -138,12 +138,16 @@ struct BGemmParams {
   // BE_SWIGLU: tile j holds gate rows 128j.. then up rows 128j..; u = SiLU(g) up
   uint16_t* u_act;           // ACT128 [Mp/128][F/64]
   int F;
-  // BE_QKV: RoPE on q, k; q -> qbuf [B][Hkv][q_rows][hd]; k, v -> cache rows P + t
+  // BE_QKV: RoPE on q, k; q -> qbuf [B][Hkv][q_rows][hd]; k, v -> cache rows
+  // P_b + t of request b = m / T, t = m % T.  The prefix cache builder uses the
+  // same epilogue with no q heads (Hq = 0), T = the prefix length, P_dev null
+  // (rows start at 0) and one RoPE table shared by all requests.
   uint16_t* qbuf;
   uint16_t* kc;              // this layer's K cache [B_cap][Hkv][S_max][hd]
   uint16_t* vc;
-  const float* rope;         // [B_cap][T][hd/2] (cos, sin) at positions P_b + t
-  const int* P_dev;          // [B_cap] prefix length per request
+  const float* rope;         // (cos, sin) rows [b * rope_stride_b + t][hd/2]
+  int rope_stride_b;         // T for the chunk (per-request positions), 0 for the prefix
+  const int* P_dev;          // [B_cap] prefix length per request, or null (offset 0)
   int T, Hq, Hkv, hd, S_max, q_rows;
   uint32_t* err;
   long long spin_budget;

@@ -31,6 +31,7 @@ cudaError_t launch_step(const StepParams& p, cudaStream_t st);
 int bgemm_bn(int epi, int N);   // weight tile width the GEMM uses for this epilogue
 cudaError_t launch_bgemm(const BGemmParams& p, int epi, int n_sms, cudaStream_t st);
 cudaError_t launch_binproj(const BRowParams& p, cudaStream_t st);
+cudaError_t launch_rows_to_act128(const uint16_t* src, int M, int Mp, int K, uint16_t* dst, cudaStream_t st);
 cudaError_t launch_bresnorm(const BRowParams& p, cudaStream_t st);
 cudaError_t launch_boutproj(const BRowParams& p, cudaStream_t st);
 cudaError_t launch_battn(const BAttnParams& p, cudaStream_t st);

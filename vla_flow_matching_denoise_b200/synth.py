@@ -16,9 +16,10 @@ Recipe (the pages print no inputs, so these are synthetic stand-ins):
     bf16 with round-to-nearest-even;
   * prefix K/V ~ N(0, 1), rounded to bf16 the same way;
   * x0 (the action chunk at t = 1) ~ N(0, 1) in fp32, not rounded.
-Three independent PCG64 streams are derived from one seed with
+Independent PCG64 streams are derived from one seed with
 ``np.random.SeedSequence([seed, stream])``: stream 0 = weights, 1 = prefix K/V,
-2 = x0.  Weight order: time_w1, time_w2, in_proj, out_proj, then per layer
+2 = x0, 3 = the prefix K/V projection weights of the backbone, 4 = the prefix
+hidden states those project.  Weight order: time_w1, time_w2, in_proj, out_proj, then per layer
 (wq, wk, wv, wo, w_gate, w_up, w_down).  Prefix order: per layer K then V, each
 [B, P, H_kv, hd].  Requests of a batch are drawn consecutively.
 """
@@ -157,6 +158,24 @@ def make_prefix(shape: ExpertShape, seed: int = 0, batch: int | None = None,
         ks.append(_bf16_normal(rng, kshape, 1.0))
         vs.append(_bf16_normal(rng, kshape, 1.0))
     return ks, vs
+
+
+def make_prefix_builder(shape: ExpertShape, d_prefix: int, seed: int = 0):
+    """Per-layer prefix K/V projection weights of the backbone: bf16 bits
+    [H_kv * hd, d_prefix] each, N(0, 0.02^2); stream 3, layer by layer (wk, wv)."""
+    rng = _stream(seed, 3)
+    rows = shape.n_kv_heads * shape.head_dim
+    return [(_bf16_normal(rng, (rows, d_prefix), shape.weight_std),
+             _bf16_normal(rng, (rows, d_prefix), shape.weight_std)) for _ in range(shape.n_layers)]
+
+
+def make_prefix_hidden(shape: ExpertShape, d_prefix: int, seed: int = 0, batch: int | None = None,
+                       prefix_len: int | None = None):
+    """Per-layer prefix hidden states, bf16 bits [B, P, d_prefix] ~ N(0, 1); stream 4."""
+    B = shape.batch if batch is None else batch
+    P = shape.prefix_len if prefix_len is None else prefix_len
+    rng = _stream(seed, 4)
+    return [_bf16_normal(rng, (B, P, d_prefix), 1.0) for _ in range(shape.n_layers)]
 
 
 def make_x0(shape: ExpertShape, seed: int = 0, batch: int | None = None) -> np.ndarray:
