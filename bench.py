@@ -44,7 +44,13 @@ UNIT = "denoise steps/s"
 # DRAM bytes of one launch of the loop kernel from an ncu capture, keyed by
 # workload, with the hash of the kernel sources it was taken on; reported as
 # null when the sources changed since.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # step_kernel, bench workload: dram__bytes_read.sum + dram__bytes_write.sum of one
+    # `python bench.py --workload lingbot_l4_p256_n10 --once` launch (4 layers x 1 Euler
+    # step: 140.909 + 3.717 MB), scaled by the 90x layer-steps of a 36-layer, 10-step
+    # launch (weight and KV traffic grow in proportion).
+    "lingbot_p256_n10": {"source_hash": "832090014b1dc8fe", "dram_bytes": 144.626e6 * 90},
+}
 
 
 def kernel_source_hash() -> str:
