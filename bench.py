@@ -96,7 +96,14 @@ def loop_bytes(shape: synth.ExpertShape, steps: int, batch: int) -> float:
     ws = s.weight_shapes()
     per_layer = sum(int(np.prod(ws[k])) for k in synth.LAYER_KEYS)
     rows = sum(ws[k][0] for k in synth.LAYER_KEYS)
-    wbytes = s.n_layers * (per_layer * (1.0 if s.fp8 else 2.0) + (rows * 4.0 if s.fp8 else 0.0))
+    if s.nvfp4_gu:
+        # E4M3 + row scales for wq/wk/wv/wo/w_down; NVFP4 (half a byte per code,
+        # one E4M3 scale per 16 codes, one fp32 per tensor) for w_gate, w_up
+        gu = int(np.prod(ws["w_gate"])) + int(np.prod(ws["w_up"]))
+        rows_8 = rows - ws["w_gate"][0] - ws["w_up"][0]
+        wbytes = s.n_layers * ((per_layer - gu) * 1.0 + rows_8 * 4.0 + gu * (0.5 + 1.0 / 16) + 8.0)
+    else:
+        wbytes = s.n_layers * (per_layer * (1.0 if s.fp8 else 2.0) + (rows * 4.0 if s.fp8 else 0.0))
     io = (int(np.prod(ws["in_proj"])) + int(np.prod(ws["out_proj"]))) * 2.0
     kv = batch * s.n_layers * 2 * (s.prefix_len + s.chunk_len) * s.n_kv_heads * s.head_dim * 2.0
     return steps * (wbytes + io + kv)
@@ -347,7 +354,7 @@ def main():
     lb = loop_bytes(shape, n, B)
     achieved = lb / (ms_loop / 1000.0) / 1e9
     lf = loop_flops(shape, n, B)
-    batched = B >= 2 and not shape.fp8
+    batched = B >= 2 and not shape.fp8 and not shape.nvfp4_gu
     traffic = None
     rec = NCU_TRAFFIC.get(args.workload)
     if rec and rec.get("source_hash") == kernel_source_hash():
@@ -367,7 +374,8 @@ def main():
                    "heads": f"{shape.n_q_heads}q/{shape.n_kv_heads}kv x {shape.head_dim}",
                    "d_ff": shape.d_ff, "prefix_len": shape.prefix_len,
                    "chunk": f"{shape.chunk_len}x{shape.action_dim}", "euler_steps": n,
-                   "requests_per_gpu": B, "weights": "fp8-e4m3" if shape.fp8 else "bf16",
+                   "requests_per_gpu": B,
+                   "weights": "fp8-e4m3 + nvfp4 gate_up" if shape.nvfp4_gu else "fp8-e4m3" if shape.fp8 else "bf16",
                    "parallelism": f"replicas x{ws}",
                    "l2": f"inputs larger than L2: {loop_bytes(shape, 1, B) / 1e9:.3f} GB of weights and KV "
                          "stream per Euler step (L2 126 MB)"},

@@ -70,8 +70,13 @@ typedef enum fm_status {
 
 typedef enum fm_wtype {
   FM_W_BF16 = 0,            /* per-layer linears kept in bf16                   */
-  FM_W_FP8_E4M3 = 1         /* per-layer linears quantised to E4M3, one fp32
+  FM_W_FP8_E4M3 = 1,        /* per-layer linears quantised to E4M3, one fp32
                                scale per output row (s = absmax / 448)          */
+  FM_W_FP8_NVFP4_GU = 2     /* E4M3 as above for wq/wk/wv/wo/w_down; w_gate and
+                               w_up in NVFP4: E2M1 codes, one E4M3 scale per 16
+                               inputs, one fp32 scale per tensor ("LingBot-VLA
+                               on Thor (sm_110)", §1: FP8 weights with an FP4
+                               gate_up)                                          */
 } fm_wtype;
 
 /* Model shape and capacities.  Requirements (checked by fm_expert_create):
@@ -225,6 +230,14 @@ fm_status fm_trace_velocity(fm_expert *h, const float *x, int step_index, int st
  * handle. */
 fm_status fm_get_fp8_weights(fm_expert *h, int layer, int which, uint8_t *codes,
                              float *scale);
+
+/* Test hook: the NVFP4 weights of w_gate (which = 4) or w_up (5) of `layer`
+ * in a FM_W_FP8_NVFP4_GU handle, read back from the packed arena: codes
+ * [out, in] one E2M1 code (0..15, bit 3 = sign) per byte, block scales
+ * [out, in/16] E4M3 codes, and the tensor's fp32 scale g; host buffers.
+ * Dequantised weight = e2m1(code) * e4m3(block scale) * g. */
+fm_status fm_get_nvfp4_weights(fm_expert *h, int layer, int which, uint8_t *codes,
+                               uint8_t *block_scales, float *g);
 
 /* Profiling hook: runs `iters` times the two kernels of one denoise (the
  * time MLP, then the denoise loop for every request) outside any graph, with

@@ -40,6 +40,10 @@ The pages print no formula, so the conventions below are the plainest readings
      nearest-even of (w / s_c) in fp32, saturated at 448; w' = q * s_c.
   R9 prefix cache rows: K = RoPE(x Wk^T) at positions 0 .. P-1, V = x Wv^T
      from each layer's prefix hidden states x, stored as bf16.
+  R10 NVFP4 gate_up (with E4M3 R8 for the other linears): per tensor
+     g = amax / (6 * 448) (fp32); per row and 16-column block
+     s_b = E4M3 nearest-even of (amax_b / (6 g)) in fp32; codes = E2M1
+     nearest-even of (w / (s_b g)) in fp32, saturated at 6; w' = q s_b g.
 
 Every function below is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, hand values, brute force or independent library routines.
@@ -155,7 +159,7 @@ def gqa_attention(q: np.ndarray, k: np.ndarray, v: np.ndarray) -> np.ndarray:
 class Weights:
     """Decoded weights of one expert (float arrays, [out, in])."""
 
-    def __init__(self, raw: Dict, dtype=np.float64, fp8: bool = False):
+    def __init__(self, raw: Dict, dtype=np.float64, fp8: bool = False, nvfp4_gu: bool = False):
         self.dtype = dtype
         self.time_w1 = decode_bf16(raw["time_w1"], dtype)
         self.time_w2 = decode_bf16(raw["time_w2"], dtype)
@@ -166,7 +170,9 @@ class Weights:
             d = {}
             for key, bits in lw.items():
                 w = decode_bf16(bits, np.float64)
-                if fp8:
+                if nvfp4_gu and key in ("w_gate", "w_up"):
+                    w = nvfp4_dequantize(*nvfp4_quantize(bits))
+                elif fp8 or nvfp4_gu:
                     codes, scale = fp8_quantize_rows(bits)
                     w = fp8_dequantize_rows(codes, scale)
                 d[key] = w.astype(dtype)
@@ -336,3 +342,58 @@ def fp8_quantize_rows(w_bits: np.ndarray):
 def fp8_dequantize_rows(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:
     """w' = decode(q) * s_c in float64."""
     return e4m3_decode(codes) * np.asarray(scale, dtype=np.float64)[:, None]
+
+
+# ----------------------------------------------------------------------------
+# NVFP4 weight quantiser (R10): E2M1 elements, 16-element E4M3 block scales,
+# one fp32 scale per tensor
+# ----------------------------------------------------------------------------
+E2M1_VALUES = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+NVFP4_BLOCK = 16
+
+
+def e2m1_decode(codes: np.ndarray) -> np.ndarray:
+    """4-bit E2M1 codes (bit 3 = sign) -> float64 values."""
+    c = np.asarray(codes).astype(np.int64)
+    return np.where(c & 8, -1.0, 1.0) * E2M1_VALUES[c & 7]
+
+
+def e2m1_encode(v: np.ndarray) -> np.ndarray:
+    """Nearest E2M1 code of fp32 values, ties to the even code, saturating at 6."""
+    a = np.abs(np.asarray(v, dtype=np.float32).astype(np.float64))
+    # distance to every magnitude; ties go to the even index
+    d = np.abs(a[..., None] - E2M1_VALUES)
+    best = np.zeros(a.shape, dtype=np.int64)
+    bd = d[..., 0]
+    for i in range(1, 8):
+        take = (d[..., i] < bd) | ((d[..., i] == bd) & (i % 2 == 0))
+        best = np.where(take, i, best)
+        bd = np.where(take, d[..., i], bd)
+    best = np.where(a >= 6.0, 7, best)
+    sign = np.signbit(np.asarray(v, dtype=np.float32)) & (best > 0)
+    return (best | np.where(sign, 8, 0)).astype(np.uint8)
+
+
+def nvfp4_quantize(w_bits: np.ndarray):
+    """R10 on bf16 weight bits [rows, K] (K a multiple of 16) ->
+    (codes uint8 [rows, K] in 0..15, block scales uint8 E4M3 [rows, K/16], g float32)."""
+    w = decode_bf16(w_bits, np.float32)
+    rows, K = w.shape
+    amax = np.float32(np.max(np.abs(w)))
+    g = np.float32(amax / np.float32(6.0 * E4M3_MAX)) if amax > 0 else np.float32(1.0)
+    blocks = w.reshape(rows, K // NVFP4_BLOCK, NVFP4_BLOCK)
+    bmax = np.max(np.abs(blocks), axis=2).astype(np.float32)
+    sb = e4m3_encode((bmax / (np.float32(6.0) * g)).astype(np.float32))
+    sbv = e4m3_decode(sb).astype(np.float32)
+    denom = (sbv * g).astype(np.float32)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        ratio = np.where(denom[:, :, None] > 0, (blocks / denom[:, :, None]).astype(np.float32), np.float32(0.0))
+    codes = e2m1_encode(ratio).reshape(rows, K)
+    return codes, sb, g
+
+
+def nvfp4_dequantize(codes: np.ndarray, sb: np.ndarray, g) -> np.ndarray:
+    """w' = e2m1(q) * e4m3(s_b) * g in float64."""
+    rows, K = codes.shape
+    q = e2m1_decode(codes).reshape(rows, K // NVFP4_BLOCK, NVFP4_BLOCK)
+    return (q * e4m3_decode(sb)[:, :, None] * float(g)).reshape(rows, K)

@@ -415,3 +415,35 @@ def test_bf16_round_bits_ties_to_even_and_exact_values():
     # 1 + 2^-8 is halfway between 1 and 1 + 2^-7: ties to even (1.0);
     # 1 + 3 * 2^-8 is halfway between 1 + 2^-7 and 1 + 2^-6: ties to even (1 + 2^-6)
     assert list(O.decode_bf16(bits)) == [1.0, 1.0, 1.0 + 2.0 ** -6, -2.5, 0.0]
+
+
+# --------------------------------------------------------------------------- NVFP4 (R10)
+def test_e2m1_table_and_ties_to_even():
+    # the eight E2M1 magnitudes (1 exponent bias, 1 mantissa bit)
+    assert list(O.e2m1_decode(np.arange(8))) == [0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0]
+    assert list(O.e2m1_decode(np.arange(8, 16))) == [-0.0, -0.5, -1.0, -1.5, -2.0, -3.0, -4.0, -6.0]
+    # exact values round trip; midpoints go to the even code
+    for c in range(16):
+        assert O.e2m1_encode(O.e2m1_decode(np.array([c]))) == (0 if c == 8 else c)
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    assert list(O.e2m1_encode(mids)) == [0, 2, 2, 4, 4, 6, 6]
+    assert list(O.e2m1_encode(np.array([7.0, 100.0, -9.0]))) == [7, 7, 15]
+
+
+def test_nvfp4_block_max_maps_to_six_and_zero_blocks():
+    rng = np.random.default_rng(31)
+    w = rng.standard_normal((3, 64)).astype(np.float32) * 0.02
+    w[1, 16:32] = 0.0                                   # an all-zero block
+    bits = O.bf16_round_bits(w)
+    codes, sb, g = O.nvfp4_quantize(bits)
+    wd = O.decode_bf16(bits)
+    assert g == np.float32(np.float32(np.max(np.abs(wd))) / np.float32(2688.0))
+    assert sb[1, 1] == 0 and not codes[1, 16:32].any()
+    deq = O.nvfp4_dequantize(codes, sb, g)
+    # every dequantised weight is a bf16 value times g: e2m1 x e4m3 needs <= 5 significant bits
+    prod = O.e2m1_decode(codes).reshape(3, 4, 16) * O.e4m3_decode(sb)[:, :, None]
+    assert np.array_equal(O.decode_bf16(O.bf16_round_bits(prod)), prod.astype(np.float32).astype(np.float64))
+    # relative error per block is bounded by half an E2M1 step at the block's top (and the scale rounding)
+    err = np.abs(deq - wd).reshape(3, 4, 16).max(axis=2)
+    top = np.abs(wd).reshape(3, 4, 16).max(axis=2)
+    assert np.all(err <= 0.35 * top + 1e-12)

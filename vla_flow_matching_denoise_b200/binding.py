@@ -20,13 +20,14 @@ LIB_PATH = os.path.join(_PKG, "libfm_expert.so")
 
 FM_W_BF16 = 0
 FM_W_FP8_E4M3 = 1
+FM_W_FP8_NVFP4_GU = 2
 
 STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_NOT_READY", 3: "FM_ERR_OOM",
           4: "FM_ERR_CUDA", 5: "FM_ERR_TIMEOUT", 6: "FM_ERR_UNSUPPORTED"}
 
 # Every symbol include/fm_expert.h declares.
 EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_set_prefix_varlen", "fm_set_prefix_builder",
-           "fm_build_prefix", "fm_get_prefix_kv", "fm_denoise", "fm_velocity", "fm_time_modulation",
+           "fm_build_prefix", "fm_get_prefix_kv", "fm_get_nvfp4_weights", "fm_denoise", "fm_velocity", "fm_time_modulation",
            "fm_trace_bytes", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
            "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
            "fm_expert_destroy", "fm_last_error", "fm_status_string",
@@ -91,6 +92,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_set_prefix_builder.argtypes = [vp, vp, ip]
     lib.fm_build_prefix.argtypes = [vp, vp, ip, ip, vp]
     lib.fm_get_prefix_kv.argtypes = [vp, ip, ip, vp, vp]
+    lib.fm_get_nvfp4_weights.argtypes = [vp, ip, ip, vp, vp, vp]
     lib.fm_get_geometry.argtypes = [vp, ctypes.POINTER(ip), ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.fm_expert_destroy.argtypes = [vp]
     lib.fm_expert_destroy.restype = sz
@@ -102,7 +104,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     for name in ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity",
                  "fm_time_modulation", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
                  "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
-                 "fm_set_prefix_varlen", "fm_set_prefix_builder", "fm_build_prefix", "fm_get_prefix_kv"):
+                 "fm_set_prefix_varlen", "fm_set_prefix_builder", "fm_build_prefix", "fm_get_prefix_kv",
+                 "fm_get_nvfp4_weights"):
         getattr(lib, name).restype = ip
     _lib = lib
     return lib
@@ -141,7 +144,8 @@ def make_config(shape: ExpertShape, max_prefix: Optional[int] = None, max_batch:
                     shape.d_ff, shape.action_dim, shape.chunk_len,
                     shape.prefix_len if max_prefix is None else max_prefix,
                     shape.batch if max_batch is None else max_batch, max_steps,
-                    shape.rms_eps, shape.rope_base, FM_W_FP8_E4M3 if shape.fp8 else FM_W_BF16)
+                    shape.rms_eps, shape.rope_base,
+                    FM_W_FP8_NVFP4_GU if shape.nvfp4_gu else FM_W_FP8_E4M3 if shape.fp8 else FM_W_BF16)
 
 
 class Expert:
@@ -277,6 +281,15 @@ class Expert:
         self._check("fm_get_fp8_weights", self.lib.fm_get_fp8_weights(self.h, layer, which, _ptr(codes),
                                                                        _ptr(scale)))
         return codes, scale
+
+    def get_nvfp4_weights(self, layer: int, which: int, rows: int, cols: int):
+        """(codes [rows, cols] one E2M1 code per byte, block scales [rows, cols/16] E4M3, g)."""
+        codes = np.empty((rows, cols), dtype=np.uint8)
+        sb = np.empty((rows, cols // 16), dtype=np.uint8)
+        g = np.zeros(1, dtype=np.float32)
+        self._check("fm_get_nvfp4_weights", self.lib.fm_get_nvfp4_weights(self.h, layer, which, _ptr(codes),
+                                                                           _ptr(sb), _ptr(g)))
+        return codes, sb, np.float32(g[0])
 
     def profile(self, batch: int, steps: int, iters: int, stream=None):
         """Mean (time-MLP ms, loop ms) over `iters` event-timed runs."""

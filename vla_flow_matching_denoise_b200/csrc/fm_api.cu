@@ -67,6 +67,7 @@ struct fm_expert {
   std::vector<PackChunk> pack_jobs;
   std::vector<int32_t> pack_rows;
   std::vector<float> row_scale;      // [L][rows of QKV + O + GU + DOWN]
+  std::vector<float> nv4_g;          // NVFP4 gate_up: [L][2] tensor scales (gate, up)
   // batched path (B >= 2 requests advance together, M = B * T rows)
   bool batched = false;
   uint8_t* barena = nullptr;         // per layer: [N/BN][K/64] chunks of each linear
@@ -286,8 +287,12 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   const fm_config& c = h->cfg;
   const int d = c.d_model, F = c.d_ff, qn = c.n_q_heads * c.head_dim,
             kn = c.n_kv_heads * c.head_dim;
-  const bool fp8 = c.wtype == FM_W_FP8_E4M3;
-  const uint64_t row_bytes = fp8 ? 64 : 128;   // one chunk row: 64 weights
+  // quantised weights: E4M3 rows for every linear, or for all but gate_up,
+  // whose rows are NVFP4 (64 codes + 4 block scales = 36 bytes)
+  const bool nv4 = c.wtype == FM_W_FP8_NVFP4_GU;
+  const bool fp8 = c.wtype == FM_W_FP8_E4M3 || nv4;
+  auto fmt_of = [&](int g) { return !fp8 ? 0 : (nv4 && g == G_GU) ? 2 : 1; };
+  auto row_bytes = [&](int g) -> uint64_t { const int f = fmt_of(g); return f == 0 ? 128 : f == 1 ? 64 : 36; };
   // Per-layer packing jobs (identical for every layer) and CTA spans.
   std::vector<PackChunk> jobs;
   std::vector<int32_t> rows;
@@ -310,9 +315,9 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
         pc.nrows = (uint16_t)ng;
         pc.mat = (uint8_t)g;
         pc.kb = (uint32_t)(ks * gp.nchunk + i);
-        pc.fp8 = fp8 ? 1 : 0;
+        pc.fp8 = (uint8_t)fmt_of(g);
         jobs.push_back(pc);
-        off += (uint64_t)ng * row_bytes;
+        off += (uint64_t)ng * row_bytes(g);
       }
     }
   }
@@ -341,6 +346,7 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
     h->pack_jobs = jobs;
     h->pack_rows = rows;
     h->row_scale.assign((size_t)c.n_layers * (mrows[0] + mrows[1] + mrows[2] + mrows[3]), 0.f);
+    if (nv4) h->nv4_g.assign((size_t)2 * c.n_layers, 1.f);
     DALLOC(h->wscale, (size_t)c.n_layers * h->sc_stride * 4);
   }
   std::vector<float> sc_host(fp8 ? (size_t)c.n_layers * h->sc_stride : 0, 0.f);
@@ -397,8 +403,9 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   if (e == cudaSuccess) e = cudaMalloc(&tmp[3], sz_dn * 2);
   if (e == cudaSuccess) e = cudaMalloc(&tmp[4], jobs.size() * sizeof(PackChunk) + rows.size() * 4 + 64);
   if (e == cudaSuccess) e = cudaMalloc(&tmp[5], 8 * sizeof(void*) + 4 * sizeof(int));
-  // E4M3: codes of the four linears and their row scales
-  if (e == cudaSuccess && fp8) e = cudaMalloc(&tmp[6], sz_qkv + sz_o + sz_gu + sz_dn);
+  // E4M3: codes of the four linears and their row scales (NVFP4 gate_up:
+  // one code per byte, then its block scales, two tensor scales, the amax word)
+  if (e == cudaSuccess && fp8) e = cudaMalloc(&tmp[6], sz_qkv + sz_o + sz_gu + sz_dn + sz_gu / 16 + 64);
   if (e == cudaSuccess && fp8) e = cudaMalloc(&tmp[7], (size_t)(mrows[0] + mrows[1] + mrows[2] + mrows[3]) * 4);
   if (e == cudaSuccess && h->batched)
     e = cudaMalloc(&tmp[8], bjobs.size() * sizeof(PackChunk) + brows.size() * 4 + 64);
@@ -417,11 +424,17 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
     const int matk[4] = {d, qn, d, F};
     uint8_t* q8[4] = {};
     float* rs[4] = {};
+    uint8_t* sb4 = nullptr;     // NVFP4 gate_up block scales [2F][d/16]
+    float* g4 = nullptr;        // [2]: gate, up tensor scales
+    unsigned int* amax4 = nullptr;
     if (fp8) {
       q8[0] = static_cast<uint8_t*>(tmp[6]);
       q8[1] = q8[0] + sz_qkv;
       q8[2] = q8[1] + sz_o;
       q8[3] = q8[2] + sz_gu;
+      sb4 = q8[3] + sz_dn;
+      g4 = reinterpret_cast<float*>(sb4 + sz_gu / 16 + 16 - (sz_gu / 16) % 16);
+      amax4 = reinterpret_cast<unsigned int*>(g4 + 4);
       rs[0] = static_cast<float*>(tmp[7]);
       for (int g = 1; g < 4; ++g) rs[g] = rs[g - 1] + mrows[g - 1];
     }
@@ -454,9 +467,24 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
         // R8: per-row absmax / 448 and E4M3 codes of every linear, then the
         // codes go into the arena and the scales into the packed-order table
         for (int g = 0; g < 4 && e == cudaSuccess; ++g) e = launch_fp8_quantize(mats[g], mrows[g], matk[g], rs[g], q8[g], 0);
+        if (e == cudaSuccess && nv4) {
+          // R10 for gate and up separately (their own tensor scales), over the
+          // E4M3 codes of gate_up, which only the scale table below still reads
+          for (int t = 0; t < 2 && e == cudaSuccess; ++t)
+            e = launch_nvfp4_quantize(mats[G_GU] + (size_t)t * F * d, F, d, amax4, q8[G_GU] + (size_t)t * F * d,
+                                      sb4 + (size_t)t * F * (d / 16), g4 + t, 0);
+        }
         if (e == cudaSuccess)
           e = launch_pack8(d_jobs, (int)jobs.size(), d_rows, reinterpret_cast<const uint8_t* const*>(d_mats), d_matk,
                            h->arena + (size_t)l * off, 0);
+        if (e == cudaSuccess && nv4)
+          e = launch_pack_nvfp4(d_jobs, (int)jobs.size(), d_rows, q8[G_GU], sb4, d, h->arena + (size_t)l * off, 0);
+        float gh[2] = {1.f, 1.f};
+        if (e == cudaSuccess && nv4) e = cudaMemcpy(gh, g4, 8, cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess && nv4) {
+          h->nv4_g[2 * l] = gh[0];
+          h->nv4_g[2 * l + 1] = gh[1];
+        }
         float* lrs = h->row_scale.data() + (size_t)l * (mrows[0] + mrows[1] + mrows[2] + mrows[3]);
         if (e == cudaSuccess)
           e = cudaMemcpy(lrs, rs[0], (size_t)(mrows[0] + mrows[1] + mrows[2] + mrows[3]) * 4, cudaMemcpyDeviceToHost);
@@ -464,7 +492,11 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
           const float* src = lrs;
           for (int g = 0; g < 4; ++g) {
             float* dst = sc_host.data() + (size_t)l * h->sc_stride + h->sc_off[g];
-            for (size_t i = 0; i < sc_src[g].size(); ++i) dst[i] = sc_src[g][i] >= 0 ? src[sc_src[g][i]] : 0.f;
+            for (size_t i = 0; i < sc_src[g].size(); ++i) {
+              const int sr = sc_src[g][i];
+              // NVFP4 gate_up columns carry their tensor's scale (gate rows, then up rows)
+              dst[i] = sr < 0 ? 0.f : (nv4 && g == G_GU) ? h->nv4_g[2 * l + (sr < F ? 0 : 1)] : src[sr];
+            }
             src += mrows[g];
           }
         }
@@ -574,7 +606,7 @@ fm_status check_config(const fm_config* c) {
   if (c->max_steps > kRows) return set_err(h, FM_ERR_INVALID_ARG, "max_steps must be <= %d", kRows);
   if (!(c->rms_eps > 0.f) || !(c->rope_base > 0.f))
     return set_err(h, FM_ERR_INVALID_ARG, "rms_eps and rope_base must be positive");
-  if (c->wtype != FM_W_BF16 && c->wtype != FM_W_FP8_E4M3)
+  if (c->wtype != FM_W_BF16 && c->wtype != FM_W_FP8_E4M3 && c->wtype != FM_W_FP8_NVFP4_GU)
     return set_err(h, FM_ERR_INVALID_ARG, "unknown wtype %d", c->wtype);
   return FM_OK;
 }
@@ -644,7 +676,8 @@ StepParams base_params(const fm_expert* h) {
   p.vcache = h->vcache;
   p.bar_count = h->bar_count;
   p.err = h->err_word;
-  p.fp8 = c.wtype == FM_W_FP8_E4M3 ? 1 : 0;
+  for (int g = 0; g < 4; ++g)
+    p.wfmt[g] = c.wtype == FM_W_BF16 ? 0 : (c.wtype == FM_W_FP8_NVFP4_GU && g == G_GU) ? 2 : 1;
   p.wscale = h->wscale;
   p.sc_stride = h->sc_stride;
   for (int g = 0; g < 4; ++g) p.sc_off[g] = h->sc_off[g];
@@ -1413,7 +1446,9 @@ fm_status fm_get_prefix_kv(fm_expert* h, int layer, int request, uint16_t* k, ui
 fm_status fm_get_fp8_weights(fm_expert* h, int layer, int which, uint8_t* codes, float* scale) {
   if (!h) return FM_ERR_INVALID_ARG;
   const fm_config& c = h->cfg;
-  if (c.wtype != FM_W_FP8_E4M3) return set_err(h, FM_ERR_INVALID_ARG, "handle holds bf16 weights");
+  if (c.wtype == FM_W_BF16) return set_err(h, FM_ERR_INVALID_ARG, "handle holds bf16 weights");
+  if (c.wtype == FM_W_FP8_NVFP4_GU && (which == 4 || which == 5))
+    return set_err(h, FM_ERR_INVALID_ARG, "gate_up is NVFP4 in this handle (fm_get_nvfp4_weights)");
   if (layer < 0 || layer >= c.n_layers || which < 0 || which > 6 || !codes || !scale)
     return set_err(h, FM_ERR_INVALID_ARG, "layer %d / which %d invalid or NULL buffer", layer, which);
   const int d = c.d_model, F = c.d_ff, qn = c.n_q_heads * c.head_dim, kn = c.n_kv_heads * c.head_dim;
@@ -1440,6 +1475,39 @@ fm_status fm_get_fp8_weights(fm_expert* h, int layer, int which, uint8_t* codes,
   size_t base = (size_t)layer * (mrows[0] + mrows[1] + mrows[2] + mrows[3]);
   for (int i = 0; i < g; ++i) base += mrows[i];
   std::memcpy(scale, h->row_scale.data() + base + r0, (size_t)R * 4);
+  return FM_OK;
+}
+
+fm_status fm_get_nvfp4_weights(fm_expert* h, int layer, int which, uint8_t* codes, uint8_t* block_scales,
+                               float* g) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  const fm_config& c = h->cfg;
+  if (c.wtype != FM_W_FP8_NVFP4_GU) return set_err(h, FM_ERR_INVALID_ARG, "handle has no NVFP4 weights");
+  if (layer < 0 || layer >= c.n_layers || (which != 4 && which != 5) || !codes || !block_scales || !g)
+    return set_err(h, FM_ERR_INVALID_ARG, "layer %d / which %d invalid or NULL buffer", layer, which);
+  const int d = c.d_model, F = c.d_ff, r0 = which == 4 ? 0 : F;
+  CK(cudaSetDevice(h->device));
+  std::vector<uint8_t> lay(h->layer_bytes);
+  CK(cudaMemcpy(lay.data(), h->arena + (size_t)layer * h->layer_bytes, h->layer_bytes, cudaMemcpyDeviceToHost));
+  std::memset(codes, 0, (size_t)F * d);
+  std::memset(block_scales, 0, (size_t)F * (d / 16));
+  for (const PackChunk& pc : h->pack_jobs) {
+    if (pc.mat != G_GU) continue;
+    const int R = pc.nrows;
+    for (int q = 0; q < R; ++q) {
+      const int sr = h->pack_rows[pc.rowidx_off + q];
+      if (sr < r0 || sr >= r0 + F) continue;
+      const uint8_t* crow = lay.data() + pc.dst_off + (size_t)q * 32;
+      const uint8_t* srow = lay.data() + pc.dst_off + (size_t)R * 32 + (size_t)q * 4;
+      uint8_t* out = codes + (size_t)(sr - r0) * d + (size_t)pc.kb * 64;
+      for (int i = 0; i < 32; ++i) {
+        out[2 * i] = crow[i] & 0xF;
+        out[2 * i + 1] = crow[i] >> 4;
+      }
+      std::memcpy(block_scales + (size_t)(sr - r0) * (d / 16) + (size_t)pc.kb * 4, srow, 4);
+    }
+  }
+  *g = h->nv4_g[2 * layer + (which == 4 ? 0 : 1)];
   return FM_OK;
 }
 

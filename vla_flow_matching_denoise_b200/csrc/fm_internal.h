@@ -74,7 +74,9 @@ struct StepParams {
   // weights
   const uint8_t* arena;      // packed per-layer weights (bf16 image or E4M3 codes)
   uint64_t layer_bytes;      // bytes of one layer in the arena
-  int fp8;                   // 1: the arena holds E4M3 codes, widened in shared memory
+  int wfmt[4];               // per linear: 0 bf16 image, 1 E4M3 rows (64 B), 2 NVFP4 rows
+                             // (32 B of codes, then 4 B of block scales per row); 1 and 2
+                             // are widened to bf16 in shared memory
   const float* wscale;       // fp8: [L][sc_stride] fp32 row scales by packed channel; else null
   int sc_stride;             // floats per layer in wscale
   int sc_off[4];             // first entry of each linear inside a layer's table
@@ -198,7 +200,7 @@ struct PackChunk {
   uint32_t rowidx_off;
   uint16_t nrows;
   uint8_t mat;
-  uint8_t fp8;
+  uint8_t fp8;               // format: 0 bf16, 1 E4M3, 2 NVFP4
   uint32_t kb;
 };
 

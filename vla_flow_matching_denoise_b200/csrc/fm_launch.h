@@ -13,6 +13,10 @@ cudaError_t launch_pack(const PackChunk* chunks, int nchunks, const int32_t* row
                         cudaStream_t st);
 cudaError_t launch_pack8(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
                          const uint8_t* const* mats, const int* mat_k, uint8_t* dst, cudaStream_t st);
+cudaError_t launch_nvfp4_quantize(const uint16_t* w, int rows, int K, unsigned int* amax_scratch, uint8_t* codes,
+                                  uint8_t* sb, float* g, cudaStream_t st);
+cudaError_t launch_pack_nvfp4(const PackChunk* chunks, int nchunks, const int32_t* rowidx, const uint8_t* codes,
+                              const uint8_t* sb, int K, uint8_t* dst, cudaStream_t st);
 cudaError_t launch_fp8_quantize(const uint16_t* w, int rows, int K, float* scale, uint8_t* q,
                                 cudaStream_t st);
 cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, const int* lens, int Hkv, int hd, int S_max,

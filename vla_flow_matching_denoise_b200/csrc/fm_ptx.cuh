@@ -321,6 +321,33 @@ __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
   return r;
 }
 
+// Two E2M1 codes (low nibble = first element) -> two f16 values (low half =
+// first), exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t h2;
+  asm("{\n\t.reg .b8 b;\n\tcvt.u8.u32 b, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, b;\n\t}" : "=r"(h2) : "r"(byte));
+  return h2;
+}
+// An E4M3 code -> its value as f16 in both halves, exact (E4M3 values are f16 values).
+__device__ __forceinline__ uint32_t e4m3_to_f16x2_bcast(uint32_t code) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"((uint16_t)((code & 0xFFu) * 0x101u)));
+  return h2;
+}
+// f16x2 product (exact when both factors have few significant bits), then the
+// two values as bf16x2 (exact: f16 -> f32 -> bf16 of a value with <= 8
+// significant bits and an exponent inside the bf16 range).
+__device__ __forceinline__ uint32_t f16x2_mul_to_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t p, r;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(p) : "r"(a), "r"(b));
+  float lo, hi;
+  asm("{\n\t.reg .f16 x, y;\n\tmov.b32 {x, y}, %2;\n\tcvt.f32.f16 %0, x;\n\tcvt.f32.f16 %1, y;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(p));
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 // ----------------------------------------------------------------- mma.sync (attention)
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
                                         uint32_t& r3) {

@@ -210,9 +210,10 @@ __device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* 
     nch[g] = ng > 0 ? (uint32_t)p.g[g].nchunk : 0u;
     bytes[g] = (uint32_t)ng * 128u;
   }
-  // E4M3: a chunk's codes (half its bf16 size) land in the upper half of its
-  // slot and are widened in place
-  const uint32_t shift = p.fp8 ? 1u : 0u;
+  // E4M3 / NVFP4: a chunk's codes land at the end of its slot and are
+  // widened in place; copy bytes per chunk row: 128 (bf16), 64, 36
+  uint32_t rowb[4];
+  for (int g = 0; g < 4; ++g) rowb[g] = p.wfmt[g] == 0 ? 128u : p.wfmt[g] == 1 ? 64u : 36u;
   uint32_t st[kRingSlots], en[kRingSlots];
   uint32_t head = 0, tail = 0, pos = 0;
   const uint32_t span0 = p.span_off[cta];
@@ -246,7 +247,7 @@ __device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* 
           en[slot] = at + sz;
           if (p.tlog != nullptr && (int)head < p.tlog_chunks)
             p.tlog[(size_t)cta * p.tlog_stride + p.tlog_chunk_off + p.tlog_chunks + head] = gtimer();
-          const uint32_t csz = sz >> shift;
+          const uint32_t csz = (sz >> 7) * rowb[g];
           mbar_arrive_expect_tx(smem_u32(&ctl->full[slot]), csz);
           bulk_g2s(smem_u32(ring + at + (sz - csz)), src, csz, smem_u32(&ctl->full[slot]), pol);
           src += csz;
@@ -283,38 +284,77 @@ __device__ __noinline__ void converter(const StepParams& p, uint8_t* ring, Ctrl*
   for (int s = p.step0; s < p.step1 && good; ++s) {
     for (int l = p.layer0; l < p.layer1 && good; ++l) {
       for (int g = 0; g < 4 && good; ++g) {
-        const int npieces = (int)(bytes[g] >> 5);   // ng rows x 4 pieces
+        const int npieces = (int)(bytes[g] >> 5);   // E4M3: ng rows x 4 pieces
         for (uint32_t c = 0; c < nch[g]; ++c, ++it) {
           const uint32_t at = ring_place(pos, bytes[g]);
           const uint32_t slot = it % kRingSlots;
+          if (p.wfmt[g] == 0) continue;   // bf16 chunk: the MMA warp waits on `full` itself
           if (!wait_ab(smem_u32(&ctl->full[slot]), (it / kRingSlots) & 1, p.spin_budget, &ctl->abort)) {
             good = false;
             break;
           }
           uint8_t* base = ring + at;
-          const uint8_t* codes = base + (bytes[g] >> 1);
-          uint4 v[kMaxPieces];
+          if (p.wfmt[g] == 1) {
+            const uint8_t* codes = base + (bytes[g] >> 1);
+            uint4 v[kMaxPieces];
 #pragma unroll
-          for (int j = 0; j < kMaxPieces; ++j) {
-            const int i = ctid + kCT * j;
-            if (i < npieces) v[j] = *reinterpret_cast<const uint4*>(codes + 16 * i);
-          }
-          named_bar_sync(2, kCT);
-#pragma unroll
-          for (int j = 0; j < kMaxPieces; ++j) {
-            const int i = ctid + kCT * j;
-            if (i >= npieces) break;
-            const int r = i >> 2, q = i & 3;   // row, 16-code quarter -> bf16 pieces 2q, 2q + 1
-            const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
-            uint32_t o[8];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              o[2 * k] = e4m3x2_to_bf16x2((uint16_t)(w[k] & 0xFFFFu));
-              o[2 * k + 1] = e4m3x2_to_bf16x2((uint16_t)(w[k] >> 16));
+            for (int j = 0; j < kMaxPieces; ++j) {
+              const int i = ctid + kCT * j;
+              if (i < npieces) v[j] = *reinterpret_cast<const uint4*>(codes + 16 * i);
             }
-            uint8_t* row = base + (r >> 3) * 1024 + (r & 7) * 128;
-            *reinterpret_cast<uint4*>(row + (((2 * q) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
-            *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+            named_bar_sync(2, kCT);
+#pragma unroll
+            for (int j = 0; j < kMaxPieces; ++j) {
+              const int i = ctid + kCT * j;
+              if (i >= npieces) break;
+              const int r = i >> 2, q = i & 3;   // row, 16-code quarter -> bf16 pieces 2q, 2q + 1
+              const uint32_t w[4] = {v[j].x, v[j].y, v[j].z, v[j].w};
+              uint32_t o[8];
+#pragma unroll
+              for (int k = 0; k < 4; ++k) {
+                o[2 * k] = e4m3x2_to_bf16x2((uint16_t)(w[k] & 0xFFFFu));
+                o[2 * k + 1] = e4m3x2_to_bf16x2((uint16_t)(w[k] >> 16));
+              }
+              uint8_t* row = base + (r >> 3) * 1024 + (r & 7) * 128;
+              *reinterpret_cast<uint4*>(row + (((2 * q) ^ (r & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+              *reinterpret_cast<uint4*>(row + (((2 * q + 1) ^ (r & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+            }
+          } else {
+            // NVFP4 rows: 32 bytes of E2M1 codes (two per byte, first in the low
+            // nibble), then 4 E4M3 scales, one per 16-column block; every code x
+            // scale product is exact in f16 and in bf16
+            constexpr int kMaxRows = 256 / kCT;
+            const int R = (int)(bytes[g] >> 7);
+            const uint8_t* src = base + bytes[g] - (uint32_t)R * 36u;
+            uint4 c0[kMaxRows], c1[kMaxRows];
+            uint32_t scw[kMaxRows];
+#pragma unroll
+            for (int j = 0; j < kMaxRows; ++j) {
+              const int q = ctid + kCT * j;
+              if (q < R) {
+                c0[j] = *reinterpret_cast<const uint4*>(src + 32 * q);
+                c1[j] = *reinterpret_cast<const uint4*>(src + 32 * q + 16);
+                scw[j] = *reinterpret_cast<const uint32_t*>(src + 32 * R + 4 * q);
+              }
+            }
+            named_bar_sync(2, kCT);
+#pragma unroll
+            for (int j = 0; j < kMaxRows; ++j) {
+              const int q = ctid + kCT * j;
+              if (q >= R) break;
+              const uint32_t cw[8] = {c0[j].x, c0[j].y, c0[j].z, c0[j].w, c1[j].x, c1[j].y, c1[j].z, c1[j].w};
+              uint8_t* row = base + (q >> 3) * 1024 + (q & 7) * 128;
+#pragma unroll
+              for (int b = 0; b < 4; ++b) {
+                const uint32_t s2 = e4m3_to_f16x2_bcast(scw[j] >> (8 * b));
+                uint32_t o[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k)
+                  o[k] = f16x2_mul_to_bf16x2(e2m1x2_to_f16x2((cw[2 * b + (k >> 2)] >> (8 * (k & 3))) & 0xFFu), s2);
+                *reinterpret_cast<uint4*>(row + (((2 * b) ^ (q & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<uint4*>(row + (((2 * b + 1) ^ (q & 7)) << 4)) = make_uint4(o[4], o[5], o[6], o[7]);
+              }
+            }
           }
           // generic-proxy stores must be visible to the tensor cores' reads
           fence_proxy_async_smem();
@@ -359,7 +399,7 @@ __device__ __noinline__ void mma_issuer(const StepParams& p, uint8_t* ring, uint
         for (uint32_t c = 0; c < nch[g]; ++c, ++it) {
           const uint32_t at = ring_place(pos, bytes[g]);
           const uint32_t slot = it % kRingSlots;
-          if (!wait_ab(smem_u32(p.fp8 ? &ctl->conv[slot] : &ctl->full[slot]), (it / kRingSlots) & 1,
+          if (!wait_ab(smem_u32(p.wfmt[g] ? &ctl->conv[slot] : &ctl->full[slot]), (it / kRingSlots) & 1,
                        p.spin_budget, &ctl->abort)) {
             good = false;
             break;
@@ -1270,7 +1310,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_cons
     if (lane == 0) mma_issuer(p, ring, work, ctl, tmem, cluster);
     __syncwarp();
   } else if (warp >= 2 + kComputeWarps) {
-    if (p.fp8) converter(p, ring, ctl, cluster, threadIdx.x - 32 * (2 + kComputeWarps));
+    if (p.wfmt[0] | p.wfmt[1] | p.wfmt[2] | p.wfmt[3])
+      converter(p, ring, ctl, cluster, threadIdx.x - 32 * (2 + kComputeWarps));
   } else {
     Ctx c;
     c.p = &p;

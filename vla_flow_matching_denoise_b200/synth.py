@@ -54,6 +54,7 @@ class ExpertShape:
     rope_base: float = 10000.0
     weight_std: float = 0.02
     fp8: bool = False
+    nvfp4_gu: bool = False     # E4M3 linears with an NVFP4 gate_up
 
     @property
     def n_mod(self) -> int:
@@ -94,6 +95,8 @@ WORKLOADS: Dict[str, ExpertShape] = {
     "lingbot_p832_n50_a55": ExpertShape(36, 1024, 16, 2, 128, 4096, 55, 832, 50),
     # FP8 E4M3 per-output-channel weights, bf16 activations and KV.
     "lingbot_fp8_p256_n10": ExpertShape(36, 1024, 16, 2, 128, 4096, 75, 256, 10, fp8=True),
+    # E4M3 linears with an NVFP4 gate_up (the Thor page's weight formats).
+    "lingbot_nvfp4_p256_n10": ExpertShape(36, 1024, 16, 2, 128, 4096, 75, 256, 10, nvfp4_gu=True),
     # 64 independent requests on one GPU.
     "lingbot_b64_p256_n10": ExpertShape(36, 1024, 16, 2, 128, 4096, 75, 256, 10, batch=64),
     # Four layers of the LingBot-shaped expert: the profiling case (same layer
