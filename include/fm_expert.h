@@ -124,9 +124,12 @@ typedef struct fm_weights {
 typedef struct fm_expert fm_expert;
 
 /* Create a handle on `device`.  COPIES every weight into a library-owned,
- * kernel-ready arena (and, for FM_W_FP8_E4M3, quantises the per-layer
- * linears itself); the caller may free its copies when the call returns.
- * Allocates every buffer the loop needs for the capacities in `cfg`.
+ * kernel-ready arena (and, for FM_W_FP8_E4M3 / FM_W_FP8_NVFP4_GU, quantises
+ * the per-layer linears itself); the caller may free its copies when the call
+ * returns.  Allocates every buffer the loop needs for the capacities in
+ * `cfg`; a bf16 handle with max_batch >= 2 also packs the weights a second
+ * time in the batched path's tile layout (B >= 2 requests then advance through
+ * each Euler step together as M = B*T-row tensor-core GEMMs).
  * Returns FM_ERR_INVALID_ARG for a bad config, FM_ERR_UNSUPPORTED for a
  * device that is not sm_100, FM_ERR_OOM when the arena does not fit. */
 fm_status fm_expert_create(const fm_config *cfg, const fm_weights *w, int device,

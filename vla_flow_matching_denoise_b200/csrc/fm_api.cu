@@ -315,7 +315,7 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
         pc.nrows = (uint16_t)ng;
         pc.mat = (uint8_t)g;
         pc.kb = (uint32_t)(ks * gp.nchunk + i);
-        pc.fp8 = (uint8_t)fmt_of(g);
+        pc.fmt = (uint8_t)fmt_of(g);
         jobs.push_back(pc);
         off += (uint64_t)ng * row_bytes(g);
       }

@@ -77,7 +77,8 @@ struct StepParams {
   int wfmt[4];               // per linear: 0 bf16 image, 1 E4M3 rows (64 B), 2 NVFP4 rows
                              // (32 B of codes, then 4 B of block scales per row); 1 and 2
                              // are widened to bf16 in shared memory
-  const float* wscale;       // fp8: [L][sc_stride] fp32 row scales by packed channel; else null
+  const float* wscale;       // quantised weights: [L][sc_stride] fp32 column scales by packed
+                             // channel (E4M3 row scale or NVFP4 tensor scale); bf16: null
   int sc_stride;             // floats per layer in wscale
   int sc_off[4];             // first entry of each linear inside a layer's table
   const uint32_t* span_off;  // [n_ctas + 1]: byte offset of each CTA's span in a layer
@@ -200,7 +201,7 @@ struct PackChunk {
   uint32_t rowidx_off;
   uint16_t nrows;
   uint8_t mat;
-  uint8_t fp8;               // format: 0 bf16, 1 E4M3, 2 NVFP4
+  uint8_t fmt;               // weight format: 0 bf16, 1 E4M3, 2 NVFP4
   uint32_t kb;
 };
 

@@ -36,7 +36,7 @@ __global__ void pack8_kernel(const PackChunk* __restrict__ chunks, const int32_t
                              const uint8_t* const* __restrict__ mats, const int* __restrict__ mat_k,
                              uint8_t* __restrict__ dst) {
   const PackChunk ch = chunks[blockIdx.x];
-  if (ch.fp8 != 1) return;   // not an E4M3 chunk (NVFP4 chunks have their own packer)
+  if (ch.fmt != 1) return;   // not an E4M3 chunk (NVFP4 chunks have their own packer)
   const uint8_t* src = mats[ch.mat];
   const int K = mat_k[ch.mat];
   const int pieces = ch.nrows * 4;
@@ -137,7 +137,7 @@ __global__ void pack_nvfp4_kernel(const PackChunk* __restrict__ chunks, const in
                                   const uint8_t* __restrict__ codes, const uint8_t* __restrict__ sb, int K,
                                   uint8_t* __restrict__ dst) {
   const PackChunk ch = chunks[blockIdx.x];
-  if (ch.fp8 != 2) return;   // only NVFP4 chunks
+  if (ch.fmt != 2) return;   // only NVFP4 chunks
   const int R = ch.nrows;
   for (int q = threadIdx.x; q < R; q += blockDim.x) {
     const int sr = rowidx[ch.rowidx_off + q];
