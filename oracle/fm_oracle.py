@@ -40,6 +40,9 @@ The pages print no formula, so the conventions below are the plainest readings
      nearest-even of (w / s_c) in fp32, saturated at 448; w' = q * s_c.
   R9 prefix cache rows: K = RoPE(x Wk^T) at positions 0 .. P-1, V = x Wv^T
      from each layer's prefix hidden states x, stored as bf16.
+  R11 E4M3 activations (the batched path's W8A8 option): each input row of
+     the four per-layer linears, taken in fp32, is quantised per token:
+     s = amax_row / 448 (fp32), y' = E4M3(y / s) s.
   R10 NVFP4 gate_up (with E4M3 R8 for the other linears): per tensor
      g = amax / (6 * 448) (fp32); per row and 16-column block
      s_b = E4M3 nearest-even of (amax_b / (6 g)) in fp32; codes = E2M1
@@ -182,13 +185,15 @@ class Weights:
 def expert_velocity(x: np.ndarray, m: np.ndarray, W: Weights, k_prefix: List[np.ndarray],
                     v_prefix: List[np.ndarray], eps: float, rope_base: float,
                     n_q_heads: int, n_kv_heads: int, out_bias: Optional[np.ndarray] = None,
-                    trace: Optional[List[Dict[str, np.ndarray]]] = None) -> np.ndarray:
+                    trace: Optional[List[Dict[str, np.ndarray]]] = None, act_fp8: bool = False) -> np.ndarray:
     """Velocity v(x, t) of one request's chunk.
 
     x: [T, A]; m: modulation row for this t; k_prefix / v_prefix: per layer
     [P, H_kv, hd] (already rotated).  If ``trace`` is a list, one dict of
-    intermediates per layer is appended, then a final dict.
+    intermediates per layer is appended, then a final dict.  ``act_fp8``
+    quantises the input rows of the four per-layer linears per token (R11).
     """
+    aq = fp8_quant_act if act_fp8 else (lambda a: a)
     dt_ = W.dtype
     T = x.shape[0]
     L = len(W.layers)
@@ -201,7 +206,7 @@ def expert_velocity(x: np.ndarray, m: np.ndarray, W: Weights, k_prefix: List[np.
         vp = v_prefix[l].astype(dt_)
         P, _, hd = kp.shape
         rec = {"h_in": h.copy()} if trace is not None else None
-        y = ada_rms(h, s_a, b_a, eps)
+        y = aq(ada_rms(h, s_a, b_a, eps))
         q = (y @ lw["wq"].T).reshape(T, n_q_heads, hd)
         kc = (y @ lw["wk"].T).reshape(T, n_kv_heads, hd)
         vc = (y @ lw["wv"].T).reshape(T, n_kv_heads, hd)
@@ -211,12 +216,12 @@ def expert_velocity(x: np.ndarray, m: np.ndarray, W: Weights, k_prefix: List[np.
         K = np.concatenate([kp, kc], axis=0)
         V = np.concatenate([vp, vc], axis=0)
         o = gqa_attention(q, K, V).reshape(T, n_q_heads * hd)
-        h = h + g_a * (o @ lw["wo"].T)
+        h = h + g_a * (aq(o) @ lw["wo"].T)
         if rec is not None:
             rec.update(q=q, k=kc, v=vc, o=o, h_mid=h.copy())
-        y = ada_rms(h, s_f, b_f, eps)
+        y = aq(ada_rms(h, s_f, b_f, eps))
         u = silu(y @ lw["w_gate"].T) * (y @ lw["w_up"].T)
-        h = h + g_f * (u @ lw["w_down"].T)
+        h = h + g_f * (aq(u) @ lw["w_down"].T)
         if rec is not None:
             rec.update(u=u, h_out=h.copy())
             trace.append(rec)
@@ -243,7 +248,7 @@ def euler(x0: np.ndarray, n: int, velocity: Callable[[np.ndarray, int, float], n
 
 def denoise(x0: np.ndarray, n: int, raw_weights: Dict, k_prefix, v_prefix, shape,
             dtype=np.float64, out_bias=None, W: Optional[Weights] = None,
-            velocities: Optional[List[np.ndarray]] = None) -> np.ndarray:
+            velocities: Optional[List[np.ndarray]] = None, act_fp8: bool = False) -> np.ndarray:
     """Denoise a batch of chunks: x0 [B, T, A] -> x_n [B, T, A].
 
     k_prefix / v_prefix: per layer bf16 bits [B, P, H_kv, hd].  All requests
@@ -261,7 +266,7 @@ def denoise(x0: np.ndarray, n: int, raw_weights: Dict, k_prefix, v_prefix, shape
 
         def vel(x, k, t, kp=kp, vp=vp):
             return expert_velocity(x, M[k], W, kp, vp, shape.rms_eps, shape.rope_base,
-                                   shape.n_q_heads, shape.n_kv_heads, out_bias).astype(np.float64)
+                                   shape.n_q_heads, shape.n_kv_heads, out_bias, act_fp8=act_fp8).astype(np.float64)
 
         rec = [] if velocities is not None else None
         out[b] = euler(x0[b], n, vel, rec)
@@ -337,6 +342,16 @@ def fp8_quantize_rows(w_bits: np.ndarray):
     scale = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
     ratio = (w / scale[:, None]).astype(np.float32)
     return e4m3_encode(ratio), scale
+
+
+def fp8_quant_act(y: np.ndarray) -> np.ndarray:
+    """R11: per-token E4M3 of activation rows (last axis), returned dequantised
+    in float64: s = amax_row / 448 in fp32 of the fp32 values, y' = E4M3(y / s) s."""
+    y32 = np.asarray(y, dtype=np.float32)
+    amax = np.max(np.abs(y32), axis=-1)
+    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    codes = e4m3_encode((y32 / s[..., None]).astype(np.float32))
+    return e4m3_decode(codes) * s[..., None].astype(np.float64)
 
 
 def fp8_dequantize_rows(codes: np.ndarray, scale: np.ndarray) -> np.ndarray:

@@ -447,3 +447,48 @@ def test_nvfp4_block_max_maps_to_six_and_zero_blocks():
     err = np.abs(deq - wd).reshape(3, 4, 16).max(axis=2)
     top = np.abs(wd).reshape(3, 4, 16).max(axis=2)
     assert np.all(err <= 0.35 * top + 1e-12)
+
+
+# --------------------------------------------------------------------------- E4M3 activations (R11)
+def test_fp8_quant_act_row_max_exact_zero_row_and_grid_round_trip():
+    y = np.array([[3.0, -1.5, 0.25, 0.0], [0.0, 0.0, 0.0, 0.0], [-7.0, 1.0, 2.0, 3.5]])
+    q = O.fp8_quant_act(y)
+    # the row maximum maps to code 448, i.e. to 448 * s with s the fp32 quotient
+    # amax / 448 (rounded, so 3/448 does not come back as exactly 3); a zero row stays zero
+    assert q[0, 0] == 448.0 * float(np.float32(3.0) / np.float32(448.0))
+    assert q[2, 0] == -7.0 and not q[1].any()
+    # values on the row's E4M3 grid round-trip exactly: s = 1/64 here
+    s = 7.0 / 448.0
+    grid = O.e4m3_decode(np.array([0x7E, 0x40, 0x38, 0x31], dtype=np.uint8)) * s   # 448 s, 2 s, 1 s, 0.5625 s
+    row = np.array([[-grid[0], grid[1], grid[2], grid[3]]])
+    assert np.array_equal(O.fp8_quant_act(row), row)
+    # relative error per entry is at most half an E4M3 step (2^-4) of its binade
+    r = np.random.default_rng(41).standard_normal((5, 64))
+    qr = O.fp8_quant_act(r)
+    big = np.abs(r) > np.max(np.abs(r), axis=1, keepdims=True) * 2.0 ** -6
+    assert np.all(np.abs(qr - r)[big] <= np.abs(r)[big] * 2.0 ** -4 + 1e-12)
+
+
+def test_act_fp8_quantises_the_inputs_of_the_four_linears(monkeypatch):
+    """R11 applies to the inputs of QKV, o_proj, gate_up and down, once each
+    per layer; with quantisation the chunk stays close to the plain one."""
+    s = synth.WORKLOADS["tiny"]
+    raw = synth.make_weights(s)
+    kp, vp = synth.make_prefix(s)
+    x0 = synth.make_x0(s)
+    seen = []
+    real = O.fp8_quant_act
+    W = O.Weights(raw, fp8=True)
+    monkeypatch.setattr(O, "fp8_quant_act", lambda a: seen.append(a.shape) or real(a))
+    M = O.time_modulation(np.array([1.0]), W.time_w1, W.time_w2)
+    O.expert_velocity(x0[0], M[0], W, [O.decode_bf16(k[0]) for k in kp], [O.decode_bf16(v[0]) for v in vp],
+                      s.rms_eps, s.rope_base,
+                      s.n_q_heads, s.n_kv_heads, act_fp8=True)
+    T, d, hq, F = s.chunk_len, s.d_model, s.n_q_heads * s.head_dim, s.d_ff
+    assert seen == [(T, d), (T, hq), (T, d), (T, F)] * s.n_layers
+    monkeypatch.setattr(O, "fp8_quant_act", real)
+    a = O.denoise(x0, s.steps, raw, kp, vp, s, W=W)
+    b = O.denoise(x0, s.steps, raw, kp, vp, s, W=W, act_fp8=True)
+    assert not np.array_equal(a, b)
+    c = np.dot(a.ravel(), b.ravel()) / np.linalg.norm(a) / np.linalg.norm(b)
+    assert c > 0.99
