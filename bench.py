@@ -103,7 +103,8 @@ def loop_bytes(shape: synth.ExpertShape, steps: int, batch: int) -> float:
         rows_8 = rows - ws["w_gate"][0] - ws["w_up"][0]
         wbytes = s.n_layers * ((per_layer - gu) * 1.0 + rows_8 * 4.0 + gu * (0.5 + 1.0 / 16) + 8.0)
     else:
-        wbytes = s.n_layers * (per_layer * (1.0 if s.fp8 else 2.0) + (rows * 4.0 if s.fp8 else 0.0))
+        q8 = s.fp8 or s.w8a8
+        wbytes = s.n_layers * (per_layer * (1.0 if q8 else 2.0) + (rows * 4.0 if q8 else 0.0))
     io = (int(np.prod(ws["in_proj"])) + int(np.prod(ws["out_proj"]))) * 2.0
     kv = batch * s.n_layers * 2 * (s.prefix_len + s.chunk_len) * s.n_kv_heads * s.head_dim * 2.0
     return steps * (wbytes + io + kv)
@@ -178,7 +179,7 @@ class OracleRunner:
         raw = synth.make_weights(shape, seed)
         kp, vp = synth.make_prefix(shape, seed, batch=1)
         self.x0 = synth.make_x0(shape, seed, batch=1)[0]
-        self.W = O.Weights(raw, fp8=shape.fp8)
+        self.W = O.Weights(raw, fp8=shape.fp8 or shape.w8a8, nvfp4_gu=shape.nvfp4_gu)
         self.kp = [O.decode_bf16(k[0]) for k in kp]
         self.vp = [O.decode_bf16(v[0]) for v in vp]
         try:
@@ -199,7 +200,7 @@ class OracleRunner:
             x = self.x0.astype(np.float64)
             for k in range(min(s.steps, n_sample - done)):
                 v = O.expert_velocity(x, M[k], self.W, self.kp, self.vp, s.rms_eps, s.rope_base, s.n_q_heads,
-                                      s.n_kv_heads)
+                                      s.n_kv_heads, act_fp8=s.w8a8)
                 x = x + dt * v
                 done += 1
         return time.perf_counter() - t0
@@ -354,7 +355,11 @@ def main():
     lb = loop_bytes(shape, n, B)
     achieved = lb / (ms_loop / 1000.0) / 1e9
     lf = loop_flops(shape, n, B)
-    batched = B >= 2 and not shape.fp8 and not shape.nvfp4_gu
+    batched = shape.w8a8 or (B >= 2 and not shape.fp8 and not shape.nvfp4_gu)
+    # an E4M3 contraction takes the measured bf16 peak x the nominal fp8 / bf16 ratio (4.5 / 2.25)
+    tpeak = tflops_sus * (2.0 if shape.w8a8 else 1.0)
+    tpeak_burst = tflops * (2.0 if shape.w8a8 else 1.0)
+    per_layer_launches = 9 if shape.w8a8 else 7   # W8A8: two row-quantiser passes per layer
     traffic = None
     rec = NCU_TRAFFIC.get(args.workload)
     if rec and rec.get("source_hash") == kernel_source_hash():
@@ -368,26 +373,29 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_call, "ms_per_chunk": ms_call,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "e4m3" if shape.w8a8 else "bf16",
         "data": "synthetic",
         "config": {"workload": args.workload, "layers": shape.n_layers, "d_model": shape.d_model,
                    "heads": f"{shape.n_q_heads}q/{shape.n_kv_heads}kv x {shape.head_dim}",
                    "d_ff": shape.d_ff, "prefix_len": shape.prefix_len,
                    "chunk": f"{shape.chunk_len}x{shape.action_dim}", "euler_steps": n,
                    "requests_per_gpu": B,
-                   "weights": "fp8-e4m3 + nvfp4 gate_up" if shape.nvfp4_gu else "fp8-e4m3" if shape.fp8 else "bf16",
+                   "weights": ("fp8-e4m3 + nvfp4 gate_up" if shape.nvfp4_gu else "fp8-e4m3" if shape.fp8
+                               else "fp8-e4m3, per-token e4m3 activations" if shape.w8a8 else "bf16"),
                    "parallelism": f"replicas x{ws}",
                    "l2": f"inputs larger than L2: {loop_bytes(shape, 1, B) / 1e9:.3f} GB of weights and KV "
                          "stream per Euler step (L2 126 MB)"},
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_chunk": ms_e2e / args.steps,
                 "h2d_bytes_per_step": int(x0.nbytes), "d2h_bytes_per_step": int(x0.nbytes)},
-        "gpu_launches": args.steps * ((2 + n * (7 * shape.n_layers + 2)) if batched else (2 + B)),
-        "roofline": ({"bound": "tensor", "achieved": lf / (ms_loop / 1000.0) / 1e12, "peak": tflops_sus,
-                      "unit": "TFLOP/s", "frac": lf / (ms_loop / 1000.0) / 1e12 / tflops_sus,
-                      "traffic": traffic, "peak_kind": peak_kind + " sustained bf16",
+        "gpu_launches": args.steps * ((2 + n * (per_layer_launches * shape.n_layers + 2)) if batched else (2 + B)),
+        "roofline": ({"bound": "tensor", "achieved": lf / (ms_loop / 1000.0) / 1e12, "peak": tpeak,
+                      "unit": "TFLOP/s", "frac": lf / (ms_loop / 1000.0) / 1e12 / tpeak,
+                      "traffic": traffic,
+                      "peak_kind": peak_kind + (" sustained bf16 x 2 (fp8)" if shape.w8a8 else " sustained bf16"),
                       "kernel": "batched loop (bgemm + attention + row kernels)", "flops_per_launch": lf,
-                      "ms_per_launch": ms_loop, "frac_of_burst": lf / (ms_loop / 1000.0) / 1e12 / tflops}
+                      "ms_per_launch": ms_loop, "frac_of_burst": lf / (ms_loop / 1000.0) / 1e12 / tpeak_burst}
                      if batched else
                      {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s",
                       "frac": achieved / hbm, "traffic": traffic, "peak_kind": peak_kind,

@@ -72,11 +72,20 @@ typedef enum fm_wtype {
   FM_W_BF16 = 0,            /* per-layer linears kept in bf16                   */
   FM_W_FP8_E4M3 = 1,        /* per-layer linears quantised to E4M3, one fp32
                                scale per output row (s = absmax / 448)          */
-  FM_W_FP8_NVFP4_GU = 2     /* E4M3 as above for wq/wk/wv/wo/w_down; w_gate and
+  FM_W_FP8_NVFP4_GU = 2,    /* E4M3 as above for wq/wk/wv/wo/w_down; w_gate and
                                w_up in NVFP4: E2M1 codes, one E4M3 scale per 16
                                inputs, one fp32 scale per tensor ("LingBot-VLA
                                on Thor (sm_110)", §1: FP8 weights with an FP4
                                gate_up)                                          */
+  FM_W_W8A8_E4M3 = 3        /* E4M3 weights as FM_W_FP8_E4M3 and E4M3 inputs of
+                               the four per-layer linears, one fp32 scale per
+                               token row (s = amax_row / 448); every batch size
+                               runs on the batched tensor-core path (kind::f8f6f4
+                               MMAs).  Needs d_model a multiple of 256 and at
+                               most 1024, n_q_heads*head_dim and d_ff multiples
+                               of 256 and at most 4096, head_dim 64 or 128.
+                               The trace and profile hooks of the one-request
+                               kernel return FM_ERR_UNSUPPORTED.                 */
 } fm_wtype;
 
 /* Model shape and capacities.  Requirements (checked by fm_expert_create):
@@ -124,14 +133,16 @@ typedef struct fm_weights {
 typedef struct fm_expert fm_expert;
 
 /* Create a handle on `device`.  COPIES every weight into a library-owned,
- * kernel-ready arena (and, for FM_W_FP8_E4M3 / FM_W_FP8_NVFP4_GU, quantises
- * the per-layer linears itself); the caller may free its copies when the call
+ * kernel-ready arena (and, for FM_W_FP8_E4M3 / FM_W_FP8_NVFP4_GU /
+ * FM_W_W8A8_E4M3, quantises the per-layer linears itself); the caller may free its copies when the call
  * returns.  Allocates every buffer the loop needs for the capacities in
  * `cfg`; a bf16 handle with max_batch >= 2 also packs the weights a second
  * time in the batched path's tile layout (B >= 2 requests then advance through
- * each Euler step together as M = B*T-row tensor-core GEMMs).
+ * each Euler step together as M = B*T-row tensor-core GEMMs); a
+ * FM_W_W8A8_E4M3 handle packs only that layout, in E4M3.
  * Returns FM_ERR_INVALID_ARG for a bad config, FM_ERR_UNSUPPORTED for a
- * device that is not sm_100, FM_ERR_OOM when the arena does not fit. */
+ * device that is not sm_100 or a W8A8 shape the batched path cannot take,
+ * FM_ERR_OOM when the arena does not fit. */
 fm_status fm_expert_create(const fm_config *cfg, const fm_weights *w, int device,
                            fm_expert **out);
 
@@ -229,8 +240,9 @@ fm_status fm_trace_velocity(fm_expert *h, const float *x, int step_index, int st
 
 /* Test hook: the E4M3 codes [out, in] and fp32 row scales [out] the handle
  * holds for per-layer linear `which` (0 wq, 1 wk, 2 wv, 3 wo, 4 w_gate,
- * 5 w_up, 6 w_down) of `layer`; host buffers.  FM_ERR_INVALID_ARG for a bf16
- * handle. */
+ * 5 w_up, 6 w_down) of `layer`; host buffers, read back from the arena the
+ * kernels stream (for FM_W_W8A8_E4M3 the batched GEMM's tile arena).
+ * FM_ERR_INVALID_ARG for a bf16 handle. */
 fm_status fm_get_fp8_weights(fm_expert *h, int layer, int which, uint8_t *codes,
                              float *scale);
 
@@ -241,6 +253,15 @@ fm_status fm_get_fp8_weights(fm_expert *h, int layer, int which, uint8_t *codes,
  * Dequantised weight = e2m1(code) * e4m3(block scale) * g. */
 fm_status fm_get_nvfp4_weights(fm_expert *h, int layer, int which, uint8_t *codes,
                                uint8_t *block_scales, float *g);
+
+/* Test hook: R11 per-token E4M3 of `M` bf16 rows x[M, K] (host or device)
+ * with the row-quantiser kernel of the W8A8 path (the pass that follows
+ * attention and SwiGLU): s_m = amax_m / 448 in fp32 (1 for a zero row),
+ * codes = E4M3(x / s_m), nearest-even, saturating.  Writes host codes
+ * [M, K] and host scales [M].  K a multiple of 256 and at most 4096.
+ * Allocates and frees temporary device memory; synchronises `stream`. */
+fm_status fm_quantize_act_e4m3(fm_expert *h, const uint16_t *x, int M, int K, uint8_t *codes,
+                               float *scales, void *stream);
 
 /* Profiling hook: runs `iters` times the two kernels of one denoise (the
  * time MLP, then the denoise loop for every request) outside any graph, with

@@ -248,14 +248,19 @@ def euler(x0: np.ndarray, n: int, velocity: Callable[[np.ndarray, int, float], n
 
 def denoise(x0: np.ndarray, n: int, raw_weights: Dict, k_prefix, v_prefix, shape,
             dtype=np.float64, out_bias=None, W: Optional[Weights] = None,
-            velocities: Optional[List[np.ndarray]] = None, act_fp8: bool = False) -> np.ndarray:
+            velocities: Optional[List[np.ndarray]] = None, act_fp8: Optional[bool] = None) -> np.ndarray:
     """Denoise a batch of chunks: x0 [B, T, A] -> x_n [B, T, A].
 
     k_prefix / v_prefix: per layer bf16 bits [B, P, H_kv, hd].  All requests
     share the modulation rows (same t grid); each has its own prefix and x0.
+    Without W, the weights follow the shape's formats; act_fp8 None follows
+    the shape's W8A8 flag (R11).
     """
+    w8a8 = bool(getattr(shape, "w8a8", False))
+    if act_fp8 is None:
+        act_fp8 = w8a8
     if W is None:
-        W = Weights(raw_weights, dtype, fp8=shape.fp8)
+        W = Weights(raw_weights, dtype, fp8=shape.fp8 or w8a8, nvfp4_gu=bool(getattr(shape, "nvfp4_gu", False)))
     ts, _ = time_schedule(n)
     M = time_modulation(ts, W.time_w1, W.time_w2, dtype)
     x0 = np.asarray(x0, dtype=np.float64)
@@ -344,13 +349,21 @@ def fp8_quantize_rows(w_bits: np.ndarray):
     return e4m3_encode(ratio), scale
 
 
-def fp8_quant_act(y: np.ndarray) -> np.ndarray:
-    """R11: per-token E4M3 of activation rows (last axis), returned dequantised
-    in float64: s = amax_row / 448 in fp32 of the fp32 values, y' = E4M3(y / s) s."""
+def fp8_quantize_act(y: np.ndarray):
+    """R11: per-token E4M3 of activation rows (last axis) of the fp32 values:
+    s = amax_row / 448 in fp32 (1 for an all-zero row), codes = E4M3(y / s)
+    with the quotient in fp32.  Returns (codes uint8, s float32)."""
     y32 = np.asarray(y, dtype=np.float32)
     amax = np.max(np.abs(y32), axis=-1)
     s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
     codes = e4m3_encode((y32 / s[..., None]).astype(np.float32))
+    return codes, s
+
+
+def fp8_quant_act(y: np.ndarray) -> np.ndarray:
+    """R11 as the linears see it: the rows quantised, returned dequantised in
+    float64, y' = E4M3(y / s) s."""
+    codes, s = fp8_quantize_act(y)
     return e4m3_decode(codes) * s[..., None].astype(np.float64)
 
 

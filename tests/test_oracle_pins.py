@@ -492,3 +492,16 @@ def test_act_fp8_quantises_the_inputs_of_the_four_linears(monkeypatch):
     assert not np.array_equal(a, b)
     c = np.dot(a.ravel(), b.ravel()) / np.linalg.norm(a) / np.linalg.norm(b)
     assert c > 0.99
+
+
+def test_fp8_quantize_act_codes_ties_and_subnormals():
+    """R11 codes: with amax = 448 the scale is exactly 1, so the codes are the
+    E4M3 nearest-even codes of the values themselves: midpoints go to the even
+    code, half the smallest subnormal flushes to zero, the sign bit is bit 7."""
+    row = np.zeros(8, dtype=np.float32)
+    row[:7] = [448.0, 1.0625, 1.1875, 2.0 ** -10, 3 * 2.0 ** -10, -1.0, -448.0]
+    codes, s = O.fp8_quantize_act(row[None])
+    assert s[0] == 1.0
+    assert list(codes[0]) == [0x7E, 0x38, 0x3A, 0x00, 0x02, 0xB8, 0xFE, 0x00]
+    codes, s = O.fp8_quantize_act(np.zeros((2, 16), dtype=np.float32))
+    assert np.all(s == 1.0) and not codes.any()

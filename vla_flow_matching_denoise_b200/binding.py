@@ -21,13 +21,14 @@ LIB_PATH = os.path.join(_PKG, "libfm_expert.so")
 FM_W_BF16 = 0
 FM_W_FP8_E4M3 = 1
 FM_W_FP8_NVFP4_GU = 2
+FM_W_W8A8_E4M3 = 3
 
 STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_NOT_READY", 3: "FM_ERR_OOM",
           4: "FM_ERR_CUDA", 5: "FM_ERR_TIMEOUT", 6: "FM_ERR_UNSUPPORTED"}
 
 # Every symbol include/fm_expert.h declares.
 EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_set_prefix_varlen", "fm_set_prefix_builder",
-           "fm_build_prefix", "fm_get_prefix_kv", "fm_get_nvfp4_weights", "fm_denoise", "fm_velocity", "fm_time_modulation",
+           "fm_build_prefix", "fm_get_prefix_kv", "fm_get_nvfp4_weights", "fm_quantize_act_e4m3", "fm_denoise", "fm_velocity", "fm_time_modulation",
            "fm_trace_bytes", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
            "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
            "fm_expert_destroy", "fm_last_error", "fm_status_string",
@@ -93,6 +94,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_build_prefix.argtypes = [vp, vp, ip, ip, vp]
     lib.fm_get_prefix_kv.argtypes = [vp, ip, ip, vp, vp]
     lib.fm_get_nvfp4_weights.argtypes = [vp, ip, ip, vp, vp, vp]
+    lib.fm_quantize_act_e4m3.argtypes = [vp, vp, ip, ip, vp, vp, vp]
     lib.fm_get_geometry.argtypes = [vp, ctypes.POINTER(ip), ctypes.POINTER(ip), ctypes.POINTER(ip)]
     lib.fm_expert_destroy.argtypes = [vp]
     lib.fm_expert_destroy.restype = sz
@@ -105,7 +107,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
                  "fm_time_modulation", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
                  "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
                  "fm_set_prefix_varlen", "fm_set_prefix_builder", "fm_build_prefix", "fm_get_prefix_kv",
-                 "fm_get_nvfp4_weights"):
+                 "fm_get_nvfp4_weights", "fm_quantize_act_e4m3"):
         getattr(lib, name).restype = ip
     _lib = lib
     return lib
@@ -145,7 +147,8 @@ def make_config(shape: ExpertShape, max_prefix: Optional[int] = None, max_batch:
                     shape.prefix_len if max_prefix is None else max_prefix,
                     shape.batch if max_batch is None else max_batch, max_steps,
                     shape.rms_eps, shape.rope_base,
-                    FM_W_FP8_NVFP4_GU if shape.nvfp4_gu else FM_W_FP8_E4M3 if shape.fp8 else FM_W_BF16)
+                    FM_W_W8A8_E4M3 if shape.w8a8 else FM_W_FP8_NVFP4_GU if shape.nvfp4_gu
+                    else FM_W_FP8_E4M3 if shape.fp8 else FM_W_BF16)
 
 
 class Expert:
@@ -290,6 +293,17 @@ class Expert:
         self._check("fm_get_nvfp4_weights", self.lib.fm_get_nvfp4_weights(self.h, layer, which, _ptr(codes),
                                                                            _ptr(sb), _ptr(g)))
         return codes, sb, np.float32(g[0])
+
+    def quantize_act_e4m3(self, x_bits: np.ndarray, stream=None):
+        """(codes [M, K] uint8, scales [M] fp32) of bf16 rows x_bits [M, K] by
+        the W8A8 path's row-quantiser kernel."""
+        x = np.ascontiguousarray(x_bits, dtype=np.uint16)
+        M, K = x.shape
+        codes = np.empty((M, K), dtype=np.uint8)
+        scales = np.empty(M, dtype=np.float32)
+        self._check("fm_quantize_act_e4m3", self.lib.fm_quantize_act_e4m3(self.h, _ptr(x), M, K, _ptr(codes),
+                                                                           _ptr(scales), _stream(stream)))
+        return codes, scales
 
     def profile(self, batch: int, steps: int, iters: int, stream=None):
         """Mean (time-MLP ms, loop ms) over `iters` event-timed runs."""

@@ -70,7 +70,8 @@ struct fm_expert {
   std::vector<float> nv4_g;          // NVFP4 gate_up: [L][2] tensor scales (gate, up)
   // batched path (B >= 2 requests advance together, M = B * T rows)
   bool batched = false;
-  uint8_t* barena = nullptr;         // per layer: [N/BN][K/64] chunks of each linear
+  bool w8a8 = false;                 // E4M3 weights and per-token E4M3 activations (every B batched)
+  uint8_t* barena = nullptr;         // per layer: [N/BN][K/64] chunks of each linear (W8A8: [N/BN][K/128])
   uint64_t blayer_bytes = 0;
   uint64_t boff[4] = {0, 0, 0, 0};
   int Mp = 0;                        // padded rows of the batched activations
@@ -81,6 +82,15 @@ struct fm_expert {
   float* bh = nullptr;               // [Mp][d] residual
   float* bdelta = nullptr;           // [Mp][d] gated branch of o_proj / down
   uint16_t* bq = nullptr;            // [B_cap][Hkv][q_rows][hd]
+  // W8A8: weight scales by GEMM column, activation codes and their row scales
+  float* bwscale = nullptr;          // [L][bw_stride]: the four linears' columns in tile order
+  int bw_stride = 0;
+  int bw_off[4] = {0, 0, 0, 0};
+  std::vector<PackChunk> bpack_jobs; // tile chunks and their source rows (fm_get_fp8_weights)
+  std::vector<int32_t> bpack_rows;
+  uint8_t* bo8 = nullptr;            // ACT8 [Mp/128][Hq*hd/128]
+  uint8_t* bu8 = nullptr;            // ACT8 [Mp/128][F/128]
+  float* bsa = nullptr;              // [4][Mp]: row scales of z_a, o, z_f, u
   // prefix cache builder (fm_set_prefix_builder / fm_build_prefix)
   int pre_d = 0;                     // backbone hidden width (0: no builder weights)
   uint8_t* pre_arena = nullptr;      // per layer: [Wk; Wv] in [N/BN][d/64] chunks
@@ -290,7 +300,8 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   // quantised weights: E4M3 rows for every linear, or for all but gate_up,
   // whose rows are NVFP4 (64 codes + 4 block scales = 36 bytes)
   const bool nv4 = c.wtype == FM_W_FP8_NVFP4_GU;
-  const bool fp8 = c.wtype == FM_W_FP8_E4M3 || nv4;
+  const bool w8a8 = c.wtype == FM_W_W8A8_E4M3;   // only the batched arena, in E4M3
+  const bool fp8 = c.wtype == FM_W_FP8_E4M3 || nv4 || w8a8;
   auto fmt_of = [&](int g) { return !fp8 ? 0 : (nv4 && g == G_GU) ? 2 : 1; };
   auto row_bytes = [&](int g) -> uint64_t { const int f = fmt_of(g); return f == 0 ? 128 : f == 1 ? 64 : 36; };
   // Per-layer packing jobs (identical for every layer) and CTA spans.
@@ -351,17 +362,20 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   }
   std::vector<float> sc_host(fp8 ? (size_t)c.n_layers * h->sc_stride : 0, 0.f);
   // Batched-path packing: each linear as [N/BN][K/64] chunks of BN rows
-  // (gate_up tile j: gate rows 128 j .. then up rows 128 j ..).
+  // (gate_up tile j: gate rows 128 j .. then up rows 128 j ..); W8A8: E4M3
+  // codes in [N/BN][K/128] chunks, same 128-byte rows.
   std::vector<PackChunk> bjobs;
   std::vector<int32_t> brows;
   if (h->batched) {
     const int Ns[4] = {qn + 2 * kn, d, 2 * F, d};
     const int Ks[4] = {d, qn, d, F};
     const int epi[4] = {BE_QKV, BE_RESID, BE_SWIGLU, BE_RESID};
+    const int kcols = w8a8 ? 128 : 64;
     uint64_t boff = 0;
     for (int g = 0; g < 4; ++g) {
-      const int bn = bgemm_bn(epi[g], Ns[g]), nkb = Ks[g] / 64;
+      const int bn = bgemm_bn(epi[g], Ns[g]), nkb = Ks[g] / kcols;
       h->boff[g] = boff;
+      h->bw_off[g] = (int)brows.size();
       for (int nt = 0; nt < Ns[g] / bn; ++nt) {
         const uint32_t roff = (uint32_t)brows.size();
         for (int q = 0; q < bn; ++q) {
@@ -376,20 +390,28 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
           pc.nrows = (uint16_t)bn;
           pc.mat = (uint8_t)g;
           pc.kb = (uint32_t)kb;
+          pc.fmt = (uint8_t)(w8a8 ? 1 : 0);
           bjobs.push_back(pc);
         }
       }
-      boff += (uint64_t)Ns[g] * Ks[g] * 2;
+      boff += (uint64_t)Ns[g] * Ks[g] * (w8a8 ? 1 : 2);
     }
     h->blayer_bytes = boff;
     DALLOC(h->barena, (size_t)c.n_layers * boff);
+    if (w8a8) {
+      h->bw_stride = (int)brows.size();
+      DALLOC(h->bwscale, (size_t)c.n_layers * h->bw_stride * 4);
+      h->bpack_jobs = bjobs;
+      h->bpack_rows = brows;
+    }
   }
+  std::vector<float> bw_host(w8a8 ? (size_t)c.n_layers * h->bw_stride : 0, 0.f);
 
   PackChunk* d_jobs = nullptr;
   int32_t* d_rows = nullptr;
   uint16_t** d_mats = nullptr;
   int* d_matk = nullptr;
-  DALLOC(h->arena, (size_t)c.n_layers * off);
+  if (!w8a8) DALLOC(h->arena, (size_t)c.n_layers * off);
   DALLOC(h->span_off, span.size() * 4);
   CK(cudaMemcpy(h->span_off, span.data(), span.size() * 4, cudaMemcpyHostToDevice));
   // temporary buffers (freed at the end)
@@ -474,9 +496,12 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
             e = launch_nvfp4_quantize(mats[G_GU] + (size_t)t * F * d, F, d, amax4, q8[G_GU] + (size_t)t * F * d,
                                       sb4 + (size_t)t * F * (d / 16), g4 + t, 0);
         }
-        if (e == cudaSuccess)
+        if (e == cudaSuccess && !w8a8)
           e = launch_pack8(d_jobs, (int)jobs.size(), d_rows, reinterpret_cast<const uint8_t* const*>(d_mats), d_matk,
                            h->arena + (size_t)l * off, 0);
+        if (e == cudaSuccess && w8a8)
+          e = launch_pack8_tile(d_bjobs, (int)bjobs.size(), d_brows, reinterpret_cast<const uint8_t* const*>(d_mats),
+                                d_matk, h->barena + (size_t)l * h->blayer_bytes, 0);
         if (e == cudaSuccess && nv4)
           e = launch_pack_nvfp4(d_jobs, (int)jobs.size(), d_rows, q8[G_GU], sb4, d, h->arena + (size_t)l * off, 0);
         float gh[2] = {1.f, 1.f};
@@ -488,6 +513,16 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
         float* lrs = h->row_scale.data() + (size_t)l * (mrows[0] + mrows[1] + mrows[2] + mrows[3]);
         if (e == cudaSuccess)
           e = cudaMemcpy(lrs, rs[0], (size_t)(mrows[0] + mrows[1] + mrows[2] + mrows[3]) * 4, cudaMemcpyDeviceToHost);
+        if (e == cudaSuccess && w8a8) {
+          // GEMM column i of linear g holds source row brows[i] of that linear
+          int rbase = 0;
+          for (int g = 0; g < 4; ++g) {
+            const int end = g < 3 ? h->bw_off[g + 1] : h->bw_stride;
+            for (int i = h->bw_off[g]; i < end; ++i)
+              bw_host[(size_t)l * h->bw_stride + i] = lrs[rbase + brows[i]];
+            rbase += mrows[g];
+          }
+        }
         if (e == cudaSuccess) {
           const float* src = lrs;
           for (int g = 0; g < 4; ++g) {
@@ -511,6 +546,7 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
     }
     if (st == FM_OK && fp8) {
       e = cudaMemcpy(h->wscale, sc_host.data(), sc_host.size() * 4, cudaMemcpyHostToDevice);
+      if (e == cudaSuccess && w8a8) e = cudaMemcpy(h->bwscale, bw_host.data(), bw_host.size() * 4, cudaMemcpyHostToDevice);
       if (e != cudaSuccess) st = set_err(h, FM_ERR_CUDA, "scale table: %s", cudaGetErrorString(e));
     }
   }
@@ -606,7 +642,8 @@ fm_status check_config(const fm_config* c) {
   if (c->max_steps > kRows) return set_err(h, FM_ERR_INVALID_ARG, "max_steps must be <= %d", kRows);
   if (!(c->rms_eps > 0.f) || !(c->rope_base > 0.f))
     return set_err(h, FM_ERR_INVALID_ARG, "rms_eps and rope_base must be positive");
-  if (c->wtype != FM_W_BF16 && c->wtype != FM_W_FP8_E4M3 && c->wtype != FM_W_FP8_NVFP4_GU)
+  if (c->wtype != FM_W_BF16 && c->wtype != FM_W_FP8_E4M3 && c->wtype != FM_W_FP8_NVFP4_GU &&
+      c->wtype != FM_W_W8A8_E4M3)
     return set_err(h, FM_ERR_INVALID_ARG, "unknown wtype %d", c->wtype);
   return FM_OK;
 }
@@ -755,6 +792,15 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
   g.q_rows = h->q_rows;
   g.err = h->err_word;
   g.spin_budget = 4000000000LL;
+  // W8A8: row scales of the four GEMM inputs; o and u are quantised by a
+  // row pass after the kernels that write them in bf16
+  const size_t Mcap = (size_t)h->Mp;
+  float* sa_za = h->w8a8 ? h->bsa : nullptr;
+  float* sa_o = h->w8a8 ? h->bsa + Mcap : nullptr;
+  float* sa_zf = h->w8a8 ? h->bsa + 2 * Mcap : nullptr;
+  float* sa_u = h->w8a8 ? h->bsa + 3 * Mcap : nullptr;
+  BQuantParams qo{h->bo, h->bo8, sa_o, M, qn};
+  BQuantParams qu{h->bu, h->bu8, sa_u, M, F};
   BAttnParams a{};
   a.qbuf = h->bq;
   a.o_act = h->bo;
@@ -775,12 +821,17 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
     r.s = mrow;
     r.b = mrow + d;
     r.z = h->bz_a;
+    r.zs = sa_za;
     e = launch_binproj(r, st);
     for (int l = 0; l < L && e == cudaSuccess; ++l) {
       const float* lm = mrow + (size_t)6 * l * d;
       const uint8_t* wl = h->barena + (size_t)l * h->blayer_bytes;
+      const float* bws = h->w8a8 ? h->bwscale + (size_t)l * h->bw_stride : nullptr;
+      auto wsc = [&](int gi) { return bws != nullptr ? bws + h->bw_off[gi] : nullptr; };
       // QKV + RoPE -> q, cache rows P .. P + T - 1
       g.A = reinterpret_cast<const uint8_t*>(h->bz_a);
+      g.a_scale = sa_za;
+      g.w_scale = wsc(G_QKV);
       g.W = wl + h->boff[G_QKV];
       g.K = d;
       g.N = qn + 2 * kn;
@@ -790,8 +841,11 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       a.kc = h->kcache + l * lay;
       a.vc = h->vcache + l * lay;
       if (e == cudaSuccess) e = launch_battn(a, st);
+      if (e == cudaSuccess && h->w8a8) e = launch_browquant(qo, st);
       // o_proj + gated residual, then the FFN norm
-      g.A = reinterpret_cast<const uint8_t*>(h->bo);
+      g.A = h->w8a8 ? h->bo8 : reinterpret_cast<const uint8_t*>(h->bo);
+      g.a_scale = sa_o;
+      g.w_scale = wsc(G_O);
       g.W = wl + h->boff[G_O];
       g.K = qn;
       g.N = d;
@@ -800,14 +854,20 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       r.s = lm + 3 * d;
       r.b = lm + 4 * d;
       r.z = h->bz_f;
+      r.zs = sa_zf;
       if (e == cudaSuccess) e = launch_bresnorm(r, st);
       // gate_up + SwiGLU, down + gated residual
       g.A = reinterpret_cast<const uint8_t*>(h->bz_f);
+      g.a_scale = sa_zf;
+      g.w_scale = wsc(G_GU);
       g.W = wl + h->boff[G_GU];
       g.K = d;
       g.N = 2 * F;
       if (e == cudaSuccess) e = launch_bgemm(g, BE_SWIGLU, h->n_sms, st);
-      g.A = reinterpret_cast<const uint8_t*>(h->bu);
+      if (e == cudaSuccess && h->w8a8) e = launch_browquant(qu, st);
+      g.A = h->w8a8 ? h->bu8 : reinterpret_cast<const uint8_t*>(h->bu);
+      g.a_scale = sa_u;
+      g.w_scale = wsc(G_DOWN);
       g.W = wl + h->boff[G_DOWN];
       g.K = F;
       g.N = d;
@@ -818,6 +878,7 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       r.s = lm + 6 * d;
       r.b = lm + 7 * d;
       r.z = l + 1 < L ? h->bz_a : nullptr;
+      r.zs = sa_za;
       if (e == cudaSuccess) e = launch_bresnorm(r, st);
     }
     r.s = mrow + (size_t)6 * L * d;
@@ -827,9 +888,13 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
   return e;
 }
 
+// Whether `batch` requests run on the batched path: B >= 2 on a handle that
+// has it, every B on a W8A8 handle.
+bool use_batched(const fm_expert* h, int batch) { return h->batched && (batch >= 2 || h->w8a8); }
+
 // Enqueues one full denoise of `batch` requests (x already in h->x).
 cudaError_t enqueue_denoise(fm_expert* h, int batch, int steps, cudaStream_t st) {
-  if (batch >= 2 && h->batched) {
+  if (use_batched(h, batch)) {
     cudaError_t e = launch_time(time_params(h, steps), h->n_sms, st);
     if (e != cudaSuccess) return e;
     return enqueue_batched(h, batch, 0, steps, steps, true, st);
@@ -944,9 +1009,17 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
     // the batched path needs whole 128-column weight tiles, the in-proj's
     // 256-column thread mapping and at most 1024 residual columns
     const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
-    h->batched = c.wtype == FM_W_BF16 && c.max_batch >= 2 && c.d_model % 256 == 0 && c.d_model <= 1024 &&
-                 c.d_ff % 128 == 0 && qkv % 128 == 0 && (c.n_q_heads * c.head_dim) % 64 == 0 &&
-                 (c.head_dim == 64 || c.head_dim == 128);
+    const bool shape_ok = c.d_model % 256 == 0 && c.d_model <= 1024 && c.d_ff % 128 == 0 && qkv % 128 == 0 &&
+                          (c.n_q_heads * c.head_dim) % 64 == 0 && (c.head_dim == 64 || c.head_dim == 128);
+    h->w8a8 = c.wtype == FM_W_W8A8_E4M3;
+    h->batched = shape_ok && ((c.wtype == FM_W_BF16 && c.max_batch >= 2) || h->w8a8);
+    // W8A8 additionally quantises o and u per row (K a multiple of 256, at
+    // most 4096) and runs every batch size on the batched path
+    const int qn = c.n_q_heads * c.head_dim;
+    if (h->w8a8 && !(shape_ok && qn % 256 == 0 && qn <= 4096 && c.d_ff % 256 == 0 && c.d_ff <= 4096)) {
+      set_err(h, FM_ERR_UNSUPPORTED, "W8A8 needs the batched path's shapes (d %% 256, H_q*hd and d_ff %% 256, <= 4096)");
+      return bail(FM_ERR_UNSUPPORTED);
+    }
   }
   if ((st = pack_weights(h, w)) != FM_OK) return bail(st);
 
@@ -987,6 +1060,11 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
     ALLOC_OR_BAIL(h->bh, Mp * d * 4);
     ALLOC_OR_BAIL(h->bdelta, Mp * d * 4);
     ALLOC_OR_BAIL(h->bq, B * c.n_kv_heads * h->q_rows * c.head_dim * 2);
+    if (h->w8a8) {
+      ALLOC_OR_BAIL(h->bo8, Mp * c.n_q_heads * c.head_dim);
+      ALLOC_OR_BAIL(h->bu8, Mp * c.d_ff);
+      ALLOC_OR_BAIL(h->bsa, 4 * Mp * 4);
+    }
   }
 #undef ALLOC_OR_BAIL
   if (cudaDeviceSynchronize() != cudaSuccess) {
@@ -1171,7 +1249,7 @@ fm_status fm_velocity(fm_expert* h, const float* x, int batch, int step_index, i
   if (s != FM_OK) return s;
   const fm_config& c = h->cfg;
   const size_t xs = (size_t)c.chunk_len * c.action_dim;
-  if (batch >= 2 && h->batched) {
+  if (use_batched(h, batch)) {
     CK(enqueue_batched(h, batch, step_index, step_index + 1, steps, false, st));
   } else {
     for (int b = 0; b < batch; ++b) {
@@ -1225,6 +1303,7 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
                             void* stream) {
   if (!h) return FM_ERR_INVALID_ARG;
   if (!trace) return set_err(h, FM_ERR_INVALID_ARG, "trace is NULL");
+  if (h->w8a8) return set_err(h, FM_ERR_UNSUPPORTED, "a W8A8 handle has no one-request kernel to trace");
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   fm_status s = velocity_common(h, x, 1, step_index, steps, st);
   if (s != FM_OK) return s;
@@ -1461,6 +1540,26 @@ fm_status fm_get_fp8_weights(fm_expert* h, int layer, int which, uint8_t* codes,
   const int mrows[4] = {qn + 2 * kn, d, 2 * F, d};
   const int r0 = r0s[which], R = nrows[which], K = kdim[g];
   CK(cudaSetDevice(h->device));
+  size_t base = (size_t)layer * (mrows[0] + mrows[1] + mrows[2] + mrows[3]);
+  for (int i = 0; i < g; ++i) base += mrows[i];
+  if (h->w8a8) {
+    // tile arena: chunk rows of 128 codes, 16-byte pieces swizzled by (row & 7)
+    std::vector<uint8_t> lay(h->blayer_bytes);
+    CK(cudaMemcpy(lay.data(), h->barena + (size_t)layer * h->blayer_bytes, h->blayer_bytes, cudaMemcpyDeviceToHost));
+    std::memset(codes, 0, (size_t)R * K);
+    for (const PackChunk& pc : h->bpack_jobs) {
+      if (pc.mat != g) continue;
+      for (int q = 0; q < pc.nrows; ++q) {
+        const int sr = h->bpack_rows[pc.rowidx_off + q];
+        if (sr < r0 || sr >= r0 + R) continue;
+        for (int j = 0; j < 8; ++j)
+          std::memcpy(codes + (size_t)(sr - r0) * K + (size_t)pc.kb * 128 + j * 16,
+                      lay.data() + pc.dst_off + (size_t)q * 128 + ((j ^ (q & 7)) << 4), 16);
+      }
+    }
+    std::memcpy(scale, h->row_scale.data() + base + r0, (size_t)R * 4);
+    return FM_OK;
+  }
   std::vector<uint8_t> lay(h->layer_bytes);
   CK(cudaMemcpy(lay.data(), h->arena + (size_t)layer * h->layer_bytes, h->layer_bytes, cudaMemcpyDeviceToHost));
   std::memset(codes, 0, (size_t)R * K);
@@ -1472,9 +1571,43 @@ fm_status fm_get_fp8_weights(fm_expert* h, int layer, int which, uint8_t* codes,
       std::memcpy(codes + (size_t)(sr - r0) * K + (size_t)pc.kb * 64, lay.data() + pc.dst_off + (size_t)q * 64, 64);
     }
   }
-  size_t base = (size_t)layer * (mrows[0] + mrows[1] + mrows[2] + mrows[3]);
-  for (int i = 0; i < g; ++i) base += mrows[i];
   std::memcpy(scale, h->row_scale.data() + base + r0, (size_t)R * 4);
+  return FM_OK;
+}
+
+fm_status fm_quantize_act_e4m3(fm_expert* h, const uint16_t* x, int M, int K, uint8_t* codes, float* scales,
+                               void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  if (!x || !codes || !scales || M < 1 || K < 256 || K % 256 != 0 || K > 4096)
+    return set_err(h, FM_ERR_INVALID_ARG, "M %d / K %d invalid or NULL buffer", M, K);
+  CK(cudaSetDevice(h->device));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int Mp = (M + kBM - 1) / kBM * kBM;
+  uint16_t* rows = nullptr;
+  uint16_t* act = nullptr;
+  uint8_t* q = nullptr;
+  float* sc = nullptr;
+  std::vector<uint8_t> hq((size_t)Mp * K);
+  cudaError_t e = cudaMalloc(&rows, (size_t)M * K * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&act, (size_t)Mp * K * 2);
+  if (e == cudaSuccess) e = cudaMalloc(&q, (size_t)Mp * K);
+  if (e == cudaSuccess) e = cudaMalloc(&sc, (size_t)Mp * 4);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(rows, x, (size_t)M * K * 2, cudaMemcpyDefault, st);
+  if (e == cudaSuccess) e = launch_rows_to_act128(rows, M, Mp, K, act, st);
+  if (e == cudaSuccess) e = launch_browquant(BQuantParams{act, q, sc, M, K}, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(hq.data(), q, hq.size(), cudaMemcpyDeviceToHost, st);
+  if (e == cudaSuccess) e = cudaMemcpyAsync(scales, sc, (size_t)M * 4, cudaMemcpyDefault, st);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(st);
+  for (void* p : {static_cast<void*>(rows), static_cast<void*>(act), static_cast<void*>(q), static_cast<void*>(sc)})
+    if (p) cudaFree(p);
+  if (e != cudaSuccess) return set_err(h, FM_ERR_CUDA, "quantize: %s", cudaGetErrorString(e));
+  // ACT8: blocks of 128 rows x 128 codes, 16-byte pieces swizzled by (m & 7)
+  for (int m = 0; m < M; ++m)
+    for (int c = 0; c < K; c += 16)
+      std::memcpy(codes + (size_t)m * K + c,
+                  hq.data() + ((size_t)(m >> 7) * (K >> 7) + (c >> 7)) * (kBM * 128) + (size_t)(m & 127) * 128 +
+                      ((((c & 127) >> 4) ^ (m & 7)) << 4),
+                  16);
   return FM_OK;
 }
 
@@ -1530,8 +1663,8 @@ fm_status fm_profile_denoise(fm_expert* h, int batch, int steps, int iters, floa
     cudaError_t e = cudaEventRecord(ev[0], st);
     if (e == cudaSuccess) e = launch_time(time_params(h, steps), h->n_sms, st);
     if (e == cudaSuccess) e = cudaEventRecord(ev[1], st);
-    if (e == cudaSuccess && batch >= 2 && h->batched) e = enqueue_batched(h, batch, 0, steps, steps, true, st);
-    for (int b = 0; b < batch && e == cudaSuccess && !(batch >= 2 && h->batched); ++b) {
+    if (e == cudaSuccess && use_batched(h, batch)) e = enqueue_batched(h, batch, 0, steps, steps, true, st);
+    for (int b = 0; b < batch && e == cudaSuccess && !use_batched(h, batch); ++b) {
       StepParams p = base_params(h);
       p.b = b;
       p.x = h->x + b * xs;
@@ -1561,6 +1694,7 @@ fm_status fm_profile_phases(fm_expert* h, int steps, uint64_t* out, size_t* n, v
   if (!h) return FM_ERR_INVALID_ARG;
   const fm_config& c = h->cfg;
   if (!n) return set_err(h, FM_ERR_INVALID_ARG, "n is NULL");
+  if (h->w8a8) return set_err(h, FM_ERR_UNSUPPORTED, "a W8A8 handle has no one-request kernel to profile");
   if (steps < 1 || steps > c.max_steps) return set_err(h, FM_ERR_INVALID_ARG, "steps %d invalid", steps);
   const int n_phases = steps * (2 + 5 * c.n_layers), n_gemms = steps * 4 * c.n_layers;
   int per_layer = 0;

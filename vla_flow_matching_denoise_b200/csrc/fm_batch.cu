@@ -18,7 +18,15 @@
 // fused epilogue (RoPE + cache scatter, gated residual, or SwiGLU), so the
 // epilogue of tile i overlaps the main loop of tile i + 1.  Tiles are ordered
 // m-fastest, so the CTAs in flight share each weight chunk through L2.
+//
+// W8A8 variant: the same kernels with E4M3 operands.  The inputs of the four
+// per-layer linears are quantised per token (s = amax_row / 448): the norm
+// kernels emit the codes of z directly, a row-quantiser pass follows attention
+// (o) and the gate_up GEMM (u).  The GEMM streams 128-byte rows of codes
+// (K = 128 per k-block), issues tcgen05.mma kind::f8f6f4 (K = 32 each), and
+// the epilogue scales D by s_a[m] s_w[n] before the fused work.
 #include <cuda_bf16.h>
+#include <cuda_fp8.h>
 #include <cstddef>
 #include <cstdint>
 #include <utility>
@@ -55,7 +63,35 @@ __device__ __forceinline__ size_t act128_off(int m, int c, int K) {
          ((((c & 63) >> 3) ^ (m & 7)) << 3) + (c & 7);
 }
 
+// Byte offset of (row m, column c) in an ACT8 matrix (E4M3 codes) with K
+// columns: blocks of 128 rows x 128 codes, 16-byte pieces swizzled by (m & 7).
+__device__ __forceinline__ size_t act8_off(int m, int c, int K) {
+  return ((size_t)(m >> 7) * (K >> 7) + (c >> 7)) * (kBM * 128) + (size_t)(m & 127) * 128 +
+         ((((c & 127) >> 4) ^ (m & 7)) << 4) + (c & 15);
+}
+
 __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
+// R11 per-token scale of a row with largest magnitude `amax` (1 for a zero row).
+__device__ __forceinline__ float act_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f; }
+
+// E4M3 code of y / s (true division, nearest-even, saturating finite).
+__device__ __forceinline__ uint32_t e4m3_of(float y, float s) {
+  return (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(y, s), __NV_SATFINITE, __NV_E4M3);
+}
+
+// Multiplies v[0..15] by sa * sw[n0 .. n0 + 15] (E4M3 GEMM dequantisation).
+__device__ __forceinline__ void dequant16(float (&v)[16], float sa, const float* sw) {
+  const float4* w4 = reinterpret_cast<const float4*>(sw);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const float4 w = w4[q];
+    v[4 * q] *= sa * w.x;
+    v[4 * q + 1] *= sa * w.y;
+    v[4 * q + 2] *= sa * w.z;
+    v[4 * q + 3] *= sa * w.w;
+  }
+}
 
 // ------------------------------------------------------------------ epilogues
 // Thread = one accumulator row (TMEM lane); `ta` is the TMEM address of column
@@ -63,8 +99,9 @@ __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __e
 
 // Gated residual branch: delta[m][n] = gate[n] * D[m][n] (fp32, stores only;
 // the row kernel that follows adds it to h and normalises).
-template <int BN>
+template <int BN, bool F8>
 __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt) {
+  const float sa = (F8 && valid) ? p.a_scale[m] : 1.f;
 #pragma unroll 1
   for (int cb = 0; cb < BN / 16; ++cb) {
     float v[16];
@@ -72,6 +109,7 @@ __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int
     tmem_ld_wait();
     if (!valid) continue;
     const int n0 = nt * BN + cb * 16;
+    if (F8) dequant16(v, sa, p.w_scale + n0);
     float4* dp = reinterpret_cast<float4*>(p.h + (size_t)m * p.N + n0);
     const float4* gp = reinterpret_cast<const float4*>(p.gate + n0);
 #pragma unroll
@@ -82,9 +120,10 @@ __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int
   }
 }
 
-template <int BN>
+template <int BN, bool F8>
 __device__ __forceinline__ void epi_swiglu(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt) {
   constexpr int HALF = BN / 2;
+  const float sa = (F8 && valid) ? p.a_scale[m] : 1.f;
 #pragma unroll 1
   for (int j = 0; j < HALF / 16; ++j) {
     float g[16], u[16];
@@ -92,6 +131,10 @@ __device__ __forceinline__ void epi_swiglu(const BGemmParams& p, uint32_t ta, in
     tmem_ld16(ta + HALF + j * 16, u);
     tmem_ld_wait();
     if (!valid) continue;
+    if (F8) {
+      dequant16(g, sa, p.w_scale + nt * BN + j * 16);
+      dequant16(u, sa, p.w_scale + nt * BN + HALF + j * 16);
+    }
     const int uc = nt * HALF + j * 16;
     uint32_t pk[8];
 #pragma unroll
@@ -112,8 +155,9 @@ __device__ __forceinline__ void store_row16(uint16_t* rowp, int row, int e0, con
   *reinterpret_cast<uint4*>(rowp + (((pc + 1) ^ (row & 7)) << 3)) = make_uint4(pk[4], pk[5], pk[6], pk[7]);
 }
 
-template <int BN>
+template <int BN, bool F8>
 __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt) {
+  const float sa = (F8 && valid) ? p.a_scale[m] : 1.f;
   const int hd = p.hd, half = hd / 2;
   const int qn = p.Hq * hd, kn = p.Hkv * hd, G = p.Hq / p.Hkv;
   const int b = valid ? m / p.T : 0, t = valid ? m % p.T : 0;
@@ -142,6 +186,10 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
         tmem_ld16(ta + ho + half + c, hi);
         tmem_ld_wait();
         if (!valid) continue;
+        if (F8) {
+          dequant16(lo, sa, p.w_scale + col0 + c);
+          dequant16(hi, sa, p.w_scale + col0 + half + c);
+        }
         float ol[16], oh[16];
         const float4* r4 = reinterpret_cast<const float4*>(rope + c);   // (cos, sin) pairs, 128 B
 #pragma unroll
@@ -161,14 +209,16 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
         float v[16];
         tmem_ld16(ta + ho + c, v);
         tmem_ld_wait();
-        if (valid) store_row16(rowp, row, c, v);
+        if (!valid) continue;
+        if (F8) dequant16(v, sa, p.w_scale + col0 + c);
+        store_row16(rowp, row, c, v);
       }
     }
   }
 }
 
 // ------------------------------------------------------------------ GEMM
-template <int BN, int EPI>
+template <int BN, int EPI, bool F8>
 __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constant__ BGemmParams p) {
   using C = BCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
@@ -182,7 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int nkb = p.K / 64;
+  const int nkb = F8 ? p.K / 128 : p.K / 64;   // k-blocks of 128-byte rows
   const int MT = p.Mp / kBM, NT = p.N / BN;
   const int ntiles = MT * NT;   // m-tile fastest
   const long long budget = p.spin_budget;
@@ -255,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
     }
   } else if (warp == 1) {
     if (lane == 0) {
-      const uint32_t idesc = idesc_bf16(kBM, BN);
+      const uint32_t idesc = F8 ? idesc_e4m3(kBM, BN) : idesc_bf16(kBM, BN);
       uint32_t it = 0, local = 0;
       bool ok = true;
       for (int tile = blockIdx.x; ok && tile < ntiles; tile += gridDim.x, ++local) {
@@ -277,10 +327,16 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
           tc_fence_after();
           const uint32_t a_base = smem_u32(ring + (size_t)s * C::kStage);
           const uint32_t b_base = a_base + C::kA;
+          // four MMAs per 128-byte row: K = 16 bf16 or K = 32 E4M3 each
 #pragma unroll
-          for (int k16 = 0; k16 < 4; ++k16)
-            mma_bf16(d_tmem, desc_sw128(a_base + k16 * 32), desc_sw128(b_base + k16 * 32), idesc,
-                     (kb | k16) != 0);
+          for (int k16 = 0; k16 < 4; ++k16) {
+            if (F8)
+              mma_e4m3(d_tmem, desc_sw128(a_base + k16 * 32), desc_sw128(b_base + k16 * 32), idesc,
+                       (kb | k16) != 0);
+            else
+              mma_bf16(d_tmem, desc_sw128(a_base + k16 * 32), desc_sw128(b_base + k16 * 32), idesc,
+                       (kb | k16) != 0);
+          }
           mma_commit(smem_u32(&empty[s]));
         }
         if (ok) mma_commit(smem_u32(&tfull[acc]));
@@ -305,9 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
       const int m = mt * kBM + row;
       const bool valid = m < p.M;
       const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + acc * BN;
-      if (EPI == BE_RESID) epi_resid<BN>(p, ta, m, valid, nt);
-      else if (EPI == BE_SWIGLU) epi_swiglu<BN>(p, ta, m, valid, nt);
-      else epi_qkv<BN>(p, ta, m, valid, nt);
+      if (EPI == BE_RESID) epi_resid<BN, F8>(p, ta, m, valid, nt);
+      else if (EPI == BE_SWIGLU) epi_swiglu<BN, F8>(p, ta, m, valid, nt);
+      else epi_qkv<BN, F8>(p, ta, m, valid, nt);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
@@ -325,11 +381,14 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
 // In-proj + AdaRMSNorm of layer 0: 16 rows per CTA (256 threads); thread t
 // computes columns t + 256 j of h = x W_in^T for the 16 rows, then the rows'
 // rstd (block reduction) and z = bf16(h rstd (1 + s) + b).
+// F8: z as E4M3 codes with per-row scales (p.zs).
 constexpr int kRowsIn = 16;
+template <bool F8>
 __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BRowParams p) {
   __shared__ float xs[kRowsIn][128];
   __shared__ float red[8][kRowsIn];
   __shared__ float rstd[kRowsIn];
+  __shared__ float scl[kRowsIn];
   grid_dep_launch();
   grid_dep_wait();
   const int m0 = blockIdx.x * kRowsIn;
@@ -379,6 +438,28 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
     rstd[tid] = 1.0f / sqrtf(s / (float)d + p.eps);
   }
   __syncthreads();
+  if constexpr (!F8) {
+#pragma unroll
+    for (int j = 0; j < kMaxJ; ++j) {
+      if (j >= nj) break;
+      const int n = tid + 256 * j;
+      const float sc = 1.0f + p.s[n], sh = p.b[n];
+#pragma unroll
+      for (int r = 0; r < kRowsIn; ++r) {
+        const int m = m0 + r;
+        if (m >= p.M) break;
+        p.h[(size_t)m * d + n] = acc[j][r];
+        const __nv_bfloat16 zb = __float2bfloat16_rn(fmaf(acc[j][r] * rstd[r], sc, sh));
+        p.z[act128_off(m, n, d)] = *reinterpret_cast<const uint16_t*>(&zb);
+      }
+    }
+    return;
+  }
+  // E4M3 z: y = h rstd (1 + s) + b in fp32, the row's amax (block reduction),
+  // then the codes of y / s_row
+  float am[kRowsIn];
+#pragma unroll
+  for (int r = 0; r < kRowsIn; ++r) am[r] = 0.f;
 #pragma unroll
   for (int j = 0; j < kMaxJ; ++j) {
     if (j >= nj) break;
@@ -387,10 +468,38 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
 #pragma unroll
     for (int r = 0; r < kRowsIn; ++r) {
       const int m = m0 + r;
+      if (m < p.M) p.h[(size_t)m * d + n] = acc[j][r];
+      acc[j][r] = fmaf(acc[j][r] * rstd[r], sc, sh);
+      am[r] = fmaxf(am[r], fabsf(acc[j][r]));
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kRowsIn; ++r) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) am[r] = fmaxf(am[r], __shfl_xor_sync(0xffffffffu, am[r], o));
+  }
+  if ((tid & 31) == 0)
+#pragma unroll
+    for (int r = 0; r < kRowsIn; ++r) red[tid >> 5][r] = am[r];
+  __syncthreads();
+  if (tid < kRowsIn) {
+    float a = 0.f;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w][tid]);
+    scl[tid] = act_scale(a);
+    if (m0 + tid < p.M) p.zs[m0 + tid] = scl[tid];
+  }
+  __syncthreads();
+  uint8_t* z8 = reinterpret_cast<uint8_t*>(p.z);
+#pragma unroll
+  for (int j = 0; j < kMaxJ; ++j) {
+    if (j >= nj) break;
+    const int n = tid + 256 * j;
+#pragma unroll
+    for (int r = 0; r < kRowsIn; ++r) {
+      const int m = m0 + r;
       if (m >= p.M) break;
-      p.h[(size_t)m * d + n] = acc[j][r];
-      const __nv_bfloat16 zb = __float2bfloat16_rn(fmaf(acc[j][r] * rstd[r], sc, sh));
-      p.z[act128_off(m, n, d)] = *reinterpret_cast<const uint16_t*>(&zb);
+      z8[act8_off(m, n, d)] = (uint8_t)e4m3_of(acc[j][r], scl[r]);
     }
   }
 }
@@ -420,15 +529,84 @@ __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ B
 #pragma unroll
   for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
   const float rs = 1.0f / sqrtf(s / (float)d + p.eps);
+  if (p.zs == nullptr) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i >= n4) break;
+      const int c = 4 * (lane + 32 * i);
+      const float4 sc = *reinterpret_cast<const float4*>(p.s + c);
+      const float4 sh = *reinterpret_cast<const float4*>(p.b + c);
+      const uint32_t lo = pack2_bf16(fmaf(v[i].x * rs, 1.0f + sc.x, sh.x), fmaf(v[i].y * rs, 1.0f + sc.y, sh.y));
+      const uint32_t hi = pack2_bf16(fmaf(v[i].z * rs, 1.0f + sc.z, sh.z), fmaf(v[i].w * rs, 1.0f + sc.w, sh.w));
+      *reinterpret_cast<uint2*>(p.z + act128_off(m, c, d)) = make_uint2(lo, hi);
+    }
+    return;
+  }
+  // E4M3 z: y in fp32, the row's amax across the warp, codes of y / s_row
+  float am = 0.f;
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     if (i >= n4) break;
     const int c = 4 * (lane + 32 * i);
     const float4 sc = *reinterpret_cast<const float4*>(p.s + c);
     const float4 sh = *reinterpret_cast<const float4*>(p.b + c);
-    const uint32_t lo = pack2_bf16(fmaf(v[i].x * rs, 1.0f + sc.x, sh.x), fmaf(v[i].y * rs, 1.0f + sc.y, sh.y));
-    const uint32_t hi = pack2_bf16(fmaf(v[i].z * rs, 1.0f + sc.z, sh.z), fmaf(v[i].w * rs, 1.0f + sc.w, sh.w));
-    *reinterpret_cast<uint2*>(p.z + act128_off(m, c, d)) = make_uint2(lo, hi);
+    v[i] = make_float4(fmaf(v[i].x * rs, 1.0f + sc.x, sh.x), fmaf(v[i].y * rs, 1.0f + sc.y, sh.y),
+                       fmaf(v[i].z * rs, 1.0f + sc.z, sh.z), fmaf(v[i].w * rs, 1.0f + sc.w, sh.w));
+    am = fmaxf(am, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const float sq = act_scale(am);
+  if (lane == 0) p.zs[m] = sq;
+  uint8_t* z8 = reinterpret_cast<uint8_t*>(p.z);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (i >= n4) break;
+    const int c = 4 * (lane + 32 * i);
+    const uint32_t w = e4m3_of(v[i].x, sq) | (e4m3_of(v[i].y, sq) << 8) | (e4m3_of(v[i].z, sq) << 16) |
+                       (e4m3_of(v[i].w, sq) << 24);
+    *reinterpret_cast<uint32_t*>(z8 + act8_off(m, c, d)) = w;
+  }
+}
+
+// R11 per-token E4M3 of a bf16 ACT128 matrix (attention output o, SwiGLU
+// output u): one warp per row; lane i holds pieces of 8 values at columns
+// 8 (i + 32 j), K a multiple of 256 and at most 4096.
+constexpr int kQuantPieces = 16;
+__global__ void __launch_bounds__(256) browquant_kernel(const __grid_constant__ BQuantParams p) {
+  grid_dep_launch();
+  grid_dep_wait();
+  const int m = blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (m >= p.M) return;
+  const int np = p.K / 256;
+  uint4 raw[kQuantPieces];
+  float am = 0.f;
+#pragma unroll
+  for (int i = 0; i < kQuantPieces; ++i) {
+    if (i >= np) break;
+    raw[i] = *reinterpret_cast<const uint4*>(p.src + act128_off(m, 8 * (lane + 32 * i), p.K));
+    const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q)
+      am = fmaxf(am, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
+  const float sq = act_scale(am);
+  if (lane == 0) p.scale[m] = sq;
+#pragma unroll
+  for (int i = 0; i < kQuantPieces; ++i) {
+    if (i >= np) break;
+    const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+    uint32_t out[2] = {0u, 0u};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const uint32_t lo = e4m3_of(__uint_as_float(w[q] << 16), sq);
+      const uint32_t hi = e4m3_of(__uint_as_float(w[q] & 0xFFFF0000u), sq);
+      out[q >> 1] |= (lo | (hi << 8)) << (16 * (q & 1));
+    }
+    *reinterpret_cast<uint2*>(p.dst + act8_off(m, 8 * (lane + 32 * i), p.K)) = make_uint2(out[0], out[1]);
   }
 }
 
@@ -704,15 +882,23 @@ cudaError_t launch_pdl(void (*kernel)(Params...), int grid, int block, size_t sm
   return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
 }
 
-template <int BN, int EPI>
+template <int BN, int EPI, bool F8>
 cudaError_t launch_bgemm_t(const BGemmParams& p, int n_sms, cudaStream_t st) {
   using C = BCfg<BN>;
-  cudaError_t e = cudaFuncSetAttribute(bgemm_kernel<BN, EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(bgemm_kernel<BN, EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::kSmem);
   if (e != cudaSuccess) return e;
   const int ntiles = (p.Mp / kBM) * (p.N / BN);
   const int grid = ntiles < n_sms ? ntiles : n_sms;
-  return launch_pdl(bgemm_kernel<BN, EPI>, grid, kThreads, C::kSmem, st, p);
+  return launch_pdl(bgemm_kernel<BN, EPI, F8>, grid, kThreads, C::kSmem, st, p);
+}
+
+template <bool F8>
+cudaError_t launch_bgemm_f(const BGemmParams& p, int epi, int bn, int n_sms, cudaStream_t st) {
+  if (epi == BE_RESID)
+    return bn == 256 ? launch_bgemm_t<256, BE_RESID, F8>(p, n_sms, st) : launch_bgemm_t<128, BE_RESID, F8>(p, n_sms, st);
+  if (epi == BE_SWIGLU) return launch_bgemm_t<256, BE_SWIGLU, F8>(p, n_sms, st);
+  return bn == 256 ? launch_bgemm_t<256, BE_QKV, F8>(p, n_sms, st) : launch_bgemm_t<128, BE_QKV, F8>(p, n_sms, st);
 }
 
 }  // namespace
@@ -725,12 +911,11 @@ int bgemm_bn(int epi, int N) {
   return N % 256 == 0 ? 256 : 128;
 }
 
+// E4M3 operands when p.a_scale is set (W8A8), bf16 otherwise.
 cudaError_t launch_bgemm(const BGemmParams& p, int epi, int n_sms, cudaStream_t st) {
   const int bn = bgemm_bn(epi, p.N);
-  if (epi == BE_RESID)
-    return bn == 256 ? launch_bgemm_t<256, BE_RESID>(p, n_sms, st) : launch_bgemm_t<128, BE_RESID>(p, n_sms, st);
-  if (epi == BE_SWIGLU) return launch_bgemm_t<256, BE_SWIGLU>(p, n_sms, st);
-  return bn == 256 ? launch_bgemm_t<256, BE_QKV>(p, n_sms, st) : launch_bgemm_t<128, BE_QKV>(p, n_sms, st);
+  return p.a_scale != nullptr ? launch_bgemm_f<true>(p, epi, bn, n_sms, st)
+                              : launch_bgemm_f<false>(p, epi, bn, n_sms, st);
 }
 
 // Row-major bf16 [M][K] -> ACT128 [Mp/128][K/64]; rows M .. Mp-1 are zero.
@@ -751,11 +936,17 @@ cudaError_t launch_rows_to_act128(const uint16_t* src, int M, int Mp, int K, uin
 }
 
 cudaError_t launch_binproj(const BRowParams& p, cudaStream_t st) {
-  return launch_pdl(binproj_kernel, (p.M + kRowsIn - 1) / kRowsIn, 256, 0, st, p);
+  const int grid = (p.M + kRowsIn - 1) / kRowsIn;
+  return p.zs != nullptr ? launch_pdl(binproj_kernel<true>, grid, 256, 0, st, p)
+                         : launch_pdl(binproj_kernel<false>, grid, 256, 0, st, p);
 }
 
 cudaError_t launch_bresnorm(const BRowParams& p, cudaStream_t st) {
   return launch_pdl(bresnorm_kernel, (p.M + 7) / 8, 256, 0, st, p);
+}
+
+cudaError_t launch_browquant(const BQuantParams& p, cudaStream_t st) {
+  return launch_pdl(browquant_kernel, (p.M + 7) / 8, 256, 0, st, p);
 }
 
 cudaError_t launch_boutproj(const BRowParams& p, cudaStream_t st) {

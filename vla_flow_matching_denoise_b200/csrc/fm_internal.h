@@ -132,9 +132,14 @@ constexpr int kBRing = 192 * 1024;     // batched GEMM operand ring
 enum BEpi { BE_QKV = 0, BE_RESID = 1, BE_SWIGLU = 2 };
 
 struct BGemmParams {
-  const uint8_t* A;          // ACT128 [Mp/128][K/64]
-  const uint8_t* W;          // packed [N/BN][K/64] chunks of BN x 64
+  // bf16 operands: A is ACT128 [Mp/128][K/64], W packed [N/BN][K/64] chunks of
+  // BN x 64.  E4M3 operands (the W8A8 variant): A is ACT8 [Mp/128][K/128], W
+  // [N/BN][K/128] chunks of BN x 128 codes; both 128-byte rows, same swizzle.
+  const uint8_t* A;
+  const uint8_t* W;
   int K, N, M, Mp;           // reduction, output channels, valid rows (B*T), padded rows
+  const float* a_scale;      // E4M3 only: [Mp] row scale of A (per token)
+  const float* w_scale;      // E4M3 only: [N] scale of the weight row behind each GEMM column
   // BE_RESID: h[m][n] = gate[n] * D[m][n]   (fp32 residual branch, row stride N)
   float* h;
   const float* gate;
@@ -169,7 +174,16 @@ struct BRowParams {          // in-proj, AdaRMSNorm, out-proj + Euler (row kerne
   const float* delta;        // [Mp][d] fp32 gated branch added to h (residual + norm kernel)
   const float* s;            // norm scale and shift [d]
   const float* b;
-  uint16_t* z;               // ACT128 [Mp/128][d/64]
+  uint16_t* z;               // ACT128 [Mp/128][d/64] (bf16), or ACT8 codes when zs is set
+  float* zs;                 // non-null: z gets E4M3 codes [Mp/128][d/128] and zs[m] their row scale
+};
+
+// Per-token E4M3 of a bf16 ACT128 matrix [M][K] into ACT8 codes and row scales.
+struct BQuantParams {
+  const uint16_t* src;       // ACT128 [Mp/128][K/64]
+  uint8_t* dst;              // ACT8 [Mp/128][K/128]
+  float* scale;              // [Mp]
+  int M, K;
 };
 
 struct BAttnParams {

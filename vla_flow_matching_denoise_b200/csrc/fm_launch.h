@@ -13,6 +13,8 @@ cudaError_t launch_pack(const PackChunk* chunks, int nchunks, const int32_t* row
                         cudaStream_t st);
 cudaError_t launch_pack8(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
                          const uint8_t* const* mats, const int* mat_k, uint8_t* dst, cudaStream_t st);
+cudaError_t launch_pack8_tile(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
+                              const uint8_t* const* mats, const int* mat_k, uint8_t* dst, cudaStream_t st);
 cudaError_t launch_nvfp4_quantize(const uint16_t* w, int rows, int K, unsigned int* amax_scratch, uint8_t* codes,
                                   uint8_t* sb, float* g, cudaStream_t st);
 cudaError_t launch_pack_nvfp4(const PackChunk* chunks, int nchunks, const int32_t* rowidx, const uint8_t* codes,
@@ -37,6 +39,7 @@ cudaError_t launch_bgemm(const BGemmParams& p, int epi, int n_sms, cudaStream_t 
 cudaError_t launch_binproj(const BRowParams& p, cudaStream_t st);
 cudaError_t launch_rows_to_act128(const uint16_t* src, int M, int Mp, int K, uint16_t* dst, cudaStream_t st);
 cudaError_t launch_bresnorm(const BRowParams& p, cudaStream_t st);
+cudaError_t launch_browquant(const BQuantParams& p, cudaStream_t st);
 cudaError_t launch_boutproj(const BRowParams& p, cudaStream_t st);
 cudaError_t launch_battn(const BAttnParams& p, cudaStream_t st);
 

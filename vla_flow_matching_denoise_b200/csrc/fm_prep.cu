@@ -49,6 +49,25 @@ __global__ void pack8_kernel(const PackChunk* __restrict__ chunks, const int32_t
   }
 }
 
+// Copies 16-byte pieces of E4M3 code rows into a tensor-core tile chunk of
+// R rows x 128 codes (column block ch.kb of 128), pieces swizzled by (row & 7)
+// as in the bf16 chunks: the batched W8A8 GEMM's weight layout.
+__global__ void pack8_tile_kernel(const PackChunk* __restrict__ chunks, const int32_t* __restrict__ rowidx,
+                                  const uint8_t* const* __restrict__ mats, const int* __restrict__ mat_k,
+                                  uint8_t* __restrict__ dst) {
+  const PackChunk ch = chunks[blockIdx.x];
+  const uint8_t* src = mats[ch.mat];
+  const int K = mat_k[ch.mat];
+  const int pieces = ch.nrows * 8;
+  for (int p = threadIdx.x; p < pieces; p += blockDim.x) {
+    const int row = p >> 3, c = p & 7;
+    const int sr = rowidx[ch.rowidx_off + row];
+    uint4 v = make_uint4(0, 0, 0, 0);
+    if (sr >= 0) v = *reinterpret_cast<const uint4*>(src + (size_t)sr * K + (size_t)ch.kb * 128 + c * 16);
+    *reinterpret_cast<uint4*>(dst + ch.dst_off + (size_t)row * 128 + ((c ^ (row & 7)) << 4)) = v;
+  }
+}
+
 // Per-row absmax / 448 of a bf16 matrix [rows, K] (R8: s = absmax / 448, 1 for
 // an all-zero row).  One warp per row.
 __global__ void fp8_row_scale_kernel(const uint16_t* __restrict__ w, int rows, int K,
@@ -202,6 +221,13 @@ cudaError_t launch_pack8(const PackChunk* chunks, int nchunks, const int32_t* ro
                          const uint8_t* const* mats, const int* mat_k, uint8_t* dst, cudaStream_t st) {
   if (nchunks == 0) return cudaSuccess;
   pack8_kernel<<<nchunks, 256, 0, st>>>(chunks, rowidx, mats, mat_k, dst);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pack8_tile(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
+                              const uint8_t* const* mats, const int* mat_k, uint8_t* dst, cudaStream_t st) {
+  if (nchunks == 0) return cudaSuccess;
+  pack8_tile_kernel<<<nchunks, 256, 0, st>>>(chunks, rowidx, mats, mat_k, dst);
   return cudaGetLastError();
 }
 

@@ -55,6 +55,7 @@ class ExpertShape:
     weight_std: float = 0.02
     fp8: bool = False
     nvfp4_gu: bool = False     # E4M3 linears with an NVFP4 gate_up
+    w8a8: bool = False         # E4M3 linears and per-token E4M3 linear inputs (batched path)
 
     @property
     def n_mod(self) -> int:
@@ -104,6 +105,10 @@ WORKLOADS: Dict[str, ExpertShape] = {
     "lingbot_l4_p256_n10": ExpertShape(4, 1024, 16, 2, 128, 4096, 75, 256, 10),
     # The same four layers with 64 requests: the profiling case of the batched path.
     "lingbot_l4_b64_p256_n10": ExpertShape(4, 1024, 16, 2, 128, 4096, 75, 256, 10, batch=64),
+    # 64 requests with E4M3 weights and per-token E4M3 activations (W8A8).
+    "lingbot_w8a8_b64_p256_n10": ExpertShape(36, 1024, 16, 2, 128, 4096, 75, 256, 10, batch=64, w8a8=True),
+    # Its four-layer profiling case.
+    "lingbot_l4_w8a8_b64_p256_n10": ExpertShape(4, 1024, 16, 2, 128, 4096, 75, 256, 10, batch=64, w8a8=True),
 }
 
 
