@@ -256,8 +256,9 @@ fm_status fm_get_nvfp4_weights(fm_expert *h, int layer, int which, uint8_t *code
 
 /* Test hook: R11 per-token E4M3 of `M` bf16 rows x[M, K] (host or device)
  * with the row-quantiser kernel of the W8A8 path (the pass that follows
- * attention and SwiGLU): s_m = amax_m / 448 in fp32 (1 for a zero row),
- * codes = E4M3(x / s_m), nearest-even, saturating.  Writes host codes
+ * attention and SwiGLU): s_m = amax_m / 448 and r_m = 448 / amax_m in fp32
+ * (both 1 for a zero row), codes = E4M3(x r_m) with the product in fp32,
+ * nearest-even, saturating.  Writes host codes
  * [M, K] and host scales [M].  K a multiple of 256 and at most 4096.
  * Allocates and frees temporary device memory; synchronises `stream`. */
 fm_status fm_quantize_act_e4m3(fm_expert *h, const uint16_t *x, int M, int K, uint8_t *codes,

@@ -40,9 +40,11 @@ The pages print no formula, so the conventions below are the plainest readings
      nearest-even of (w / s_c) in fp32, saturated at 448; w' = q * s_c.
   R9 prefix cache rows: K = RoPE(x Wk^T) at positions 0 .. P-1, V = x Wv^T
      from each layer's prefix hidden states x, stored as bf16.
-  R11 E4M3 activations (the batched path's W8A8 option): each input row of
-     the four per-layer linears, taken in fp32, is quantised per token:
-     s = amax_row / 448 (fp32), y' = E4M3(y / s) s.
+  R11 E4M3 activations (the batched path's W8A8 option; the pages fix FP8
+     linears but no activation quantiser): each input row of the four
+     per-layer linears, taken in fp32, is quantised per token with
+     r = 448 / amax_row and s = amax_row / 448 (both fp32, 1 for a zero row):
+     codes = E4M3(y r) with the product in fp32, y' = codes s.
   R10 NVFP4 gate_up (with E4M3 R8 for the other linears): per tensor
      g = amax / (6 * 448) (fp32); per row and 16-column block
      s_b = E4M3 nearest-even of (amax_b / (6 g)) in fp32; codes = E2M1
@@ -351,12 +353,16 @@ def fp8_quantize_rows(w_bits: np.ndarray):
 
 def fp8_quantize_act(y: np.ndarray):
     """R11: per-token E4M3 of activation rows (last axis) of the fp32 values:
-    s = amax_row / 448 in fp32 (1 for an all-zero row), codes = E4M3(y / s)
-    with the quotient in fp32.  Returns (codes uint8, s float32)."""
+    r = 448 / amax_row and s = amax_row / 448 in fp32 (both 1 for an all-zero
+    row), codes = E4M3(y r) with the product in fp32.  Returns (codes uint8,
+    s float32)."""
     y32 = np.asarray(y, dtype=np.float32)
     amax = np.max(np.abs(y32), axis=-1)
-    s = np.where(amax > 0, amax / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
-    codes = e4m3_encode((y32 / s[..., None]).astype(np.float32))
+    nz = amax > 0
+    safe = np.where(nz, amax, np.float32(1.0)).astype(np.float32)
+    s = np.where(nz, safe / np.float32(E4M3_MAX), np.float32(1.0)).astype(np.float32)
+    r = np.where(nz, np.float32(E4M3_MAX) / safe, np.float32(1.0)).astype(np.float32)
+    codes = e4m3_encode((y32 * r[..., None]).astype(np.float32))
     return codes, s
 
 

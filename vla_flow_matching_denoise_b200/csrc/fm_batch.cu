@@ -26,7 +26,6 @@
 // (K = 128 per k-block), issues tcgen05.mma kind::f8f6f4 (K = 32 each), and
 // the epilogue scales D by s_a[m] s_w[n] before the fused work.
 #include <cuda_bf16.h>
-#include <cuda_fp8.h>
 #include <cstddef>
 #include <cstdint>
 #include <utility>
@@ -39,13 +38,17 @@ namespace fm {
 
 namespace {
 
+constexpr int kBEpiWarps = 4;                        // warps 2 .. 5
+constexpr int kBThreads = 64 + 32 * kBEpiWarps;
+
 template <int BN>
 struct BCfg {
   static constexpr int kA = kBM * 128;          // A block bytes (128 rows x 64 bf16)
   static constexpr int kW = BN * 128;           // weight chunk bytes
   static constexpr int kStage = kA + kW;
   static constexpr int kStages = kBRing / kStage;
-  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStage + 256;
+  static constexpr size_t kColF = (size_t)kBEpiWarps * BN * 4;   // per-column epilogue factors, per warp
+  static constexpr size_t kSmem = 1024 + (size_t)kStages * kStage + 256 + kColF;
 };
 
 __device__ __forceinline__ uint8_t* align1024(uint8_t* p) {
@@ -72,15 +75,19 @@ __device__ __forceinline__ size_t act8_off(int m, int c, int K) {
 
 __device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
 
-// R11 per-token scale of a row with largest magnitude `amax` (1 for a zero row).
+// R11 per-token factors of a row with largest magnitude `amax`: the
+// dequantisation scale s = amax / 448 and the quantisation factor
+// r = 448 / amax (both 1 for a zero row); codes = E4M3(y r).
 __device__ __forceinline__ float act_scale(float amax) { return amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f; }
+__device__ __forceinline__ float act_rcp(float amax) { return amax > 0.f ? __fdiv_rn(448.0f, amax) : 1.0f; }
 
-// E4M3 code of y / s (true division, nearest-even, saturating finite).
-__device__ __forceinline__ uint32_t e4m3_of(float y, float s) {
-  return (uint32_t)__nv_cvt_float_to_fp8(__fdiv_rn(y, s), __NV_SATFINITE, __NV_E4M3);
+// E4M3 codes of four values times r, packed little-end first.
+__device__ __forceinline__ uint32_t e4m3x4_of(float a, float b, float c, float d, float r) {
+  return f32x2_to_e4m3x2(__fmul_rn(a, r), __fmul_rn(b, r)) | (f32x2_to_e4m3x2(__fmul_rn(c, r), __fmul_rn(d, r)) << 16);
 }
 
-// Multiplies v[0..15] by sa * sw[n0 .. n0 + 15] (E4M3 GEMM dequantisation).
+// Multiplies v[0..15] by sa * sw[0 .. 15] (E4M3 GEMM dequantisation; sw in
+// shared memory, the same address for every lane).
 __device__ __forceinline__ void dequant16(float (&v)[16], float sa, const float* sw) {
   const float4* w4 = reinterpret_cast<const float4*>(sw);
 #pragma unroll
@@ -99,9 +106,10 @@ __device__ __forceinline__ void dequant16(float (&v)[16], float sa, const float*
 
 // Gated residual branch: delta[m][n] = gate[n] * D[m][n] (fp32, stores only;
 // the row kernel that follows adds it to h and normalises).
+// `cs`: this tile's column factors in shared memory (gate[n] s_w[n]).
 template <int BN, bool F8>
-__device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt) {
-  const float sa = (F8 && valid) ? p.a_scale[m] : 1.f;
+__device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt,
+                                          const float* cs, float sa) {
 #pragma unroll 1
   for (int cb = 0; cb < BN / 16; ++cb) {
     float v[16];
@@ -109,9 +117,12 @@ __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int
     tmem_ld_wait();
     if (!valid) continue;
     const int n0 = nt * BN + cb * 16;
-    if (F8) dequant16(v, sa, p.w_scale + n0);
+    if (F8) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v[i] *= sa;
+    }
     float4* dp = reinterpret_cast<float4*>(p.h + (size_t)m * p.N + n0);
-    const float4* gp = reinterpret_cast<const float4*>(p.gate + n0);
+    const float4* gp = reinterpret_cast<const float4*>(cs + cb * 16);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float4 g = gp[q];
@@ -121,9 +132,9 @@ __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int
 }
 
 template <int BN, bool F8>
-__device__ __forceinline__ void epi_swiglu(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt) {
+__device__ __forceinline__ void epi_swiglu(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt,
+                                           const float* cs, float sa) {
   constexpr int HALF = BN / 2;
-  const float sa = (F8 && valid) ? p.a_scale[m] : 1.f;
 #pragma unroll 1
   for (int j = 0; j < HALF / 16; ++j) {
     float g[16], u[16];
@@ -132,8 +143,8 @@ __device__ __forceinline__ void epi_swiglu(const BGemmParams& p, uint32_t ta, in
     tmem_ld_wait();
     if (!valid) continue;
     if (F8) {
-      dequant16(g, sa, p.w_scale + nt * BN + j * 16);
-      dequant16(u, sa, p.w_scale + nt * BN + HALF + j * 16);
+      dequant16(g, sa, cs + j * 16);
+      dequant16(u, sa, cs + HALF + j * 16);
     }
     const int uc = nt * HALF + j * 16;
     uint32_t pk[8];
@@ -156,8 +167,8 @@ __device__ __forceinline__ void store_row16(uint16_t* rowp, int row, int e0, con
 }
 
 template <int BN, bool F8>
-__device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt) {
-  const float sa = (F8 && valid) ? p.a_scale[m] : 1.f;
+__device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt,
+                                        const float* cs, float sa) {
   const int hd = p.hd, half = hd / 2;
   const int qn = p.Hq * hd, kn = p.Hkv * hd, G = p.Hq / p.Hkv;
   const int b = valid ? m / p.T : 0, t = valid ? m % p.T : 0;
@@ -187,8 +198,8 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
         tmem_ld_wait();
         if (!valid) continue;
         if (F8) {
-          dequant16(lo, sa, p.w_scale + col0 + c);
-          dequant16(hi, sa, p.w_scale + col0 + half + c);
+          dequant16(lo, sa, cs + ho + c);
+          dequant16(hi, sa, cs + ho + half + c);
         }
         float ol[16], oh[16];
         const float4* r4 = reinterpret_cast<const float4*>(rope + c);   // (cos, sin) pairs, 128 B
@@ -210,7 +221,7 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
         tmem_ld16(ta + ho + c, v);
         tmem_ld_wait();
         if (!valid) continue;
-        if (F8) dequant16(v, sa, p.w_scale + col0 + c);
+        if (F8) dequant16(v, sa, cs + ho + c);
         store_row16(rowp, row, c, v);
       }
     }
@@ -219,7 +230,7 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
 
 // ------------------------------------------------------------------ GEMM
 template <int BN, int EPI, bool F8>
-__global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constant__ BGemmParams p) {
+__global__ void __launch_bounds__(kBThreads, 1) bgemm_kernel(const __grid_constant__ BGemmParams p) {
   using C = BCfg<BN>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* ring = align1024(smem_raw);
@@ -230,6 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
   uint64_t* tempty = tfull + 2;            // [2]
   uint64_t* drain = tempty + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  float* colf = reinterpret_cast<float*>(ring + (size_t)C::kStages * C::kStage + 256);   // [4 warps][BN]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nkb = F8 ? p.K / 128 : p.K / 64;   // k-blocks of 128-byte rows
@@ -244,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(smem_u32(&tfull[a]), 1);
-      mbar_init(smem_u32(&tempty[a]), kComputeWarps);
+      mbar_init(smem_u32(&tempty[a]), kBEpiWarps);
     }
     mbar_init(smem_u32(drain), 1);
     fence_mbar_init();
@@ -349,21 +361,37 @@ __global__ void __launch_bounds__(kThreads, 1) bgemm_kernel(const __grid_constan
     grid_dep_wait();                             // outputs and epilogue operands follow the previous kernel
     const int q4 = warp & 3;                     // TMEM lane quarter this warp may read
     const int row = 32 * q4 + lane;
+    // per-column factors, one copy per warp (no cross-warp barrier): gate *
+    // s_w (residual), s_w (E4M3 gate_up / QKV)
+    constexpr bool kColFactors = EPI == BE_RESID || F8;
+    float* cs = colf + (warp - 2) * BN;
     uint32_t local = 0;
     for (int tile = blockIdx.x; tile < ntiles; tile += gridDim.x, ++local) {
       const uint32_t acc = local & 1;
+      const int mt = tile % MT, nt = tile / MT;
+      const int m = mt * kBM + row;
+      const bool valid = m < p.M;
+      // operands that do not depend on the accumulator are read while the
+      // MMAs of this tile still run (the warp finished reading the previous
+      // tile's factors before its last __syncwarp)
+      if (kColFactors) {
+        for (int i = lane; i < BN; i += 32) {
+          const int n = nt * BN + i;
+          const float w = F8 ? p.w_scale[n] : 1.f;
+          cs[i] = EPI == BE_RESID ? p.gate[n] * w : w;
+        }
+        __syncwarp();
+      }
+      const float sa = (F8 && valid) ? p.a_scale[m] : 1.f;
       if (!mbar_wait(smem_u32(&tfull[acc]), (local >> 1) & 1, budget)) {
         atomicOr(p.err, 0x800u);
         break;
       }
       tc_fence_after();
-      const int mt = tile % MT, nt = tile / MT;
-      const int m = mt * kBM + row;
-      const bool valid = m < p.M;
       const uint32_t ta = tmem + ((uint32_t)(32 * q4) << 16) + acc * BN;
-      if (EPI == BE_RESID) epi_resid<BN, F8>(p, ta, m, valid, nt);
-      else if (EPI == BE_SWIGLU) epi_swiglu<BN, F8>(p, ta, m, valid, nt);
-      else epi_qkv<BN, F8>(p, ta, m, valid, nt);
+      if (EPI == BE_RESID) epi_resid<BN, F8>(p, ta, m, valid, nt, cs, sa);
+      else if (EPI == BE_SWIGLU) epi_swiglu<BN, F8>(p, ta, m, valid, nt, cs, sa);
+      else epi_qkv<BN, F8>(p, ta, m, valid, nt, cs, sa);
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(smem_u32(&tempty[acc]));
@@ -405,15 +433,28 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
   for (int j = 0; j < kMaxJ; ++j)
 #pragma unroll
     for (int r = 0; r < kRowsIn; ++r) acc[j][r] = 0.f;
-#pragma unroll
-  for (int j = 0; j < kMaxJ; ++j) {
-    if (j >= nj) break;
-    const uint16_t* w = p.w_in + (size_t)(tid + 256 * j) * A;
+  // 4 inputs x 4 column groups of weights in flight per iteration (the
+  // loads are L2 hits; one at a time would leave the kernel latency-bound)
+  constexpr int kK = 4;
 #pragma unroll 1
-    for (int k = 0; k < A; ++k) {
-      const float wv = __uint_as_float((uint32_t)__ldg(w + k) << 16);
+  for (int k0 = 0; k0 < A; k0 += kK) {
+    float wv[kMaxJ][kK];
 #pragma unroll
-      for (int r = 0; r < kRowsIn; ++r) acc[j][r] = fmaf(xs[r][k], wv, acc[j][r]);
+    for (int j = 0; j < kMaxJ; ++j)
+#pragma unroll
+      for (int kk = 0; kk < kK; ++kk)
+        wv[j][kk] = (j < nj && k0 + kk < A)
+                        ? __uint_as_float((uint32_t)__ldg(p.w_in + (size_t)(tid + 256 * j) * A + k0 + kk) << 16)
+                        : 0.f;
+#pragma unroll
+    for (int kk = 0; kk < kK; ++kk) {
+      if (k0 + kk >= A) break;
+#pragma unroll
+      for (int j = 0; j < kMaxJ; ++j) {
+        if (j >= nj) break;
+#pragma unroll
+        for (int r = 0; r < kRowsIn; ++r) acc[j][r] = fmaf(xs[r][k0 + kk], wv[j][kk], acc[j][r]);
+      }
     }
   }
   float sq[kRowsIn];
@@ -486,8 +527,8 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
     float a = 0.f;
 #pragma unroll
     for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w][tid]);
-    scl[tid] = act_scale(a);
-    if (m0 + tid < p.M) p.zs[m0 + tid] = scl[tid];
+    scl[tid] = act_rcp(a);
+    if (m0 + tid < p.M) p.zs[m0 + tid] = act_scale(a);
   }
   __syncthreads();
   uint8_t* z8 = reinterpret_cast<uint8_t*>(p.z);
@@ -499,7 +540,7 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
     for (int r = 0; r < kRowsIn; ++r) {
       const int m = m0 + r;
       if (m >= p.M) break;
-      z8[act8_off(m, n, d)] = (uint8_t)e4m3_of(acc[j][r], scl[r]);
+      z8[act8_off(m, n, d)] = (uint8_t)(f32x2_to_e4m3x2(__fmul_rn(acc[j][r], scl[r]), 0.f) & 0xFFu);
     }
   }
 }
@@ -556,23 +597,23 @@ __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ B
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  const float sq = act_scale(am);
-  if (lane == 0) p.zs[m] = sq;
+  const float rq = act_rcp(am);
+  if (lane == 0) p.zs[m] = act_scale(am);
   uint8_t* z8 = reinterpret_cast<uint8_t*>(p.z);
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     if (i >= n4) break;
     const int c = 4 * (lane + 32 * i);
-    const uint32_t w = e4m3_of(v[i].x, sq) | (e4m3_of(v[i].y, sq) << 8) | (e4m3_of(v[i].z, sq) << 16) |
-                       (e4m3_of(v[i].w, sq) << 24);
-    *reinterpret_cast<uint32_t*>(z8 + act8_off(m, c, d)) = w;
+    *reinterpret_cast<uint32_t*>(z8 + act8_off(m, c, d)) = e4m3x4_of(v[i].x, v[i].y, v[i].z, v[i].w, rq);
   }
 }
 
 // R11 per-token E4M3 of a bf16 ACT128 matrix (attention output o, SwiGLU
-// output u): one warp per row; lane i holds pieces of 8 values at columns
-// 8 (i + 32 j), K a multiple of 256 and at most 4096.
-constexpr int kQuantPieces = 16;
+// output u): one warp per row, lane i taking the pieces of 8 values at
+// columns 8 (i + 32 j), K a multiple of 256 and at most 4096.  Two passes
+// over the row: its amax, then the codes; the second read of the row comes
+// from L2 (the matrix was just written and is at most 26 MB), which keeps
+// the kernel small enough for many warps in flight per SM.
 __global__ void __launch_bounds__(256) browquant_kernel(const __grid_constant__ BQuantParams p) {
   grid_dep_launch();
   grid_dep_wait();
@@ -580,33 +621,31 @@ __global__ void __launch_bounds__(256) browquant_kernel(const __grid_constant__ 
   const int lane = threadIdx.x & 31;
   if (m >= p.M) return;
   const int np = p.K / 256;
-  uint4 raw[kQuantPieces];
+  const uint16_t* src = p.src;
   float am = 0.f;
-#pragma unroll
-  for (int i = 0; i < kQuantPieces; ++i) {
-    if (i >= np) break;
-    raw[i] = *reinterpret_cast<const uint4*>(p.src + act128_off(m, 8 * (lane + 32 * i), p.K));
-    const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll 4
+  for (int i = 0; i < np; ++i) {
+    const uint4 v = __ldcg(reinterpret_cast<const uint4*>(src + act128_off(m, 8 * (lane + 32 * i), p.K)));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
     for (int q = 0; q < 4; ++q)
       am = fmaxf(am, fmaxf(fabsf(__uint_as_float(w[q] << 16)), fabsf(__uint_as_float(w[q] & 0xFFFF0000u))));
   }
 #pragma unroll
   for (int o = 16; o; o >>= 1) am = fmaxf(am, __shfl_xor_sync(0xffffffffu, am, o));
-  const float sq = act_scale(am);
-  if (lane == 0) p.scale[m] = sq;
+  const float rq = act_rcp(am);
+  if (lane == 0) p.scale[m] = act_scale(am);
+#pragma unroll 4
+  for (int i = 0; i < np; ++i) {
+    const int c = 8 * (lane + 32 * i);
+    const uint4 v = __ldcs(reinterpret_cast<const uint4*>(src + act128_off(m, c, p.K)));
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    uint32_t out[2];
 #pragma unroll
-  for (int i = 0; i < kQuantPieces; ++i) {
-    if (i >= np) break;
-    const uint32_t w[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
-    uint32_t out[2] = {0u, 0u};
-#pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const uint32_t lo = e4m3_of(__uint_as_float(w[q] << 16), sq);
-      const uint32_t hi = e4m3_of(__uint_as_float(w[q] & 0xFFFF0000u), sq);
-      out[q >> 1] |= (lo | (hi << 8)) << (16 * (q & 1));
-    }
-    *reinterpret_cast<uint2*>(p.dst + act8_off(m, 8 * (lane + 32 * i), p.K)) = make_uint2(out[0], out[1]);
+    for (int q = 0; q < 2; ++q)
+      out[q] = e4m3x4_of(__uint_as_float(w[2 * q] << 16), __uint_as_float(w[2 * q] & 0xFFFF0000u),
+                         __uint_as_float(w[2 * q + 1] << 16), __uint_as_float(w[2 * q + 1] & 0xFFFF0000u), rq);
+    *reinterpret_cast<uint2*>(p.dst + act8_off(m, c, p.K)) = make_uint2(out[0], out[1]);
   }
 }
 
@@ -642,11 +681,21 @@ __global__ void __launch_bounds__(256) boutproj_kernel(const __grid_constant__ B
     float acc[kRowsIn];
 #pragma unroll
     for (int r = 0; r < kRowsIn; ++r) acc[r] = 0.f;
+    // 8 weights in flight per lane per iteration (L2 hits)
+    constexpr int kU = 8;
 #pragma unroll 1
-    for (int c = lane; c < d; c += 32) {
-      const float wv = __uint_as_float((uint32_t)__ldg(w + c) << 16);
+    for (int c0 = lane; c0 < d; c0 += 32 * kU) {
+      float wv[kU];
 #pragma unroll
-      for (int r = 0; r < kRowsIn; ++r) acc[r] = fmaf(ys[(size_t)r * d + c], wv, acc[r]);
+      for (int u = 0; u < kU; ++u)
+        wv[u] = c0 + 32 * u < d ? __uint_as_float((uint32_t)__ldg(w + c0 + 32 * u) << 16) : 0.f;
+#pragma unroll
+      for (int u = 0; u < kU; ++u) {
+        const int c = c0 + 32 * u;
+        if (c >= d) break;
+#pragma unroll
+        for (int r = 0; r < kRowsIn; ++r) acc[r] = fmaf(ys[(size_t)r * d + c], wv[u], acc[r]);
+      }
     }
 #pragma unroll
     for (int r = 0; r < kRowsIn; ++r)
@@ -885,12 +934,13 @@ cudaError_t launch_pdl(void (*kernel)(Params...), int grid, int block, size_t sm
 template <int BN, int EPI, bool F8>
 cudaError_t launch_bgemm_t(const BGemmParams& p, int n_sms, cudaStream_t st) {
   using C = BCfg<BN>;
+  static_assert(C::kSmem <= 232448, "bgemm shared memory exceeds the per-block limit");
   cudaError_t e = cudaFuncSetAttribute(bgemm_kernel<BN, EPI, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)C::kSmem);
   if (e != cudaSuccess) return e;
   const int ntiles = (p.Mp / kBM) * (p.N / BN);
   const int grid = ntiles < n_sms ? ntiles : n_sms;
-  return launch_pdl(bgemm_kernel<BN, EPI, F8>, grid, kThreads, C::kSmem, st, p);
+  return launch_pdl(bgemm_kernel<BN, EPI, F8>, grid, kBThreads, C::kSmem, st, p);
 }
 
 template <bool F8>

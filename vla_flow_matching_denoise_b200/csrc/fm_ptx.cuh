@@ -327,6 +327,15 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 // Two E4M3 codes (low byte = first element) -> two bf16 values (low half =
 // first).  E4M3 -> f16 -> f32 -> bf16 is exact at every step: an E4M3 value
 // has 4 significant bits and a binary exponent in [-9, 8].
+// E4M3 codes of two fp32 values (nearest-even, saturating finite): code(lo)
+// in bits 0-7, code(hi) in bits 8-15 (cvt puts its first source in the upper
+// half).
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
   uint32_t h2, r;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
