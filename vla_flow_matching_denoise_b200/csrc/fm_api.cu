@@ -80,7 +80,6 @@ struct fm_expert {
   uint16_t* bo = nullptr;            // ACT128 [Mp/128][Hq*hd/64]
   uint16_t* bu = nullptr;            // ACT128 [Mp/128][F/64]
   float* bh = nullptr;               // [Mp][d] residual
-  float* bdelta = nullptr;           // [Mp][d] gated branch of o_proj / down
   uint16_t* bq = nullptr;            // [B_cap][Hkv][q_rows][hd]
   // W8A8: weight scales by GEMM column, activation codes and their row scales
   float* bwscale = nullptr;          // [L][bw_stride]: the four linears' columns in tile order
@@ -773,11 +772,10 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
   r.w_out = h->w_out;
   r.out_bias = h->out_bias;
   r.h = h->bh;
-  r.delta = h->bdelta;
   BGemmParams g{};
   g.M = M;
   g.Mp = Mp;
-  g.h = h->bdelta;
+  g.h = h->bh;   // the residual GEMMs add their branch into h
   g.u_act = h->bu;
   g.F = F;
   g.qbuf = h->bq;
@@ -873,13 +871,13 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       g.N = d;
       g.gate = lm + 5 * d;
       if (e == cudaSuccess) e = launch_bgemm(g, BE_RESID, h->n_sms, st);
-      // h += gated down branch; the next layer's attention norm (none after
-      // the last layer: the out-proj kernel applies the final norm)
+      // the next layer's attention norm (none after the last layer: the
+      // out-proj kernel applies the final norm)
       r.s = lm + 6 * d;
       r.b = lm + 7 * d;
-      r.z = l + 1 < L ? h->bz_a : nullptr;
+      r.z = h->bz_a;
       r.zs = sa_za;
-      if (e == cudaSuccess) e = launch_bresnorm(r, st);
+      if (e == cudaSuccess && l + 1 < L) e = launch_bresnorm(r, st);
     }
     r.s = mrow + (size_t)6 * L * d;
     r.b = r.s + d;
@@ -1058,7 +1056,6 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
     ALLOC_OR_BAIL(h->bo, Mp * c.n_q_heads * c.head_dim * 2);
     ALLOC_OR_BAIL(h->bu, Mp * c.d_ff * 2);
     ALLOC_OR_BAIL(h->bh, Mp * d * 4);
-    ALLOC_OR_BAIL(h->bdelta, Mp * d * 4);
     ALLOC_OR_BAIL(h->bq, B * c.n_kv_heads * h->q_rows * c.head_dim * 2);
     if (h->w8a8) {
       ALLOC_OR_BAIL(h->bo8, Mp * c.n_q_heads * c.head_dim);

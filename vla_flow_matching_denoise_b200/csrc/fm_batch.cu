@@ -8,8 +8,9 @@
 // One Euler step is a chain of launches (captured in one CUDA graph per
 // (B, n) by the host):
 //   in-proj + AdaRMSNorm -> L x (QKV GEMM + RoPE -> GQA attention -> o_proj
-//   GEMM + gated residual -> AdaRMSNorm -> gate_up GEMM + SwiGLU -> down GEMM
-//   + gated residual -> AdaRMSNorm) -> final AdaRMSNorm + out-proj + Euler.
+//   GEMM adding its gated branch into h -> AdaRMSNorm -> gate_up GEMM + SwiGLU
+//   -> down GEMM adding its gated branch into h -> AdaRMSNorm, except after
+//   the last layer) -> final AdaRMSNorm + out-proj + Euler.
 //
 // GEMM (bgemm_kernel): persistent, one CTA per SM.  Warp 0 streams the 16 KB
 // A block and the BN x 64 weight chunk of every k-block into a 192 KB ring by
@@ -104,8 +105,9 @@ __device__ __forceinline__ void dequant16(float (&v)[16], float sa, const float*
 // Thread = one accumulator row (TMEM lane); `ta` is the TMEM address of column
 // 0 of this tile for the thread's lane quarter.
 
-// Gated residual branch: delta[m][n] = gate[n] * D[m][n] (fp32, stores only;
-// the row kernel that follows adds it to h and normalises).
+// Gated residual: h[m][n] += gate[n] * D[m][n], one vector atomic add per 4
+// elements (no read back into the epilogue; the row kernel that follows
+// normalises h).
 // `cs`: this tile's column factors in shared memory (gate[n] s_w[n]).
 template <int BN, bool F8>
 __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int m, bool valid, int nt,
@@ -121,12 +123,12 @@ __device__ __forceinline__ void epi_resid(const BGemmParams& p, uint32_t ta, int
 #pragma unroll
       for (int i = 0; i < 16; ++i) v[i] *= sa;
     }
-    float4* dp = reinterpret_cast<float4*>(p.h + (size_t)m * p.N + n0);
+    float* hp = p.h + (size_t)m * p.N + n0;
     const float4* gp = reinterpret_cast<const float4*>(cs + cb * 16);
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
       const float4 g = gp[q];
-      dp[q] = make_float4(g.x * v[4 * q], g.y * v[4 * q + 1], g.z * v[4 * q + 2], g.w * v[4 * q + 3]);
+      red_add_v4(hp + 4 * q, g.x * v[4 * q], g.y * v[4 * q + 1], g.z * v[4 * q + 2], g.w * v[4 * q + 3]);
     }
   }
 }
@@ -545,8 +547,9 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
   }
 }
 
-// Gated residual + AdaRMSNorm, one warp per row: h += delta, then (unless z
-// is null) z = bf16(h rstd (1 + s) + b) in ACT128.
+// AdaRMSNorm after a residual GEMM (which added its branch into h), one warp
+// per row: unless z is null, z = bf16(h rstd (1 + s) + b) in ACT128 (or E4M3
+// codes with a row scale).
 __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ BRowParams p) {
   grid_dep_launch();
   grid_dep_wait();
@@ -560,10 +563,7 @@ __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ B
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     if (i >= n4) break;
-    const float4 br = reinterpret_cast<const float4*>(p.delta + (size_t)m * d)[lane + 32 * i];
-    const float4 a = hr[lane + 32 * i];
-    v[i] = make_float4(a.x + br.x, a.y + br.y, a.z + br.z, a.w + br.w);
-    hr[lane + 32 * i] = v[i];
+    v[i] = hr[lane + 32 * i];
     s = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, fmaf(v[i].w, v[i].w, s))));
   }
   if (p.z == nullptr) return;

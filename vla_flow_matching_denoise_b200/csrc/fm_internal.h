@@ -140,7 +140,8 @@ struct BGemmParams {
   int K, N, M, Mp;           // reduction, output channels, valid rows (B*T), padded rows
   const float* a_scale;      // E4M3 only: [Mp] row scale of A (per token)
   const float* w_scale;      // E4M3 only: [N] scale of the weight row behind each GEMM column
-  // BE_RESID: h[m][n] = gate[n] * D[m][n]   (fp32 residual branch, row stride N)
+  // BE_RESID: h[m][n] += gate[n] * D[m][n] (fp32 residual, row stride N; one
+  // atomic add per element: tiles are disjoint, so no order dependence)
   float* h;
   const float* gate;
   // BE_SWIGLU: tile j holds gate rows 128j.. then up rows 128j..; u = SiLU(g) up
@@ -171,7 +172,6 @@ struct BRowParams {          // in-proj, AdaRMSNorm, out-proj + Euler (row kerne
   const uint16_t* w_out;     // [A][d]
   const float* out_bias;     // [A] or null
   float* h;                  // [Mp][d] fp32 residual
-  const float* delta;        // [Mp][d] fp32 gated branch added to h (residual + norm kernel)
   const float* s;            // norm scale and shift [d]
   const float* b;
   uint16_t* z;               // ACT128 [Mp/128][d/64] (bf16), or ACT8 codes when zs is set

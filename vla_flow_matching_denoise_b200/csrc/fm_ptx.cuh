@@ -327,6 +327,12 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
 // Two E4M3 codes (low byte = first element) -> two bf16 values (low half =
 // first).  E4M3 -> f16 -> f32 -> bf16 is exact at every step: an E4M3 value
 // has 4 significant bits and a binary exponent in [-9, 8].
+// Four fp32 atomic adds to 16 consecutive bytes of global memory, no return.
+__device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
 // E4M3 codes of two fp32 values (nearest-even, saturating finite): code(lo)
 // in bits 0-7, code(hi) in bits 8-15 (cvt puts its first source in the upper
 // half).
