@@ -14,6 +14,7 @@
 #include <vector>
 
 #include "../../include/fm_expert.h"
+#include "fm_batch.h"
 #include "fm_internal.h"
 #include "fm_launch.h"
 
@@ -57,6 +58,7 @@ struct fm_expert {
   uint8_t* w2_packed = nullptr;
   uint16_t* w1 = nullptr;
   uint16_t* w_in = nullptr;
+  uint16_t* w_in_t = nullptr;        // [A][d]: the batched in-proj's transposed copy
   uint16_t* w_out = nullptr;
   float* out_bias = nullptr;
   // E4M3 weights: row scales by packed channel (read by the kernel) and, for
@@ -612,6 +614,11 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   DALLOC(h->w_in, (size_t)d * c.action_dim * 2);
   st = upload_rows(h, h->w_in, w->in_proj, (size_t)d * c.action_dim, "in_proj");
   if (st != FM_OK) return st;
+  if (h->batched) {
+    DALLOC(h->w_in_t, (size_t)d * c.action_dim * 2);
+    CK(launch_transpose_bf16(h->w_in, d, c.action_dim, h->w_in_t, 0));
+    CK(cudaDeviceSynchronize());
+  }
   DALLOC(h->w_out, (size_t)d * c.action_dim * 2);
   st = upload_rows(h, h->w_out, w->out_proj, (size_t)d * c.action_dim, "out_proj");
   if (st != FM_OK) return st;
@@ -769,6 +776,7 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
   r.x_out = update ? h->x : nullptr;
   r.v_out = h->vbuf;
   r.w_in = h->w_in;
+  r.w_in_t = h->w_in_t;
   r.w_out = h->w_out;
   r.out_bias = h->out_bias;
   r.h = h->bh;

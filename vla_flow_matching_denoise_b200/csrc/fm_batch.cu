@@ -31,6 +31,7 @@
 #include <cstdint>
 #include <utility>
 
+#include "fm_batch.h"
 #include "fm_internal.h"
 #include "fm_launch.h"
 #include "fm_ptx.cuh"
@@ -410,7 +411,9 @@ __global__ void __launch_bounds__(kBThreads, 1) bgemm_kernel(const __grid_consta
 // ------------------------------------------------------------------ row kernels
 // In-proj + AdaRMSNorm of layer 0: 16 rows per CTA (256 threads); thread t
 // computes columns t + 256 j of h = x W_in^T for the 16 rows, then the rows'
-// rstd (block reduction) and z = bf16(h rstd (1 + s) + b).
+// rstd (block reduction) and z = bf16(h rstd (1 + s) + b).  The weights are
+// read transposed (w_in_t [A][d]), so a warp's loads for one input are 64
+// contiguous bytes.
 // F8: z as E4M3 codes with per-row scales (p.zs).
 constexpr int kRowsIn = 16;
 template <bool F8>
@@ -446,7 +449,7 @@ __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BR
 #pragma unroll
       for (int kk = 0; kk < kK; ++kk)
         wv[j][kk] = (j < nj && k0 + kk < A)
-                        ? __uint_as_float((uint32_t)__ldg(p.w_in + (size_t)(tid + 256 * j) * A + k0 + kk) << 16)
+                        ? __uint_as_float((uint32_t)__ldg(p.w_in_t + (size_t)(k0 + kk) * d + tid + 256 * j) << 16)
                         : 0.f;
 #pragma unroll
     for (int kk = 0; kk < kK; ++kk) {
@@ -557,15 +560,20 @@ __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ B
   const int lane = threadIdx.x & 31;
   if (m >= p.M) return;
   const int d = p.d, n4 = d / 128;   // float4 per lane
-  float4* hr = reinterpret_cast<float4*>(p.h + (size_t)m * d);
-  float4 v[8];
-  float s = 0.f;
+  const float4* hr = reinterpret_cast<const float4*>(p.h + (size_t)m * d);
+  // every load of the row and of the modulation in flight before the first use
+  float4 v[8], scv[8], shv[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
-    if (i >= n4) break;
-    v[i] = hr[lane + 32 * i];
-    s = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, fmaf(v[i].w, v[i].w, s))));
+    const bool in = i < n4;
+    v[i] = in ? hr[lane + 32 * i] : make_float4(0.f, 0.f, 0.f, 0.f);
+    scv[i] = in ? *reinterpret_cast<const float4*>(p.s + 4 * (lane + 32 * i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    shv[i] = in ? *reinterpret_cast<const float4*>(p.b + 4 * (lane + 32 * i)) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    s = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, fmaf(v[i].w, v[i].w, s))));
   if (p.z == nullptr) return;
 #pragma unroll
   for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
@@ -575,8 +583,8 @@ __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ B
     for (int i = 0; i < 8; ++i) {
       if (i >= n4) break;
       const int c = 4 * (lane + 32 * i);
-      const float4 sc = *reinterpret_cast<const float4*>(p.s + c);
-      const float4 sh = *reinterpret_cast<const float4*>(p.b + c);
+      const float4 sc = scv[i];
+      const float4 sh = shv[i];
       const uint32_t lo = pack2_bf16(fmaf(v[i].x * rs, 1.0f + sc.x, sh.x), fmaf(v[i].y * rs, 1.0f + sc.y, sh.y));
       const uint32_t hi = pack2_bf16(fmaf(v[i].z * rs, 1.0f + sc.z, sh.z), fmaf(v[i].w * rs, 1.0f + sc.w, sh.w));
       *reinterpret_cast<uint2*>(p.z + act128_off(m, c, d)) = make_uint2(lo, hi);
@@ -588,9 +596,8 @@ __global__ void __launch_bounds__(256) bresnorm_kernel(const __grid_constant__ B
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     if (i >= n4) break;
-    const int c = 4 * (lane + 32 * i);
-    const float4 sc = *reinterpret_cast<const float4*>(p.s + c);
-    const float4 sh = *reinterpret_cast<const float4*>(p.b + c);
+    const float4 sc = scv[i];
+    const float4 sh = shv[i];
     v[i] = make_float4(fmaf(v[i].x * rs, 1.0f + sc.x, sh.x), fmaf(v[i].y * rs, 1.0f + sc.y, sh.y),
                        fmaf(v[i].z * rs, 1.0f + sc.z, sh.z), fmaf(v[i].w * rs, 1.0f + sc.w, sh.w));
     am = fmaxf(am, fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w))));
@@ -660,20 +667,38 @@ __global__ void __launch_bounds__(256) boutproj_kernel(const __grid_constant__ B
   const int m0 = blockIdx.x * kRowsIn;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int d = p.d, A = p.A;
+  // final norm of the block's rows: lane i holds float4 columns 4 (i + 32 j),
+  // all loads in flight before the reduction (d a multiple of 128, <= 1024)
+  const int n4 = d / 128;
   for (int r = warp; r < kRowsIn; r += 8) {
     const int m = m0 + r;
-    float* y = ys + (size_t)r * d;
-    if (m >= p.M) {
-      for (int c = lane; c < d; c += 32) y[c] = 0.f;
-      continue;
-    }
-    const float* hr = p.h + (size_t)m * d;
+    float4* y = reinterpret_cast<float4*>(ys + (size_t)r * d);
+    const bool row_ok = m < p.M;
+    const float4* hr = reinterpret_cast<const float4*>(p.h + (size_t)(row_ok ? m : 0) * d);
+    float4 v[8], scv[8], shv[8];
     float s = 0.f;
-    for (int c = lane; c < d; c += 32) s = fmaf(hr[c], hr[c], s);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool in = i < n4;
+      v[i] = in && row_ok ? hr[lane + 32 * i] : make_float4(0.f, 0.f, 0.f, 0.f);
+      scv[i] = in ? *reinterpret_cast<const float4*>(p.s + 4 * (lane + 32 * i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      shv[i] = in ? *reinterpret_cast<const float4*>(p.b + 4 * (lane + 32 * i)) : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      s = fmaf(v[i].x, v[i].x, fmaf(v[i].y, v[i].y, fmaf(v[i].z, v[i].z, fmaf(v[i].w, v[i].w, s))));
 #pragma unroll
     for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
     const float rs = 1.0f / sqrtf(s / (float)d + p.eps);
-    for (int c = lane; c < d; c += 32) y[c] = fmaf(hr[c] * rs, 1.0f + p.s[c], p.b[c]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (i >= n4) break;
+      y[lane + 32 * i] = row_ok ? make_float4(fmaf(v[i].x * rs, 1.0f + scv[i].x, shv[i].x),
+                                              fmaf(v[i].y * rs, 1.0f + scv[i].y, shv[i].y),
+                                              fmaf(v[i].z * rs, 1.0f + scv[i].z, shv[i].z),
+                                              fmaf(v[i].w * rs, 1.0f + scv[i].w, shv[i].w))
+                                : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
   __syncthreads();
   for (int a = warp; a < A; a += 8) {

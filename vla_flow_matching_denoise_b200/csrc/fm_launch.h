@@ -4,6 +4,7 @@
 #include <cstddef>
 #include <cstdint>
 
+#include "fm_batch.h"
 #include "fm_internal.h"
 
 namespace fm {
@@ -24,6 +25,7 @@ cudaError_t launch_fp8_quantize(const uint16_t* w, int rows, int K, float* scale
 cudaError_t launch_kv_copy(const uint16_t* src, int B, int P, const int* lens, int Hkv, int hd, int S_max,
                            uint16_t* cache, cudaStream_t st);
 cudaError_t launch_rope_table(int B, int T, int hd, const int* P, double base, float* tab, cudaStream_t st);
+cudaError_t launch_transpose_bf16(const uint16_t* src, int rows, int cols, uint16_t* dst, cudaStream_t st);
 
 size_t time_gemm_smem_bytes(int d);
 cudaError_t launch_time(const TimeParams& p, int n_sms, cudaStream_t st);

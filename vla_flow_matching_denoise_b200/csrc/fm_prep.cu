@@ -209,6 +209,21 @@ __global__ void rope_table_kernel(int B, int T, int hd, const int* __restrict__ 
   tab[2 * i + 1] = (float)sin(ang);
 }
 
+// dst[c][r] = src[r][c] for a bf16 matrix [rows][cols].
+__global__ void transpose_bf16_kernel(const uint16_t* __restrict__ src, int rows, int cols,
+                                      uint16_t* __restrict__ dst) {
+  const size_t n = (size_t)rows * cols;
+  for (size_t i = blockIdx.x * (size_t)blockDim.x + threadIdx.x; i < n; i += (size_t)gridDim.x * blockDim.x) {
+    const size_t r = i / cols, c = i % cols;
+    dst[c * rows + r] = src[i];
+  }
+}
+
+cudaError_t launch_transpose_bf16(const uint16_t* src, int rows, int cols, uint16_t* dst, cudaStream_t st) {
+  transpose_bf16_kernel<<<256, 256, 0, st>>>(src, rows, cols, dst);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_pack(const PackChunk* chunks, int nchunks, const int32_t* rowidx,
                         const uint16_t* const* mats, const int* mat_k, uint8_t* dst,
                         cudaStream_t st) {
