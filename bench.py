@@ -389,9 +389,10 @@ def main():
         "clocks": clk.summary(),
         "e2e": {"value": e2e_value, "unit": UNIT, "ms_per_chunk": ms_e2e / args.steps,
                 "h2d_bytes_per_step": int(x0.nbytes), "d2h_bytes_per_step": int(x0.nbytes)},
-        # per Euler step: in-proj, per layer (QKV, attention, o_proj, norm, gate_up, down,
-        # norm but none after the last layer), out-proj; per call the two time-MLP kernels
-        "gpu_launches": args.steps * ((2 + n * (per_layer_launches * shape.n_layers + 1)) if batched else (2 + B)),
+        # per Euler step: in-proj, layer 0's norm, per layer (QKV, attention, o_proj, norm,
+        # gate_up, down, norm but none after the last layer), out-proj; per call the two
+        # time-MLP kernels
+        "gpu_launches": args.steps * ((2 + n * (per_layer_launches * shape.n_layers + 2)) if batched else (2 + B)),
         "roofline": ({"bound": "tensor", "achieved": lf / (ms_loop / 1000.0) / 1e12, "peak": tpeak,
                       "unit": "TFLOP/s", "frac": lf / (ms_loop / 1000.0) / 1e12 / tpeak,
                       "traffic": traffic,

@@ -70,7 +70,8 @@ struct fm_expert {
   std::vector<int32_t> pack_rows;
   std::vector<float> row_scale;      // [L][rows of QKV + O + GU + DOWN]
   std::vector<float> nv4_g;          // NVFP4 gate_up: [L][2] tensor scales (gate, up)
-  // batched path (B >= 2 requests advance together, M = B * T rows)
+  // batched path (the requests of a call advance together, M = B * T rows: B >= 2 on
+  // a bf16 handle, every B on a W8A8 handle)
   bool batched = false;
   bool w8a8 = false;                 // E4M3 weights and per-token E4M3 activations (every B batched)
   uint8_t* barena = nullptr;         // per layer: [N/BN][K/64] chunks of each linear (W8A8: [N/BN][K/128])
@@ -829,6 +830,7 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
     r.z = h->bz_a;
     r.zs = sa_za;
     e = launch_binproj(r, st);
+    if (e == cudaSuccess) e = launch_bresnorm(r, st);   // layer 0's attention norm
     for (int l = 0; l < L && e == cudaSuccess; ++l) {
       const float* lm = mrow + (size_t)6 * l * d;
       const uint8_t* wl = h->barena + (size_t)l * h->blayer_bytes;

@@ -7,7 +7,7 @@
 //
 // One Euler step is a chain of launches (captured in one CUDA graph per
 // (B, n) by the host):
-//   in-proj + AdaRMSNorm -> L x (QKV GEMM + RoPE -> GQA attention -> o_proj
+//   in-proj -> AdaRMSNorm -> L x (QKV GEMM + RoPE -> GQA attention -> o_proj
 //   GEMM adding its gated branch into h -> AdaRMSNorm -> gate_up GEMM + SwiGLU
 //   -> down GEMM adding its gated branch into h -> AdaRMSNorm, except after
 //   the last layer) -> final AdaRMSNorm + out-proj + Euler.
@@ -409,144 +409,46 @@ __global__ void __launch_bounds__(kBThreads, 1) bgemm_kernel(const __grid_consta
 }
 
 // ------------------------------------------------------------------ row kernels
-// In-proj + AdaRMSNorm of layer 0: 16 rows per CTA (256 threads); thread t
-// computes columns t + 256 j of h = x W_in^T for the 16 rows, then the rows'
-// rstd (block reduction) and z = bf16(h rstd (1 + s) + b).  The weights are
-// read transposed (w_in_t [A][d]), so a warp's loads for one input are 64
-// contiguous bytes.
-// F8: z as E4M3 codes with per-row scales (p.zs).
+// In-proj: h = x W_in^T (fp32) for 16 rows x 256 columns per CTA, grid
+// (rows / 16, d / 256); thread t computes column 256 blockIdx.y + t for the 16
+// rows.  The weights are read transposed (w_in_t [A][d]), so a warp's loads
+// for one input are 64 contiguous bytes, four inputs in flight at a time.
+// Layer 0's AdaRMSNorm follows in the norm kernel.
 constexpr int kRowsIn = 16;
-template <bool F8>
 __global__ void __launch_bounds__(256) binproj_kernel(const __grid_constant__ BRowParams p) {
   __shared__ float xs[kRowsIn][128];
-  __shared__ float red[8][kRowsIn];
-  __shared__ float rstd[kRowsIn];
-  __shared__ float scl[kRowsIn];
   grid_dep_launch();
   grid_dep_wait();
   const int m0 = blockIdx.x * kRowsIn;
   const int tid = threadIdx.x, A = p.A, d = p.d;
+  const int n = blockIdx.y * 256 + tid;
   for (int i = tid; i < kRowsIn * A; i += 256) {
     const int r = i / A, k = i % A;
     xs[r][k] = m0 + r < p.M ? p.x[(size_t)(m0 + r) * A + k] : 0.f;
   }
   __syncthreads();
-  constexpr int kMaxJ = 4;   // d <= 1024
-  float acc[kMaxJ][kRowsIn];
-  const int nj = d / 256;
+  float acc[kRowsIn];
 #pragma unroll
-  for (int j = 0; j < kMaxJ; ++j)
-#pragma unroll
-    for (int r = 0; r < kRowsIn; ++r) acc[j][r] = 0.f;
-  // 4 inputs x 4 column groups of weights in flight per iteration (the
-  // loads are L2 hits; one at a time would leave the kernel latency-bound)
+  for (int r = 0; r < kRowsIn; ++r) acc[r] = 0.f;
   constexpr int kK = 4;
 #pragma unroll 1
   for (int k0 = 0; k0 < A; k0 += kK) {
-    float wv[kMaxJ][kK];
+    float wv[kK];
 #pragma unroll
-    for (int j = 0; j < kMaxJ; ++j)
-#pragma unroll
-      for (int kk = 0; kk < kK; ++kk)
-        wv[j][kk] = (j < nj && k0 + kk < A)
-                        ? __uint_as_float((uint32_t)__ldg(p.w_in_t + (size_t)(k0 + kk) * d + tid + 256 * j) << 16)
-                        : 0.f;
+    for (int kk = 0; kk < kK; ++kk)
+      wv[kk] = k0 + kk < A ? __uint_as_float((uint32_t)__ldg(p.w_in_t + (size_t)(k0 + kk) * d + n) << 16) : 0.f;
 #pragma unroll
     for (int kk = 0; kk < kK; ++kk) {
       if (k0 + kk >= A) break;
 #pragma unroll
-      for (int j = 0; j < kMaxJ; ++j) {
-        if (j >= nj) break;
-#pragma unroll
-        for (int r = 0; r < kRowsIn; ++r) acc[j][r] = fmaf(xs[r][k0 + kk], wv[j][kk], acc[j][r]);
-      }
-    }
-  }
-  float sq[kRowsIn];
-#pragma unroll
-  for (int r = 0; r < kRowsIn; ++r) {
-    float s = 0.f;
-#pragma unroll
-    for (int j = 0; j < kMaxJ; ++j)
-      if (j < nj) s = fmaf(acc[j][r], acc[j][r], s);
-#pragma unroll
-    for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
-    sq[r] = s;
-  }
-  if ((tid & 31) == 0)
-#pragma unroll
-    for (int r = 0; r < kRowsIn; ++r) red[tid >> 5][r] = sq[r];
-  __syncthreads();
-  if (tid < kRowsIn) {
-    float s = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) s += red[w][tid];
-    rstd[tid] = 1.0f / sqrtf(s / (float)d + p.eps);
-  }
-  __syncthreads();
-  if constexpr (!F8) {
-#pragma unroll
-    for (int j = 0; j < kMaxJ; ++j) {
-      if (j >= nj) break;
-      const int n = tid + 256 * j;
-      const float sc = 1.0f + p.s[n], sh = p.b[n];
-#pragma unroll
-      for (int r = 0; r < kRowsIn; ++r) {
-        const int m = m0 + r;
-        if (m >= p.M) break;
-        p.h[(size_t)m * d + n] = acc[j][r];
-        const __nv_bfloat16 zb = __float2bfloat16_rn(fmaf(acc[j][r] * rstd[r], sc, sh));
-        p.z[act128_off(m, n, d)] = *reinterpret_cast<const uint16_t*>(&zb);
-      }
-    }
-    return;
-  }
-  // E4M3 z: y = h rstd (1 + s) + b in fp32, the row's amax (block reduction),
-  // then the codes of y / s_row
-  float am[kRowsIn];
-#pragma unroll
-  for (int r = 0; r < kRowsIn; ++r) am[r] = 0.f;
-#pragma unroll
-  for (int j = 0; j < kMaxJ; ++j) {
-    if (j >= nj) break;
-    const int n = tid + 256 * j;
-    const float sc = 1.0f + p.s[n], sh = p.b[n];
-#pragma unroll
-    for (int r = 0; r < kRowsIn; ++r) {
-      const int m = m0 + r;
-      if (m < p.M) p.h[(size_t)m * d + n] = acc[j][r];
-      acc[j][r] = fmaf(acc[j][r] * rstd[r], sc, sh);
-      am[r] = fmaxf(am[r], fabsf(acc[j][r]));
+      for (int r = 0; r < kRowsIn; ++r) acc[r] = fmaf(xs[r][k0 + kk], wv[kk], acc[r]);
     }
   }
 #pragma unroll
   for (int r = 0; r < kRowsIn; ++r) {
-#pragma unroll
-    for (int o = 16; o; o >>= 1) am[r] = fmaxf(am[r], __shfl_xor_sync(0xffffffffu, am[r], o));
-  }
-  if ((tid & 31) == 0)
-#pragma unroll
-    for (int r = 0; r < kRowsIn; ++r) red[tid >> 5][r] = am[r];
-  __syncthreads();
-  if (tid < kRowsIn) {
-    float a = 0.f;
-#pragma unroll
-    for (int w = 0; w < 8; ++w) a = fmaxf(a, red[w][tid]);
-    scl[tid] = act_rcp(a);
-    if (m0 + tid < p.M) p.zs[m0 + tid] = act_scale(a);
-  }
-  __syncthreads();
-  uint8_t* z8 = reinterpret_cast<uint8_t*>(p.z);
-#pragma unroll
-  for (int j = 0; j < kMaxJ; ++j) {
-    if (j >= nj) break;
-    const int n = tid + 256 * j;
-#pragma unroll
-    for (int r = 0; r < kRowsIn; ++r) {
-      const int m = m0 + r;
-      if (m >= p.M) break;
-      z8[act8_off(m, n, d)] = (uint8_t)(f32x2_to_e4m3x2(__fmul_rn(acc[j][r], scl[r]), 0.f) & 0xFFu);
-    }
+    const int m = m0 + r;
+    if (m >= p.M) break;
+    p.h[(size_t)m * d + n] = acc[r];
   }
 }
 
@@ -1011,9 +913,16 @@ cudaError_t launch_rows_to_act128(const uint16_t* src, int M, int Mp, int K, uin
 }
 
 cudaError_t launch_binproj(const BRowParams& p, cudaStream_t st) {
-  const int grid = (p.M + kRowsIn - 1) / kRowsIn;
-  return p.zs != nullptr ? launch_pdl(binproj_kernel<true>, grid, 256, 0, st, p)
-                         : launch_pdl(binproj_kernel<false>, grid, 256, 0, st, p);
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.gridDim = dim3((p.M + kRowsIn - 1) / kRowsIn, p.d / 256, 1);
+  cfg.blockDim = dim3(256, 1, 1);
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, binproj_kernel, p);
 }
 
 cudaError_t launch_bresnorm(const BRowParams& p, cudaStream_t st) {
