@@ -776,7 +776,6 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
   r.x = h->x;
   r.x_out = update ? h->x : nullptr;
   r.v_out = h->vbuf;
-  r.w_in = h->w_in;
   r.w_in_t = h->w_in_t;
   r.w_out = h->w_out;
   r.out_bias = h->out_bias;

@@ -55,8 +55,7 @@ struct BRowParams {          // in-proj, AdaRMSNorm, out-proj + Euler (row kerne
   const float* x;            // [M][A] (in-proj input)
   float* x_out;              // [M][A] updated in place by out-proj (x += dt v), or null
   float* v_out;              // [M][A] velocity
-  const uint16_t* w_in;      // [d][A]
-  const uint16_t* w_in_t;    // [A][d] (the batched in-proj reads it transposed)
+  const uint16_t* w_in_t;    // [A][d]: the in-projection's weights, transposed
   const uint16_t* w_out;     // [A][d]
   const float* out_bias;     // [A] or null
   float* h;                  // [Mp][d] fp32 residual
