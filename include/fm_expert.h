@@ -65,7 +65,7 @@ typedef enum fm_status {
   FM_ERR_OOM = 3,           /* device allocation failed                         */
   FM_ERR_CUDA = 4,          /* a CUDA call failed (text in fm_last_error)       */
   FM_ERR_TIMEOUT = 5,       /* a bounded device-side wait gave up               */
-  FM_ERR_UNSUPPORTED = 6    /* shape or device this build cannot run            */
+  FM_ERR_UNSUPPORTED = 6    /* shape or device the library does not support     */
 } fm_status;
 
 typedef enum fm_wtype {

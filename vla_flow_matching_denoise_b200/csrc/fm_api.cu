@@ -982,7 +982,7 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
   if (cudaGetDeviceProperties(&prop, device) != cudaSuccess)
     return set_err(h, FM_ERR_CUDA, "cudaGetDeviceProperties failed");
   if (prop.major != 10 || prop.minor != 0)
-    return set_err(h, FM_ERR_UNSUPPORTED, "device %d is sm_%d%d; this build targets sm_100a", device,
+    return set_err(h, FM_ERR_UNSUPPORTED, "device %d is sm_%d%d; the library is compiled for sm_100a", device,
                    prop.major, prop.minor);
   if (cudaSetDevice(device) != cudaSuccess) return set_err(h, FM_ERR_CUDA, "cudaSetDevice failed");
 
