@@ -40,15 +40,15 @@ The pages print no formula, so the conventions below are the plainest readings
      nearest-even of (w / s_c) in fp32, saturated at 448; w' = q * s_c.
   R9 prefix cache rows: K = RoPE(x Wk^T) at positions 0 .. P-1, V = x Wv^T
      from each layer's prefix hidden states x, stored as bf16.
+  R10 NVFP4 gate_up (with E4M3 R8 for the other linears): per tensor
+     g = amax / (6 * 448) (fp32); per row and 16-column block
+     s_b = E4M3 nearest-even of (amax_b / (6 g)) in fp32; codes = E2M1
+     nearest-even of (w / (s_b g)) in fp32, saturated at 6; w' = q s_b g.
   R11 E4M3 activations (the batched path's W8A8 option; the pages fix FP8
      linears but no activation quantiser): each input row of the four
      per-layer linears, taken in fp32, is quantised per token with
      r = 448 / amax_row and s = amax_row / 448 (both fp32, 1 for a zero row):
      codes = E4M3(y r) with the product in fp32, y' = codes s.
-  R10 NVFP4 gate_up (with E4M3 R8 for the other linears): per tensor
-     g = amax / (6 * 448) (fp32); per row and 16-column block
-     s_b = E4M3 nearest-even of (amax_b / (6 g)) in fp32; codes = E2M1
-     nearest-even of (w / (s_b g)) in fp32, saturated at 6; w' = q s_b g.
 
 Every function below is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, hand values, brute force or independent library routines.
