@@ -44,6 +44,7 @@ def test_null_handles_are_safe(lib):
     assert lib.fm_sync(None, None) == 1
     assert lib.fm_denoise(None, None, 1, 10, None, None) == 1
     assert lib.fm_set_prefix_varlen(None, None, None, 1, None, 0, None) == 1
+    assert lib.fm_quantize_act_e4m3(None, None, 1, 256, None, None, None) == 1
 
 
 def _cfg(**kw):
