@@ -74,6 +74,21 @@ def test_create_rejects_bad_config_before_touching_the_device(lib, field, value,
     assert lib.fm_last_error(None)
 
 
+@pytest.mark.parametrize("field,value", [("d_ff", 1088), ("n_q_heads", 2), ("d_model", 192)])
+def test_create_rejects_w8a8_shapes_before_touching_the_device(lib, field, value):
+    # the W8A8 path quantises o and u per row in blocks of 256 columns and
+    # runs on the batched kernels (d a multiple of 256)
+    cfg = _cfg(wtype=binding.FM_W_W8A8_E4M3, **{field: value})
+    if field == "n_q_heads":
+        cfg.n_kv_heads = 1
+    h = ctypes.c_void_p()
+    w = binding.FmWeights()
+    st = lib.fm_expert_create(ctypes.byref(cfg), ctypes.byref(w), 0, ctypes.byref(h))
+    assert st == 6, lib.fm_last_error(None)
+    assert not h.value
+    assert b"W8A8" in lib.fm_last_error(None)
+
+
 def test_create_rejects_null_weights(lib):
     cfg = _cfg()
     h = ctypes.c_void_p()

@@ -630,6 +630,21 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
   return FM_OK;
 }
 
+// The batched path needs whole 128-column weight tiles, the in-proj's
+// 256-column thread mapping and at most 1024 residual columns.
+bool batched_shape_ok(const fm_config& c) {
+  const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
+  return c.d_model % 256 == 0 && c.d_model <= 1024 && c.d_ff % 128 == 0 && qkv % 128 == 0 &&
+         (c.n_q_heads * c.head_dim) % 64 == 0 && (c.head_dim == 64 || c.head_dim == 128);
+}
+
+// W8A8 runs every batch on the batched path and also quantises o and u per
+// row (K a multiple of 256, at most 4096).
+bool w8a8_shape_ok(const fm_config& c) {
+  const int qn = c.n_q_heads * c.head_dim;
+  return batched_shape_ok(c) && qn % 256 == 0 && qn <= 4096 && c.d_ff % 256 == 0 && c.d_ff <= 4096;
+}
+
 fm_status check_config(const fm_config* c) {
   fm_expert* h = nullptr;
   if (!c) return set_err(h, FM_ERR_INVALID_ARG, "config is NULL");
@@ -652,6 +667,10 @@ fm_status check_config(const fm_config* c) {
   if (c->wtype != FM_W_BF16 && c->wtype != FM_W_FP8_E4M3 && c->wtype != FM_W_FP8_NVFP4_GU &&
       c->wtype != FM_W_W8A8_E4M3)
     return set_err(h, FM_ERR_INVALID_ARG, "unknown wtype %d", c->wtype);
+  if (c->wtype == FM_W_W8A8_E4M3 && !w8a8_shape_ok(*c))
+    return set_err(h, FM_ERR_UNSUPPORTED,
+                   "W8A8 needs d_model a multiple of 256 (<= 1024), n_q_heads*head_dim and d_ff multiples of 256 "
+                   "(<= 4096), (n_q_heads + 2 n_kv_heads)*head_dim a multiple of 128");
   return FM_OK;
 }
 
@@ -1012,22 +1031,10 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
     set_err(h, FM_ERR_CUDA, "stream creation failed");
     return bail(FM_ERR_CUDA);
   }
-  {
-    // the batched path needs whole 128-column weight tiles, the in-proj's
-    // 256-column thread mapping and at most 1024 residual columns
-    const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
-    const bool shape_ok = c.d_model % 256 == 0 && c.d_model <= 1024 && c.d_ff % 128 == 0 && qkv % 128 == 0 &&
-                          (c.n_q_heads * c.head_dim) % 64 == 0 && (c.head_dim == 64 || c.head_dim == 128);
-    h->w8a8 = c.wtype == FM_W_W8A8_E4M3;
-    h->batched = shape_ok && ((c.wtype == FM_W_BF16 && c.max_batch >= 2) || h->w8a8);
-    // W8A8 additionally quantises o and u per row (K a multiple of 256, at
-    // most 4096) and runs every batch size on the batched path
-    const int qn = c.n_q_heads * c.head_dim;
-    if (h->w8a8 && !(shape_ok && qn % 256 == 0 && qn <= 4096 && c.d_ff % 256 == 0 && c.d_ff <= 4096)) {
-      set_err(h, FM_ERR_UNSUPPORTED, "W8A8 needs the batched path's shapes (d %% 256, H_q*hd and d_ff %% 256, <= 4096)");
-      return bail(FM_ERR_UNSUPPORTED);
-    }
-  }
+  // the batched path: bf16 handles with max_batch >= 2, and every W8A8 handle
+  // (its shapes were checked with the config)
+  h->w8a8 = c.wtype == FM_W_W8A8_E4M3;
+  h->batched = batched_shape_ok(c) && ((c.wtype == FM_W_BF16 && c.max_batch >= 2) || h->w8a8);
   if ((st = pack_weights(h, w)) != FM_OK) return bail(st);
 
   const size_t T = c.chunk_len, A = c.action_dim, d = c.d_model;
