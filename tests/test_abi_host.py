@@ -45,6 +45,11 @@ def test_null_handles_are_safe(lib):
     assert lib.fm_denoise(None, None, 1, 10, None, None) == 1
     assert lib.fm_set_prefix_varlen(None, None, None, 1, None, 0, None) == 1
     assert lib.fm_quantize_act_e4m3(None, None, 1, 256, None, None, None) == 1
+    assert lib.fm_set_prefix_builder(None, None, 64) == 1
+    assert lib.fm_build_prefix(None, None, 1, 1, None) == 1
+    assert lib.fm_get_prefix_kv(None, 0, 0, None, None) == 1
+    assert lib.fm_get_nvfp4_weights(None, 0, 4, None, None, None) == 1
+    assert lib.fm_get_fp8_weights(None, 0, 0, None, None) == 1
 
 
 def _cfg(**kw):
