@@ -588,7 +588,6 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
     }
     PackChunk* dj = static_cast<PackChunk*>(tt);
     int32_t* dr = reinterpret_cast<int32_t*>(static_cast<uint8_t*>(tt) + tj.size() * sizeof(PackChunk));
-    uint16_t** dm = reinterpret_cast<uint16_t**>(d_mats);
     // reuse a small device table for the matrix pointer / width
     void* tm = nullptr;
     e = cudaMalloc(&tm, sizeof(void*) + sizeof(int));
