@@ -597,7 +597,6 @@ fm_status pack_weights(fm_expert* h, const fm_weights* w) {
       e = cudaMemcpy(tm, &mp, sizeof(void*), cudaMemcpyHostToDevice);
       if (e == cudaSuccess) e = cudaMemcpy(static_cast<uint8_t*>(tm) + sizeof(void*), &kk, sizeof(int), cudaMemcpyHostToDevice);
     }
-    (void)dm;
     if (e == cudaSuccess && !w->time_w2) e = cudaErrorInvalidValue;
     if (e == cudaSuccess) e = cudaMemcpy(t2, w->time_w2, (size_t)n_mod * d * 2, cudaMemcpyDefault);
     if (e == cudaSuccess) e = cudaMemcpy(dj, tj.data(), tj.size() * sizeof(PackChunk), cudaMemcpyHostToDevice);
