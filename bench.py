@@ -268,7 +268,10 @@ def run_reference(args, shape):
     r = {"cores": runner.cores, "sample": runner.sample_text(n_sample, el)}
     v = statistics.mean(vals)
     line = {"metric": METRIC, "value": v, "unit": UNIT, "impl": "reference", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1000.0 / v,
+            "steps": args.steps, "warmup": args.warmup,
+            # one bench step is one denoise call of shape.steps Euler steps, as on the GPU arm
+            "ms_per_step": 1000.0 * shape.steps / v, "ms_per_chunk": 1000.0 * shape.steps / v,
+            "ms_per_euler_step": 1000.0 / v,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
             "data": "synthetic", "config": {"workload": args.workload},
             "cpu_baseline": {"value": v, "unit": UNIT, "cores": r["cores"], "kind": "oracle",
@@ -373,6 +376,7 @@ def main():
     line = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
         "warmup": max(args.warmup, 3), "ms_per_step": ms_call, "ms_per_chunk": ms_call,
+        "ms_per_euler_step": ms_call / shape.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "e4m3" if shape.w8a8 else "bf16",
         "data": "synthetic",

@@ -48,7 +48,9 @@ The pages print no formula, so the conventions below are the plainest readings
      linears but no activation quantiser): each input row of the four
      per-layer linears, taken in fp32, is quantised per token with
      r = 448 / amax_row and s = amax_row / 448 (both fp32, 1 for a zero row):
-     codes = E4M3(y r) with the product in fp32, y' = codes s.
+     codes = E4M3(y r) with the product in fp32, y' = codes s (the cast
+     multiplies by the fp32 factor fp8_max / amax, as the public FP8 recipes
+     do, e.g. NVIDIA Transformer Engine's scale = fp8_max / amax).
 
 Every function below is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, hand values, brute force or independent library routines.

@@ -324,9 +324,6 @@ __device__ __forceinline__ void named_bar_sync(uint32_t id, uint32_t nthreads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
-// Two E4M3 codes (low byte = first element) -> two bf16 values (low half =
-// first).  E4M3 -> f16 -> f32 -> bf16 is exact at every step: an E4M3 value
-// has 4 significant bits and a binary exponent in [-9, 8].
 // Four fp32 atomic adds to 16 consecutive bytes of global memory, no return.
 __device__ __forceinline__ void red_add_v4(float* addr, float a, float b, float c, float d) {
   asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
@@ -342,6 +339,9 @@ __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   return r;
 }
 
+// Two E4M3 codes (low byte = first element) -> two bf16 values (low half =
+// first).  E4M3 -> f16 -> f32 -> bf16 is exact at every step: an E4M3 value
+// has 4 significant bits and a binary exponent in [-9, 8].
 __device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint16_t v) {
   uint32_t h2, r;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(v));
