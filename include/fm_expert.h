@@ -299,13 +299,17 @@ fm_status fm_get_geometry(const fm_expert *h, int *cluster_size, int *n_clusters
  * only buffers it owns.  The pages have no counterpart of this entry point;
  * it allocates nothing.
  *   w1: device bf16 bits [d_model, 256]; w2: device bf16 bits [n_mod, d_model]
- *   (row-major, as in fm_weights); m_out: device fp32 [steps, n_mod].
+ *   (row-major, as in fm_weights); m_out: device fp32 [steps, n_mod].  All three
+ *   must be 4-byte aligned.
  *   Limits: 1 <= steps <= 64, 64 <= d_model <= 1024 (a multiple of 64).  Larger
- *   sizes return FM_ERR_INVALID_ARG and fm_last_error(NULL) says why.
+ *   sizes and misaligned pointers return FM_ERR_INVALID_ARG and
+ *   fm_last_error(NULL) says why.
  * Its only intermediate, the bf16 hidden activations (64 x 1024 at most, 128
  * KB), lives in a device array inside the library that every GPU using the
- * library holds until the process exits.  The first call on a device looks up
- * that array's address; make that first call before any stream capture.  All
+ * library holds until the process exits.  The first call on a device (and the
+ * first after cudaDeviceReset on it) looks up that array's address; make that
+ * first call before any stream capture.  Its kernels use no local-memory
+ * stack.  All
  * calls share the array and each overwrites the part it reads, so nothing
  * depends on a previous call; calls that overlap on the GPU (two streams)
  * race on it.  Stream-ordered; does not synchronise. */

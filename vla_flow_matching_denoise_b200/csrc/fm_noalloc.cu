@@ -18,6 +18,7 @@
 // bf16 rounding boundary may round the other way).
 #include <cuda_runtime.h>
 
+#include <cstdint>
 #include <cstdio>
 #include <mutex>
 
@@ -29,7 +30,6 @@ namespace {
 constexpr int kNaMaxSteps = 64;
 constexpr int kNaMaxD = 1024;
 constexpr int kNaTimeDim = 256;
-constexpr double kNaTwoPi = 6.283185307179586476925286766559;
 
 // Shared by every call on a device and kept until the process exits: the bf16
 // hidden activations [kNaMaxSteps][kNaMaxD] (128 KB).  Calls that overlap on
@@ -39,8 +39,11 @@ static __device__ __align__(256) unsigned short g_noalloc_h1[kNaMaxSteps * kNaMa
 constexpr int kNaMaxDevices = 64;
 std::mutex g_na_mu;
 void* g_na_ptr[kNaMaxDevices] = {};
+unsigned long long g_na_ctx[kNaMaxDevices] = {};   // context id the address belongs to
 
-// Hidden activations: one block per step; fp64 sinusoid, fp32 sums.
+// Hidden activations: one block per step; fp64 sinusoid, fp32 sums.  Neither
+// kernel of this file uses a local-memory stack (ptxas: 0 bytes), so a launch
+// never needs the driver to enlarge the context's local memory.
 __global__ void noalloc_embed_kernel(const unsigned short* __restrict__ w1, int d, int steps,
                                      unsigned short* __restrict__ h1) {
   __shared__ float e[kNaTimeDim];
@@ -49,9 +52,12 @@ __global__ void noalloc_embed_kernel(const unsigned short* __restrict__ w1, int 
   const int half = kNaTimeDim / 2;
   for (int j = threadIdx.x; j < half; j += blockDim.x) {
     const double period = 4e-3 * pow(4.0 / 4e-3, (double)j / (double)(half - 1));
-    const double ang = kNaTwoPi * t / period;
-    e[j] = (float)sin(ang);
-    e[j + half] = (float)cos(ang);
+    // sin / cos of 2 pi t / period, with the factor pi applied inside the
+    // argument reduction (sincospi: no stack frame)
+    double sv, cv;
+    sincospi(2.0 * t / period, &sv, &cv);
+    e[j] = (float)sv;
+    e[j + half] = (float)cv;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < d; i += blockDim.x) {
@@ -71,7 +77,10 @@ __global__ void noalloc_embed_kernel(const unsigned short* __restrict__ w1, int 
 }
 
 // m[k][j] = sum_i h1[k][i] W2[j][i]: one warp per output row j, the steps'
-// hidden rows (bf16) in shared memory.
+// hidden rows (bf16) in shared memory.  Steps go in blocks of kNaStepBlock
+// with the block's accumulators in registers (compile-time indices, no
+// local-memory stack); the weight row is read once per block.
+constexpr int kNaStepBlock = 16;
 __global__ void noalloc_mod_kernel(const unsigned short* __restrict__ w2, const unsigned short* __restrict__ h1,
                                    int d, int steps, int n_mod, float* __restrict__ m) {
   extern __shared__ unsigned short hs[];   // [steps][d]
@@ -81,30 +90,68 @@ __global__ void noalloc_mod_kernel(const unsigned short* __restrict__ w2, const 
   const int warps = blockDim.x >> 5;
   for (int j = blockIdx.x * warps + (threadIdx.x >> 5); j < n_mod; j += gridDim.x * warps) {
     const unsigned short* w = w2 + (size_t)j * d;
-    float acc[kNaMaxSteps];
-    for (int k = 0; k < steps; ++k) acc[k] = 0.f;
-    for (int c = lane * 2; c < d; c += 64) {
-      const unsigned int pair = *reinterpret_cast<const unsigned int*>(w + c);
-      const float w0 = __uint_as_float(pair << 16), w1v = __uint_as_float(pair & 0xFFFF0000u);
-      for (int k = 0; k < steps; ++k) {
-        const unsigned int hp = *reinterpret_cast<const unsigned int*>(hs + k * d + c);
-        acc[k] = fmaf(__uint_as_float(hp << 16), w0, fmaf(__uint_as_float(hp & 0xFFFF0000u), w1v, acc[k]));
+    for (int k0 = 0; k0 < steps; k0 += kNaStepBlock) {
+      float acc[kNaStepBlock];
+#pragma unroll
+      for (int kk = 0; kk < kNaStepBlock; ++kk) acc[kk] = 0.f;
+      for (int c = lane * 2; c < d; c += 64) {
+        const unsigned int pair = *reinterpret_cast<const unsigned int*>(w + c);
+        const float w0 = __uint_as_float(pair << 16), w1v = __uint_as_float(pair & 0xFFFF0000u);
+#pragma unroll
+        for (int kk = 0; kk < kNaStepBlock; ++kk) {
+          if (k0 + kk < steps) {
+            const unsigned int hp = *reinterpret_cast<const unsigned int*>(hs + (k0 + kk) * d + c);
+            acc[kk] = fmaf(__uint_as_float(hp << 16), w0, fmaf(__uint_as_float(hp & 0xFFFF0000u), w1v, acc[kk]));
+          }
+        }
       }
-    }
-    for (int k = 0; k < steps; ++k) {
-      float v = acc[k];
-      for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) m[(size_t)k * n_mod + j] = v;
+#pragma unroll
+      for (int kk = 0; kk < kNaStepBlock; ++kk) {
+        float v = acc[kk];
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0 && k0 + kk < steps) m[(size_t)(k0 + kk) * n_mod + j] = v;
+      }
     }
   }
 }
 
-// Device address of the scratch array on the current device, looked up once
-// per device: the first call on a device does this set-up, so make that call
-// before any stream capture.  Host code must not hand g_noalloc_h1 itself to a
-// kernel: in host code that name is a host-side stand-in, not a device address.
-// Nothing in the array has to start at zero: each call writes every entry it
-// reads before reading it.
+// Id of the current device context (0 if it cannot be read).  A context
+// destroyed by cudaDeviceReset and created again gets a new id, and the
+// array's address has to be looked up again in it.
+unsigned long long current_context_id() {
+  typedef int (*GetCurrent)(void**);
+  typedef int (*GetId)(void*, unsigned long long*);
+  static GetCurrent get_current = nullptr;
+  static GetId get_id = nullptr;
+  static bool looked_up = false;
+  if (!looked_up) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_current = reinterpret_cast<GetCurrent>(f);
+    f = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<GetId>(f);
+    cudaGetLastError();
+    looked_up = true;
+  }
+  void* ctx = nullptr;
+  unsigned long long id = 0;
+  if (get_current == nullptr || get_id == nullptr || get_current(&ctx) != 0 || ctx == nullptr ||
+      get_id(ctx, &id) != 0)
+    return 0;
+  return id;
+}
+
+// Device address of the scratch array on the current device.  Set-up runs on
+// the first call on a device (and again on the first call after that device's
+// context was reset): it asks the runtime for the array's address with the
+// device current, so make that call before any stream capture.  Host code must
+// not hand g_noalloc_h1 itself to a kernel: in host code that name is a
+// host-side stand-in, not a device address.  Nothing in the array has to start
+// at zero: each call writes every entry it reads before reading it.
 fm_status scratch_on_current_device(void** out, const char** why) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kNaMaxDevices) {
@@ -113,7 +160,8 @@ fm_status scratch_on_current_device(void** out, const char** why) {
     return FM_ERR_CUDA;
   }
   std::lock_guard<std::mutex> lock(g_na_mu);
-  if (g_na_ptr[dev] == nullptr) {
+  const unsigned long long ctx = current_context_id();
+  if (g_na_ptr[dev] == nullptr || ctx == 0 || ctx != g_na_ctx[dev]) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_h1);
     if (e != cudaSuccess || p == nullptr) {
@@ -122,6 +170,8 @@ fm_status scratch_on_current_device(void** out, const char** why) {
       return FM_ERR_CUDA;
     }
     g_na_ptr[dev] = p;
+    // the look-up made the device's context current if no call had yet
+    g_na_ctx[dev] = ctx != 0 ? ctx : current_context_id();
   }
   *out = g_na_ptr[dev];
   return FM_OK;
@@ -137,6 +187,10 @@ fm_status fm_time_modulation_noalloc(const uint16_t* w1, const uint16_t* w2, int
   fm::set_thread_error("");
   if (w1 == nullptr || w2 == nullptr || m_out == nullptr) {
     fm::set_thread_error("fm_time_modulation_noalloc: w1, w2 and m_out must be device pointers, not NULL");
+    return FM_ERR_INVALID_ARG;
+  }
+  if ((reinterpret_cast<uintptr_t>(w1) | reinterpret_cast<uintptr_t>(w2) | reinterpret_cast<uintptr_t>(m_out)) & 3u) {
+    fm::set_thread_error("fm_time_modulation_noalloc: w1, w2 and m_out must be 4-byte aligned");
     return FM_ERR_INVALID_ARG;
   }
   if (steps < 1 || steps > kNaMaxSteps || d_model < 64 || d_model > kNaMaxD || d_model % 64 != 0 || n_mod < 1) {
