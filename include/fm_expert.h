@@ -286,8 +286,35 @@ fm_status fm_profile_denoise(fm_expert *h, int batch, int steps, int iters, floa
  * steps*L*(chunks per CTA per layer, at most 32). */
 fm_status fm_profile_phases(fm_expert *h, int steps, uint64_t *out, size_t *n, void *stream);
 
+/* Test hook (per-kernel parity of the batched path, "LingBot-VLA v2
+ * Examples": intermediate-tensor parity): one velocity evaluation of `batch`
+ * requests (as fm_velocity) on the batched path, stopping after each kernel
+ * to copy its output to the host buffer `trace` of fm_trace_batched_bytes
+ * bytes: per layer, rows m = b T + t (M = batch T rows), fp32
+ *   h_in [M][d], y_a [M][d], q [M][Hq hd], k [M][Hkv hd], v [M][Hkv hd],
+ *   o [M][Hq hd], h_mid [M][d], y_f [M][d], u [M][F], h_out [M][d]
+ * then the velocity [M][A].  y_a and y_f are the normalised GEMM inputs as the
+ * GEMMs read them (on a W8A8 handle: codes x row scale); q, k are after RoPE;
+ * o and u are the bf16 outputs of attention and SwiGLU.  FM_ERR_UNSUPPORTED
+ * when `batch` runs on the one-request kernel.  Synchronises (slow). */
+size_t fm_trace_batched_bytes(const fm_expert *h, int batch);
+fm_status fm_trace_batched(fm_expert *h, const float *x, int batch, int step_index, int steps,
+                           float *trace, void *stream);
+
 /* Wait for `stream`, then report (and clear) any device-side timeout. */
 fm_status fm_sync(fm_expert *h, void *stream);
+
+/* Test hook for failure detection (the pages' release checks cover fault and
+ * shutdown handling; this is the device-side half).  While `on` is non-zero,
+ * the one-request loop kernel of this handle expects one writer more than
+ * exists at its QKV -> attention hand-off, so that wait can never complete,
+ * and every wait of the loop kernel gives up after `spin_cycles` SM clock
+ * cycles (0: the default of about 2 s).  The launch then ends early with the
+ * handle's error word set, and the next synchronising call returns
+ * FM_ERR_TIMEOUT; the device context stays usable.  Off by default.  Blocks
+ * until the device is idle and drops the handle's captured graphs, so later
+ * calls see the setting.  FM_ERR_INVALID_ARG for a negative spin_cycles. */
+fm_status fm_test_stall(fm_expert *h, int on, long long spin_cycles);
 
 /* Launch geometry the handle chose: CTAs per cluster, clusters, CTAs. */
 fm_status fm_get_geometry(const fm_expert *h, int *cluster_size, int *n_clusters,

@@ -29,7 +29,8 @@ STATUS = {0: "FM_OK", 1: "FM_ERR_INVALID_ARG", 2: "FM_ERR_NOT_READY", 3: "FM_ERR
 # Every symbol include/fm_expert.h declares.
 EXPORTS = ("fm_expert_create", "fm_set_prefix", "fm_set_prefix_varlen", "fm_set_prefix_builder",
            "fm_build_prefix", "fm_get_prefix_kv", "fm_get_nvfp4_weights", "fm_quantize_act_e4m3", "fm_denoise", "fm_velocity", "fm_time_modulation",
-           "fm_trace_bytes", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
+           "fm_trace_bytes", "fm_trace_velocity", "fm_trace_batched_bytes", "fm_trace_batched",
+           "fm_get_fp8_weights", "fm_sync", "fm_test_stall",
            "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
            "fm_expert_destroy", "fm_last_error", "fm_status_string",
            "fm_abi_version")
@@ -84,8 +85,12 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_trace_bytes.argtypes = [vp]
     lib.fm_trace_bytes.restype = sz
     lib.fm_trace_velocity.argtypes = [vp, vp, ip, ip, vp, vp]
+    lib.fm_trace_batched_bytes.argtypes = [vp, ip]
+    lib.fm_trace_batched_bytes.restype = sz
+    lib.fm_trace_batched.argtypes = [vp, vp, ip, ip, ip, vp, vp]
     lib.fm_get_fp8_weights.argtypes = [vp, ip, ip, vp, vp]
     lib.fm_sync.argtypes = [vp, vp]
+    lib.fm_test_stall.argtypes = [vp, ip, ctypes.c_longlong]
     lib.fm_profile_denoise.argtypes = [vp, ip, ip, ip, vp, vp]
     lib.fm_profile_phases.argtypes = [vp, ip, vp, ctypes.POINTER(sz), vp]
     lib.fm_time_modulation_noalloc.argtypes = [vp, vp, ip, ip, ip, vp, vp]
@@ -105,7 +110,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.fm_abi_version.restype = ip
     for name in ("fm_expert_create", "fm_set_prefix", "fm_denoise", "fm_velocity",
                  "fm_time_modulation", "fm_trace_velocity", "fm_get_fp8_weights", "fm_sync",
-                 "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
+                 "fm_test_stall", "fm_trace_batched", "fm_get_geometry", "fm_profile_denoise", "fm_profile_phases", "fm_time_modulation_noalloc",
                  "fm_set_prefix_varlen", "fm_set_prefix_builder", "fm_build_prefix", "fm_get_prefix_kv",
                  "fm_get_nvfp4_weights", "fm_quantize_act_e4m3"):
         getattr(lib, name).restype = ip
@@ -278,6 +283,29 @@ class Expert:
         out.append({"v": buf[o:o + T * s.action_dim].reshape(T, s.action_dim)})
         return out
 
+    def trace_batched(self, x: np.ndarray, step_index: int, steps: int, stream=None) -> List[Dict]:
+        """Per-layer intermediates of one batched velocity evaluation (see
+        fm_trace_batched); x: [B, T, A].  Arrays are [B * T, width]."""
+        s = self.shape
+        x = np.ascontiguousarray(x, dtype=np.float32)
+        B = x.shape[0]
+        n = self.lib.fm_trace_batched_bytes(self.h, B) // 4
+        buf = np.empty(n, dtype=np.float32)
+        self._check("fm_trace_batched", self.lib.fm_trace_batched(self.h, _ptr(x), B, step_index, steps,
+                                                                   _ptr(buf), _stream(stream)))
+        M, d, F = B * s.chunk_len, s.d_model, s.d_ff
+        qn, kn = s.n_q_heads * s.head_dim, s.n_kv_heads * s.head_dim
+        out, o = [], 0
+        for _ in range(s.n_layers):
+            rec = {}
+            for name, w in (("h_in", d), ("y_a", d), ("q", qn), ("k", kn), ("v", kn), ("o", qn),
+                            ("h_mid", d), ("y_f", d), ("u", F), ("h_out", d)):
+                rec[name] = buf[o:o + M * w].reshape(M, w)
+                o += M * w
+            out.append(rec)
+        out.append({"v": buf[o:o + M * s.action_dim].reshape(M, s.action_dim)})
+        return out
+
     def get_fp8_weights(self, layer: int, which: int, rows: int, cols: int):
         codes = np.empty((rows, cols), dtype=np.uint8)
         scale = np.empty(rows, dtype=np.float32)
@@ -332,3 +360,7 @@ class Expert:
 
     def sync(self, stream=None):
         self._check("fm_sync", self.lib.fm_sync(self.h, _stream(stream)))
+
+    def test_stall(self, on: bool, spin_cycles: int = 0):
+        """Test hook: make the loop kernel's QKV hand-off unreachable (see fm_test_stall)."""
+        self._check("fm_test_stall", self.lib.fm_test_stall(self.h, 1 if on else 0, int(spin_cycles)))

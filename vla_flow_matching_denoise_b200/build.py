@@ -16,7 +16,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfm_expert.so")
-SOURCES = ["fm_api.cu", "fm_prep.cu", "fm_time.cu", "fm_step.cu", "fm_batch.cu", "fm_noalloc.cu"]
+SOURCES = ["fm_api.cu", "fm_prep.cu", "fm_time.cu", "fm_step.cu", "fm_batch.cu", "fm_attn.cu", "fm_noalloc.cu"]
 HEADERS = ["fm_internal.h", "fm_batch.h", "fm_launch.h", "fm_ptx.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 

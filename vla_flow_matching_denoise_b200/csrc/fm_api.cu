@@ -8,6 +8,7 @@
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
+#include <functional>
 #include <map>
 #include <string>
 #include <utility>
@@ -119,11 +120,16 @@ struct fm_expert {
   uint16_t* qbuf = nullptr;
   uint16_t* kcache = nullptr;
   uint16_t* vcache = nullptr;
-  uint32_t* bar_count = nullptr;
+  uint32_t* flags = nullptr;       // hand-off counters of the loop kernel
   uint32_t* err_word = nullptr;
   int S_max = 0;
   int prefix_batch = 0;   // batch of the last fm_set_prefix (0 = none)
   std::vector<int> prefix_lens;   // per request, host copy of P_dev
+  // batched tensor-core attention: TMA views of the q buffer and the K/V caches
+  CUtensorMap tm_q{}, tm_k{}, tm_v{};
+  bool tm_ok = false;
+  int test_stall = 0;              // fm_test_stall: make the loop kernel's QKV hand-off unreachable
+  long long test_spin = 0;         // fm_test_stall: wait budget in cycles (0: the default)
   std::map<std::pair<int, int>, cudaGraphExec_t> graphs;
   std::map<std::pair<int, int>, cudaGraph_t> graph_defs;
 };
@@ -170,6 +176,34 @@ fm_status dalloc(fm_expert* h, T** out, size_t bytes) {
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 
+// `nseg` segments of `rows` rows of hd bf16 values as a 4-D TMA view
+// (64 elements, hd/64 halves, rows, segments) with a (64, 1, 128, 1) box: one
+// copy moves one 64-element half of 128 consecutive rows.  The driver's
+// encoder is reached through the runtime (no link-time libcuda dependency).
+bool encode_rows_map(CUtensorMap* m, void* base, int hd, int rows, int nseg) {
+  typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                               const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                               CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+  static EncodeFn fn = nullptr;
+  if (fn == nullptr) {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess || f == nullptr) {
+      cudaGetLastError();
+      return false;
+    }
+    fn = reinterpret_cast<EncodeFn>(f);
+  }
+  const cuuint64_t dims[4] = {64, (cuuint64_t)(hd / 64), (cuuint64_t)rows, (cuuint64_t)nseg};
+  const cuuint64_t strides[3] = {128, (cuuint64_t)hd * 2, (cuuint64_t)rows * hd * 2};
+  const cuuint32_t box[4] = {64, 1, 128, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+         CUDA_SUCCESS;
+}
+
 // Plans one linear over `nc` clusters (see GemmPlan).  Channels are dealt to
 // clusters in units of NS x 16 so that per-cluster work differs by at most one
 // unit; the K split starts at `max_ks` and is halved (more n-groups per
@@ -181,7 +215,8 @@ bool plan_gemm(GemmPlan& g, int N, int K, int nc, int max_ks, bool pair_cols) {
   for (int ks = max_ks; ks >= 1; ks /= 2) {
     if ((K / 64) % ks != 0) continue;
     const int NS = kClusterSize / ks;
-    const int unit = std::max(16, ks * (pair_cols ? 4 : 2));
+    // owners hold a multiple of 4 columns (16-byte partial pushes)
+    const int unit = std::max(16, ks * 4);
     const int cunit = NS * unit;
     const int U = (N + cunit - 1) / cunit;
     const int q = U / nc, r = U % nc;
@@ -247,7 +282,9 @@ fm_status build_plan(fm_expert* h) {
   const fm_config& c = h->cfg;
   const int nc = h->n_clusters;
   const int qkv = (c.n_q_heads + 2 * c.n_kv_heads) * c.head_dim;
-  if (!plan_gemm(h->plan[G_QKV], qkv, c.d_model, nc, 8, false) ||
+  // QKV splits K at most 4 ways: its N per CTA then stays <= 128, where an
+  // MMA costs the same as at half the width, and the split-K exchange halves
+  if (!plan_gemm(h->plan[G_QKV], qkv, c.d_model, nc, 4, false) ||
       !plan_gemm(h->plan[G_O], c.d_model, c.n_q_heads * c.head_dim, nc, 8, false) ||
       !plan_gemm(h->plan[G_GU], 2 * c.d_ff, c.d_model, nc, 8, true) ||
       !plan_gemm(h->plan[G_DOWN], c.d_model, c.d_ff, nc, 8, false))
@@ -735,7 +772,7 @@ StepParams base_params(const fm_expert* h) {
   p.qbuf = h->qbuf;
   p.kcache = h->kcache;
   p.vcache = h->vcache;
-  p.bar_count = h->bar_count;
+  p.flags = h->flags;
   p.err = h->err_word;
   for (int g = 0; g < 4; ++g)
     p.wfmt[g] = c.wtype == FM_W_BF16 ? 0 : (c.wtype == FM_W_FP8_NVFP4_GU && g == G_GU) ? 2 : 1;
@@ -750,7 +787,8 @@ StepParams base_params(const fm_expert* h) {
   p.do_outproj = 1;
   p.update_x = 1;
   p.dt = 0.f;
-  p.spin_budget = 4000000000LL;   // ~2 s at 2 GHz
+  p.spin_budget = h->test_spin > 0 ? h->test_spin : 4000000000LL;   // ~2 s at 2 GHz
+  p.stall_test = h->test_stall;
   p.tlog = nullptr;
   p.tlog_stride = 0;
   p.tlog_mma_off = 0;
@@ -776,8 +814,15 @@ TimeParams time_params(const fm_expert* h, int steps) {
 // Batched path: Euler steps step0 .. step1 - 1 of a `steps`-step schedule for
 // `batch` requests together (x in h->x, velocities to h->vbuf; x updated when
 // `update`).  The modulation rows must already be in h->mod.
+// `hook` (test hook, null on the product path) runs on the host after each
+// stage: (l, 0) layer l's attention norm is in bz_a and its input in bh;
+// (l, 1) q and the chunk's K/V rows; (l, 2) attention output; (l, 3) h after
+// o_proj; (l, 4) FFN norm; (l, 5) SwiGLU output; (l, 6) h after down;
+// (L, 7) the velocity.
+using BatchHook = std::function<cudaError_t(int, int)>;
+
 cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int steps, bool update,
-                            cudaStream_t st) {
+                            cudaStream_t st, const BatchHook* hook = nullptr) {
   const fm_config& c = h->cfg;
   const int T = c.chunk_len, d = c.d_model, M = batch * T, L = c.n_layers;
   const int qn = c.n_q_heads * c.head_dim, kn = c.n_kv_heads * c.head_dim, F = c.d_ff;
@@ -825,6 +870,9 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
   BQuantParams qo{h->bo, h->bo8, sa_o, M, qn};
   BQuantParams qu{h->bu, h->bu8, sa_u, M, F};
   BAttnParams a{};
+  a.tm_q = h->tm_q;
+  a.tm_k = h->tm_k;
+  a.tm_v = h->tm_v;
   a.qbuf = h->bq;
   a.o_act = h->bo;
   a.P_dev = h->P_dev;
@@ -847,7 +895,11 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
     r.zs = sa_za;
     e = launch_binproj(r, st);
     if (e == cudaSuccess) e = launch_bresnorm(r, st);   // layer 0's attention norm
+    auto stage = [&](int l, int k) {
+      if (hook != nullptr && e == cudaSuccess) e = (*hook)(l, k);
+    };
     for (int l = 0; l < L && e == cudaSuccess; ++l) {
+      stage(l, 0);
       const float* lm = mrow + (size_t)6 * l * d;
       const uint8_t* wl = h->barena + (size_t)l * h->blayer_bytes;
       const float* bws = h->w8a8 ? h->bwscale + (size_t)l * h->bw_stride : nullptr;
@@ -862,10 +914,13 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       g.kc = h->kcache + l * lay;
       g.vc = h->vcache + l * lay;
       e = launch_bgemm(g, BE_QKV, h->n_sms, st);
+      stage(l, 1);
       a.kc = h->kcache + l * lay;
       a.vc = h->vcache + l * lay;
-      if (e == cudaSuccess) e = launch_battn(a, st);
+      a.seg_base = l * c.max_batch * c.n_kv_heads;
+      if (e == cudaSuccess) e = h->tm_ok ? launch_battn_tc(a, st) : launch_battn(a, st);
       if (e == cudaSuccess && h->w8a8) e = launch_browquant(qo, st);
+      stage(l, 2);
       // o_proj + gated residual, then the FFN norm
       g.A = h->w8a8 ? h->bo8 : reinterpret_cast<const uint8_t*>(h->bo);
       g.a_scale = sa_o;
@@ -875,11 +930,13 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       g.N = d;
       g.gate = lm + 2 * d;
       if (e == cudaSuccess) e = launch_bgemm(g, BE_RESID, h->n_sms, st);
+      stage(l, 3);
       r.s = lm + 3 * d;
       r.b = lm + 4 * d;
       r.z = h->bz_f;
       r.zs = sa_zf;
       if (e == cudaSuccess) e = launch_bresnorm(r, st);
+      stage(l, 4);
       // gate_up + SwiGLU, down + gated residual
       g.A = reinterpret_cast<const uint8_t*>(h->bz_f);
       g.a_scale = sa_zf;
@@ -889,6 +946,7 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       g.N = 2 * F;
       if (e == cudaSuccess) e = launch_bgemm(g, BE_SWIGLU, h->n_sms, st);
       if (e == cudaSuccess && h->w8a8) e = launch_browquant(qu, st);
+      stage(l, 5);
       g.A = h->w8a8 ? h->bu8 : reinterpret_cast<const uint8_t*>(h->bu);
       g.a_scale = sa_u;
       g.w_scale = wsc(G_DOWN);
@@ -897,6 +955,7 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
       g.N = d;
       g.gate = lm + 5 * d;
       if (e == cudaSuccess) e = launch_bgemm(g, BE_RESID, h->n_sms, st);
+      stage(l, 6);
       // the next layer's attention norm (none after the last layer: the
       // out-proj kernel applies the final norm)
       r.s = lm + 6 * d;
@@ -908,6 +967,7 @@ cudaError_t enqueue_batched(fm_expert* h, int batch, int step0, int step1, int s
     r.s = mrow + (size_t)6 * L * d;
     r.b = r.s + d;
     if (e == cudaSuccess) e = launch_boutproj(r, st);
+    stage(L, 7);
   }
   return e;
 }
@@ -923,7 +983,7 @@ cudaError_t enqueue_denoise(fm_expert* h, int batch, int steps, cudaStream_t st)
     if (e != cudaSuccess) return e;
     return enqueue_batched(h, batch, 0, steps, steps, true, st);
   }
-  cudaError_t e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
+  cudaError_t e = cudaMemsetAsync(h->flags, 0, kFlagBytes, st);
   if (e != cudaSuccess) return e;
   e = launch_time(time_params(h, steps), h->n_sms, st);
   if (e != cudaSuccess) return e;
@@ -937,7 +997,7 @@ cudaError_t enqueue_denoise(fm_expert* h, int batch, int steps, cudaStream_t st)
     p.step1 = steps;
     p.dt = -1.0f / (float)steps;
     if (b > 0) {
-      e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
+      e = cudaMemsetAsync(h->flags, 0, kFlagBytes, st);
       if (e != cudaSuccess) return e;
     }
     e = launch_step(p, st);
@@ -1050,17 +1110,17 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
   ALLOC_OR_BAIL(h->vbuf, B * T * A * 4);
   ALLOC_OR_BAIL(h->h_a, T * d * 4);
   ALLOC_OR_BAIL(h->h_b, T * d * 4);
-  ALLOC_OR_BAIL(h->z_a, (size_t)kRows * d * 2);
-  ALLOC_OR_BAIL(h->z_f, (size_t)kRows * d * 2);
-  ALLOC_OR_BAIL(h->o_act, (size_t)kRows * c.n_q_heads * c.head_dim * 2);
-  ALLOC_OR_BAIL(h->u_act, (size_t)kRows * c.d_ff * 2);
+  ALLOC_OR_BAIL(h->z_a, (size_t)2 * kRows * d * 2);
+  ALLOC_OR_BAIL(h->z_f, (size_t)2 * kRows * d * 2);
+  ALLOC_OR_BAIL(h->o_act, (size_t)2 * kRows * c.n_q_heads * c.head_dim * 2);
+  ALLOC_OR_BAIL(h->u_act, (size_t)2 * kRows * c.d_ff * 2);
   ALLOC_OR_BAIL(h->sumsq_a, (size_t)h->n_ctas * kRows * 4);
   ALLOC_OR_BAIL(h->sumsq_f, (size_t)h->n_ctas * kRows * 4);
   ALLOC_OR_BAIL(h->qbuf, (size_t)c.n_kv_heads * h->q_rows * c.head_dim * 2);
   const size_t kv = (size_t)c.n_layers * B * c.n_kv_heads * h->S_max * c.head_dim * 2;
   ALLOC_OR_BAIL(h->kcache, kv);
   ALLOC_OR_BAIL(h->vcache, kv);
-  ALLOC_OR_BAIL(h->bar_count, (size_t)(h->n_ctas + 4) * 4);
+  ALLOC_OR_BAIL(h->flags, kFlagBytes);
   ALLOC_OR_BAIL(h->err_word, 4);
   if (h->batched) {
     h->Mp = (int)((B * T + kBM - 1) / kBM * kBM);
@@ -1071,6 +1131,10 @@ fm_status fm_expert_create(const fm_config* cfg, const fm_weights* w, int device
     ALLOC_OR_BAIL(h->bu, Mp * c.d_ff * 2);
     ALLOC_OR_BAIL(h->bh, Mp * d * 4);
     ALLOC_OR_BAIL(h->bq, B * c.n_kv_heads * h->q_rows * c.head_dim * 2);
+    h->tm_ok = battn_tc_supported(h->S_max, c.head_dim) &&
+               encode_rows_map(&h->tm_q, h->bq, c.head_dim, h->q_rows, (int)(B * c.n_kv_heads)) &&
+               encode_rows_map(&h->tm_k, h->kcache, c.head_dim, h->S_max, (int)(c.n_layers * B * c.n_kv_heads)) &&
+               encode_rows_map(&h->tm_v, h->vcache, c.head_dim, h->S_max, (int)(c.n_layers * B * c.n_kv_heads));
     if (h->w8a8) {
       ALLOC_OR_BAIL(h->bo8, Mp * c.n_q_heads * c.head_dim);
       ALLOC_OR_BAIL(h->bu8, Mp * c.d_ff);
@@ -1271,7 +1335,7 @@ fm_status fm_velocity(fm_expert* h, const float* x, int batch, int step_index, i
       p.step0 = step_index;
       p.step1 = step_index + 1;
       p.update_x = 0;
-      CK(cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st));
+      CK(cudaMemsetAsync(h->flags, 0, kFlagBytes, st));
       CK(launch_step(p, st));
     }
   }
@@ -1335,7 +1399,7 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
     p.do_inproj = inproj;
     p.do_outproj = outproj;
     p.update_x = 0;
-    CK(cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st));
+    CK(cudaMemsetAsync(h->flags, 0, kFlagBytes, st));
     CK(launch_step(p, st));
     CK(cudaStreamSynchronize(st));
     return check_err_word(h);
@@ -1367,13 +1431,13 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
       }
       out += (size_t)T * kn;
     }
-    CK(cudaMemcpy(oh.data(), h->o_act, oh.size() * 2, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(oh.data(), h->o_act + (size_t)(l & 1) * oh.size(), oh.size() * 2, cudaMemcpyDeviceToHost));
     for (int t = 0; t < T; ++t)
       for (int n = 0; n < qn; ++n) out[(size_t)t * qn + n] = act64_get(oh, t, n);
     out += (size_t)T * qn;
     CK(cudaMemcpy(out, h->h_b, (size_t)T * d * 4, cudaMemcpyDeviceToHost));   // h_mid
     out += (size_t)T * d;
-    CK(cudaMemcpy(uh.data(), h->u_act, uh.size() * 2, cudaMemcpyDeviceToHost));
+    CK(cudaMemcpy(uh.data(), h->u_act + (size_t)(l & 1) * uh.size(), uh.size() * 2, cudaMemcpyDeviceToHost));
     for (int t = 0; t < T; ++t)
       for (int n = 0; n < F; ++n) out[(size_t)t * F + n] = act64_get(uh, t, n);
     out += (size_t)T * F;
@@ -1383,6 +1447,136 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
   if ((s = run(c.n_layers, c.n_layers, 0, 1)) != FM_OK) return s;
   CK(cudaMemcpy(out, h->vbuf, (size_t)T * c.action_dim * 4, cudaMemcpyDeviceToHost));
   return FM_OK;
+}
+
+size_t fm_trace_batched_bytes(const fm_expert* h, int batch) {
+  if (!h || batch < 1) return 0;
+  const fm_config& c = h->cfg;
+  const size_t M = (size_t)batch * c.chunk_len, d = c.d_model, qn = (size_t)c.n_q_heads * c.head_dim,
+               kn = (size_t)c.n_kv_heads * c.head_dim;
+  return 4 * (c.n_layers * M * (5 * d + 2 * qn + 2 * kn + c.d_ff) + M * c.action_dim);
+}
+
+namespace {
+// Element (m, k) of a host copy of an ACT128 matrix with K columns.
+float act128_get(const std::vector<uint16_t>& a, int K, int m, int k) {
+  const size_t blk = ((size_t)(m >> 7) * (K >> 6) + (k >> 6)) * (kBM * 64);
+  const int r = m & 127;
+  return bf2f(a[blk + (size_t)r * 64 + ((((k & 63) >> 3) ^ (r & 7)) << 3) + (k & 7)]);
+}
+// Value (code x row scale) of element (m, k) of a host copy of an ACT8 matrix.
+float act8_get(const std::vector<uint8_t>& a, const std::vector<float>& sa, int K, int m, int k) {
+  const size_t blk = ((size_t)(m >> 7) * (K >> 7) + (k >> 7)) * (kBM * 128);
+  const int r = m & 127;
+  const uint8_t q = a[blk + (size_t)r * 128 + ((((k & 127) >> 4) ^ (r & 7)) << 4) + (k & 15)];
+  // E4M3: sign, 4 exponent bits (bias 7), 3 mantissa bits; 0x7F / 0xFF are NaN
+  const int e = (q >> 3) & 15, mt = q & 7;
+  float v = (q & 0x7F) == 0x7F ? NAN : e == 0 ? std::ldexp((float)mt, -9) : std::ldexp(1.0f + mt / 8.0f, e - 7);
+  return ((q & 0x80) ? -v : v) * sa[m];
+}
+}  // namespace
+
+fm_status fm_trace_batched(fm_expert* h, const float* x, int batch, int step_index, int steps, float* trace,
+                           void* stream) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  if (!trace) return set_err(h, FM_ERR_INVALID_ARG, "trace is NULL");
+  if (!use_batched(h, batch))
+    return set_err(h, FM_ERR_UNSUPPORTED, "batch %d does not run on the batched path of this handle", batch);
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  fm_status s = velocity_common(h, x, batch, step_index, steps, st);
+  if (s != FM_OK) return s;
+  const fm_config& c = h->cfg;
+  const int T = c.chunk_len, d = c.d_model, qn = c.n_q_heads * c.head_dim, kn = c.n_kv_heads * c.head_dim,
+            F = c.d_ff, hd = c.head_dim, M = batch * T, L = c.n_layers, G = c.n_q_heads / c.n_kv_heads;
+  const size_t Mp = (size_t)h->Mp;
+  const size_t lay = (size_t)c.max_batch * c.n_kv_heads * h->S_max * hd;
+  std::vector<uint16_t> a16;
+  std::vector<uint8_t> a8;
+  std::vector<float> sa, hbuf((size_t)M * d);
+  std::vector<uint16_t> qh((size_t)batch * c.n_kv_heads * h->q_rows * hd), kvh;
+  float* out = trace;
+  // copies matrix `src` (ACT128 bf16, or ACT8 codes with row scales `scale`
+  // on a W8A8 handle) of K columns into out[M][K]
+  auto put_act = [&](const void* src, const float* scale, int K) -> cudaError_t {
+    cudaError_t e;
+    if (scale != nullptr) {
+      a8.resize(Mp * K);
+      sa.resize(Mp);
+      e = cudaMemcpy(a8.data(), src, a8.size(), cudaMemcpyDeviceToHost);
+      if (e == cudaSuccess) e = cudaMemcpy(sa.data(), scale, Mp * 4, cudaMemcpyDeviceToHost);
+      if (e != cudaSuccess) return e;
+      for (int m = 0; m < M; ++m)
+        for (int k = 0; k < K; ++k) out[(size_t)m * K + k] = act8_get(a8, sa, K, m, k);
+    } else {
+      a16.resize(Mp * K);
+      e = cudaMemcpy(a16.data(), src, a16.size() * 2, cudaMemcpyDeviceToHost);
+      if (e != cudaSuccess) return e;
+      for (int m = 0; m < M; ++m)
+        for (int k = 0; k < K; ++k) out[(size_t)m * K + k] = act128_get(a16, K, m, k);
+    }
+    out += (size_t)M * K;
+    return cudaSuccess;
+  };
+  auto put_h = [&]() -> cudaError_t {
+    // rows of the residual are d apart, the first M of Mp
+    cudaError_t e = cudaMemcpy(out, h->bh, (size_t)M * d * 4, cudaMemcpyDeviceToHost);
+    out += (size_t)M * d;
+    return e;
+  };
+  const float* sa_za = h->w8a8 ? h->bsa : nullptr;
+  const float* sa_zf = h->w8a8 ? h->bsa + 2 * Mp : nullptr;
+  BatchHook hook = [&](int l, int k) -> cudaError_t {
+    cudaError_t e = cudaStreamSynchronize(st);
+    if (e != cudaSuccess) return e;
+    switch (k) {
+      case 0:
+        e = put_h();
+        if (e == cudaSuccess) e = put_act(h->bz_a, sa_za, d);
+        return e;
+      case 1: {
+        e = cudaMemcpy(qh.data(), h->bq, qh.size() * 2, cudaMemcpyDeviceToHost);
+        if (e != cudaSuccess) return e;
+        for (int m = 0; m < M; ++m) {
+          const int b = m / T, t = m % T;
+          for (int n = 0; n < qn; ++n) {
+            const int head = n / hd, el = n % hd, row = (head % G) * T + t;
+            const size_t base = (((size_t)b * c.n_kv_heads + head / G) * h->q_rows + row) * hd;
+            out[(size_t)m * qn + n] = swz_get(qh, base, row, el);
+          }
+        }
+        out += (size_t)M * qn;
+        kvh.resize(lay);
+        for (int which = 0; which < 2; ++which) {
+          e = cudaMemcpy(kvh.data(), (which == 0 ? h->kcache : h->vcache) + l * lay, lay * 2,
+                         cudaMemcpyDeviceToHost);
+          if (e != cudaSuccess) return e;
+          for (int m = 0; m < M; ++m) {
+            const int b = m / T, t = m % T, row = h->prefix_lens[b] + t;
+            for (int n = 0; n < kn; ++n) {
+              const size_t base = (((size_t)b * c.n_kv_heads + n / hd) * h->S_max + row) * hd;
+              out[(size_t)m * kn + n] = swz_get(kvh, base, row, n % hd);
+            }
+          }
+          out += (size_t)M * kn;
+        }
+        return cudaSuccess;
+      }
+      case 2: return put_act(h->bo, nullptr, qn);
+      case 3: return put_h();
+      case 4: return put_act(h->bz_f, sa_zf, d);
+      case 5: return put_act(h->bu, nullptr, F);
+      case 6: return put_h();
+      default:
+        e = cudaMemcpy(out, h->vbuf, (size_t)M * c.action_dim * 4, cudaMemcpyDeviceToHost);
+        out += (size_t)M * c.action_dim;
+        return e;
+    }
+  };
+  (void)L;
+  (void)hbuf;
+  CK(enqueue_batched(h, batch, step_index, step_index + 1, steps, false, st, &hook));
+  CK(cudaStreamSynchronize(st));
+  return check_err_word(h);
 }
 
 fm_status fm_set_prefix_builder(fm_expert* h, const fm_prefix_weights* w, int d_prefix) {
@@ -1682,7 +1876,7 @@ fm_status fm_profile_denoise(fm_expert* h, int batch, int steps, int iters, floa
       p.vbuf = h->vbuf + b * xs;
       p.step1 = steps;
       p.dt = -1.0f / (float)steps;
-      e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
+      e = cudaMemsetAsync(h->flags, 0, kFlagBytes, st);
       if (e == cudaSuccess) e = launch_step(p, st);
     }
     if (e == cudaSuccess) e = cudaEventRecord(ev[2], st);
@@ -1733,7 +1927,7 @@ fm_status fm_profile_phases(fm_expert* h, int steps, uint64_t* out, size_t* n, v
   p.tlog_mma_off = 16 * n_phases;
   p.tlog_chunk_off = 16 * n_phases + 2 * n_gemms;
   p.tlog_chunks = n_chunks;
-  if (e == cudaSuccess) e = cudaMemsetAsync(h->bar_count, 0, (size_t)h->n_ctas * 4, st);
+  if (e == cudaSuccess) e = cudaMemsetAsync(h->flags, 0, kFlagBytes, st);
   if (e == cudaSuccess) e = launch_step(p, st);
   if (e == cudaSuccess) e = cudaMemcpyAsync(out, d, need * 8, cudaMemcpyDeviceToHost, st);
   if (e == cudaSuccess) e = cudaStreamSynchronize(st);
@@ -1741,6 +1935,21 @@ fm_status fm_profile_phases(fm_expert* h, int steps, uint64_t* out, size_t* n, v
   if (e != cudaSuccess) return set_err(h, FM_ERR_CUDA, "profile phases: %s", cudaGetErrorString(e));
   *n = need;
   return check_err_word(h);
+}
+
+fm_status fm_test_stall(fm_expert* h, int on, long long spin_cycles) {
+  if (!h) return FM_ERR_INVALID_ARG;
+  if (spin_cycles < 0) return set_err(h, FM_ERR_INVALID_ARG, "spin_cycles %lld is negative", spin_cycles);
+  CK(cudaSetDevice(h->device));
+  CK(cudaDeviceSynchronize());
+  h->test_stall = on ? 1 : 0;
+  h->test_spin = spin_cycles;
+  // captured graphs hold the old launch parameters
+  for (auto& kv : h->graphs) cudaGraphExecDestroy(kv.second);
+  for (auto& kv : h->graph_defs) cudaGraphDestroy(kv.second);
+  h->graphs.clear();
+  h->graph_defs.clear();
+  return FM_OK;
 }
 
 fm_status fm_sync(fm_expert* h, void* stream) {

@@ -1,6 +1,7 @@
 // Parameter structures of the batched (throughput) path's kernels, shared by
 // the host engine (fm_api.cu) and fm_batch.cu.
 #pragma once
+#include <cuda.h>
 #include <cstdint>
 
 #include "fm_internal.h"
@@ -74,6 +75,11 @@ struct BQuantParams {
 };
 
 struct BAttnParams {
+  // tensor-core kernel: 4-D views (64 elements, hd/64 halves, rows, segments)
+  // of the q buffer (segment b Hkv + g) and of the K/V caches (segment
+  // (l B_cap + b) Hkv + g), box (64, 1, 128, 1): one TMA copy moves 128 half rows
+  CUtensorMap tm_q, tm_k, tm_v;
+  int seg_base;              // l B_cap Hkv: first cache segment of this layer
   const uint16_t* qbuf;      // [B][Hkv][q_rows][hd]
   const uint16_t* kc;        // this layer's cache [B_cap][Hkv][S_max][hd]
   const uint16_t* vc;

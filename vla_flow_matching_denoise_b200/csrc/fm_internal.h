@@ -42,6 +42,19 @@ constexpr int kSmemMax = 232448;       // dynamic shared memory per CTA (227 KB)
 
 enum GemmId { G_QKV = 0, G_O = 1, G_GU = 2, G_DOWN = 3 };
 
+// Hand-offs of the one-request loop kernel.  Each phase's writers add 1 to
+// the phase's counter (release) once their outputs are stored; a consumer
+// waits (acquire) until the counter reaches rounds x writers.
+//   F_Z   z_a, h_a and the h^2 row sums: in-projection / down owners
+//   F_ZF  z_f, h_b and the h^2 row sums: o_proj owners
+//   F_QKV q buffer and the chunk's K/V cache rows: QKV owners
+//   F_O   attention output: attention CTAs
+//   F_U   SwiGLU output: gate_up owners
+//   F_X   chunk x after the Euler update: every CTA
+enum FlagId { F_Z = 0, F_ZF = 1, F_QKV = 2, F_O = 3, F_U = 4, F_X = 5, kNumFlags = 6 };
+constexpr int kFlagStride = 32;   // 32-bit words between counters (one 128-byte line each)
+constexpr size_t kFlagBytes = (size_t)kNumFlags * kFlagStride * 4;
+
 // One linear of a layer, partitioned over clusters.  Cluster c works on
 // NS n-groups of ng[c] packed output channels each (0 = idle cluster); CTA j
 // of the cluster takes n-group j / KS and K-slice j % KS (kslice columns).
@@ -94,17 +107,18 @@ struct StepParams {
   float* vbuf;               // [T, A]
   float* h_a;                // [T, d]
   float* h_b;                // [T, d]
-  uint16_t* z_a;             // ACT64 [64, d]: h (1 + s_a), row 50 = b_a
-  uint16_t* z_f;             // ACT64 [64, d]: h (1 + s_f), row 50 = b_f
-  uint16_t* o_act;           // ACT64 [64, H_q hd]
-  uint16_t* u_act;           // ACT64 [64, F]
+  // activations of layer l live in copy (l & 1) of each buffer
+  uint16_t* z_a;             // 2 x ACT64 [64, d]: h (1 + s_a), row 50 = b_a
+  uint16_t* z_f;             // 2 x ACT64 [64, d]: h (1 + s_f), row 50 = b_f
+  uint16_t* o_act;           // 2 x ACT64 [64, H_q hd]
+  uint16_t* u_act;           // 2 x ACT64 [64, F]
   float* sumsq_a;            // [n_ctas][64] per-CTA partial row sums of h^2
   float* sumsq_f;
   uint16_t* qbuf;            // [H_kv][q_rows][hd]: row (h % G) * T + t of group h / G
   uint16_t* kcache;          // [L][B][H_kv][S_max][hd]
   uint16_t* vcache;
-  uint32_t* bar_count;       // grid barrier arrival counter, zeroed before launch
-                             // (counts CTA arrivals over all barriers of the launch)
+  uint32_t* flags;           // hand-off counters [kNumFlags][kFlagStride], zeroed before
+                             // each launch: writer CTAs add 1 (release) per round
   uint32_t* err;             // error word (non-zero: a bounded wait gave up)
   // schedule of this launch
   int step0, step1;          // modulation rows used
@@ -112,6 +126,8 @@ struct StepParams {
   int do_inproj, do_outproj, update_x;
   float dt;
   long long spin_budget;     // cycles before a wait gives up
+  int stall_test;            // test hook: one writer too many at the QKV hand-off (that wait
+                             // cannot complete; exercises the bounded waits and the abort path)
   // optional phase timeline (globaltimer ns); null when not profiling
   unsigned long long* tlog;  // [n_ctas][tlog_stride]: 8 marks per phase, 2 per GEMM (MMA warp),
   int tlog_stride;           // then per weight chunk: landed (MMA warp) and issued (producer)

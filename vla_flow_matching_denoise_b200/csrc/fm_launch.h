@@ -44,6 +44,9 @@ cudaError_t launch_bresnorm(const BRowParams& p, cudaStream_t st);
 cudaError_t launch_browquant(const BQuantParams& p, cudaStream_t st);
 cudaError_t launch_boutproj(const BRowParams& p, cudaStream_t st);
 cudaError_t launch_battn(const BAttnParams& p, cudaStream_t st);
+// tcgen05 attention: every request's keys (P_b + T <= S_max <= 384) in TMEM at once
+bool battn_tc_supported(int S_max, int hd);
+cudaError_t launch_battn_tc(const BAttnParams& p, cudaStream_t st);
 
 // Sets the text fm_last_error(NULL) returns on this thread.
 void set_thread_error(const char* msg);

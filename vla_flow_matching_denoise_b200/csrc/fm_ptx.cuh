@@ -107,6 +107,18 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
 }
+// 4-D tiled TMA load global -> this CTA's shared memory (no multicast),
+// completing tx bytes on `bar`.  `tmap`: generic address of a CUtensorMap
+// kernel parameter (__grid_constant__); the innermost coordinate c0 times the
+// element size must be a multiple of 16 bytes (callers pass 0).
+__device__ __forceinline__ void tma_load_4d(uint32_t dst, const void* tmap, int c0, int c1, int c2, int c3,
+                                            uint32_t bar, uint64_t policy) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes.L2::cache_hint "
+      "[%0], [%1, {%2, %3, %4, %5}], [%6], %7;" ::"r"(dst),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(bar), "l"(policy)
+      : "memory");
+}
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -219,6 +231,19 @@ __device__ __forceinline__ uint64_t desc_sw128(uint32_t addr) {
   d |= (uint64_t)2 << 61;                         // layout: 128-byte swizzle
   return d;
 }
+// Shared-memory matrix descriptor for an MN-major operand in the 128-byte
+// swizzled layout: 128-byte rows of 64 consecutive MN elements, one row per K
+// index, 8-row groups 1024 B apart along K; the next 64 MN elements start
+// `mn_stride` bytes further.
+__device__ __forceinline__ uint64_t desc_sw128_mn(uint32_t addr, uint32_t mn_stride) {
+  uint64_t d = 0;
+  d |= (uint64_t)((addr >> 4) & 0x3FFF);          // start address
+  d |= (uint64_t)((mn_stride >> 4) & 0x3FFF) << 16;   // leading byte offset: next 64 MN elements
+  d |= (uint64_t)(1024 >> 4) << 32;               // stride byte offset: next 8 K rows
+  d |= (uint64_t)1 << 46;                         // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                         // layout: 128-byte swizzle
+  return d;
+}
 // Instruction descriptor: kind::f16 with bf16 A and B, fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
   return (1u << 4)                 // D format f32
@@ -227,6 +252,8 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N) {
          | ((uint32_t)(N >> 3) << 17)
          | ((uint32_t)(M >> 4) << 24);
 }
+// As idesc_bf16, with B MN-major (transposed).
+__host__ __device__ constexpr uint32_t idesc_bf16_bmn(int M, int N) { return idesc_bf16(M, N) | (1u << 16); }
 // Instruction descriptor: kind::f8f6f4 with E4M3 A and B (format code 0),
 // fp32 D, both K-major.
 __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
@@ -315,6 +342,11 @@ __device__ __forceinline__ uint4 ld_relaxed_v4(const uint32_t* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
                : "l"(p)
                : "memory");
+  return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
 }
 __device__ __forceinline__ void red_release_add(uint32_t* p, uint32_t v) {

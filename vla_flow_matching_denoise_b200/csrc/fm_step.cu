@@ -8,23 +8,24 @@
 // CUDA Graph: the prefix KV cache is reused by every denoise step).
 //
 // Design (B200, one request):
-//  * The grid is every co-resident cluster of 8 CTAs, one CTA per SM.  The
-//    phases of the loop are separated by a grid barrier (release/acquire on a
-//    global counter, bounded spin).
+//  * The grid is every co-resident cluster of 8 CTAs, one CTA per SM.  There
+//    is no grid barrier: each phase's writers add 1 to that phase's counter
+//    in global memory (release) once their outputs are stored, and a phase
+//    waits (acquire, bounded spin) only for the counter of the outputs it
+//    reads, right before it reads them.  Activations alternate between two
+//    copies by layer parity.
 //  * Weights dominate the bytes (34.6 MB per layer at d = 1024), so warp 0 of
 //    every CTA streams its share of every layer, in consumption order, through
-//    a 128 KB shared-memory ring with 1-D bulk (TMA) copies.  The stream runs
-//    ahead across phases and barriers; only ring space throttles it.
-//  * Each linear is split over clusters by output channels (balanced per
-//    cluster) and, inside a cluster, over its 8 CTAs by K and n-groups.  Warp
-//    1 issues tcgen05.mma with M = 64 token rows (50 valid + the shift row +
-//    padding), N = the CTA's channels, accumulating fp32 in TMEM.
-//  * Split-K partials leave TMEM through tcgen05.ld, are staged in shared
-//    memory as one block per owner of output columns, and each block goes to
-//    its owner with one bulk copy shared::cta -> shared::cluster that
-//    completes bytes on the owner's mbarrier; the owner waits once and reduces
-//    its KS slots from local shared memory in a fixed order (results are
-//    bit-reproducible).
+//    a 126 KB shared-memory ring with 1-D bulk (TMA) copies.  The stream runs
+//    ahead across phases; only ring space throttles it.
+//  * Each linear is split over clusters by output channels and, inside a
+//    cluster, over its 8 CTAs by K and n-groups.  Warp 1 issues tcgen05.mma
+//    with M = 64 token rows (50 valid + the shift row + padding), N = the
+//    CTA's channels, accumulating fp32 in TMEM.
+//  * Split-K partials leave TMEM through tcgen05.ld straight into registers
+//    and go to the owner of each column with st.async into the owner's shared
+//    memory, completing bytes on its mbarrier; the owner reduces its KS slots
+//    in a fixed order (results are bit-reproducible).
 //  * AdaRMSNorm is folded into the linears: the owner of a residual column
 //    writes z = bf16(h (1 + s)) and, in row 50, the shift b; the consumer
 //    linear's epilogue applies rstd(row) to rows 0..49 and adds row 50
@@ -34,12 +35,12 @@
 //    rows of that group's heads) on one cluster, keys split over its 8 CTAs,
 //    mma.sync with an online softmax, partials pushed to the row owners for
 //    the log-sum-exp combine.
-//  * E4M3 weights ("LingBot-VLA on Thor (sm_110)", §2: FP8 weight path):
-//    the ring receives one-byte codes in the upper half of each chunk's slot;
-//    two extra warps widen them in place to the bf16 image (exact: every E4M3
-//    value is a bf16 value), so the tensor cores still run bf16 x bf16 with
-//    bf16 activations.  The per-output-row scale multiplies the reduced fp32
-//    sum in the epilogue.
+//  * E4M3 / NVFP4 weights ("LingBot-VLA on Thor (sm_110)", §2: FP8 weight
+//    path, FP4 gate_up) run in a second instantiation of the kernel with two
+//    extra warps that widen the codes in the ring to the bf16 image (exact),
+//    so the tensor cores still run bf16 x bf16; the per-output-row scale
+//    multiplies the reduced fp32 sum in the epilogue.  The bf16 instantiation
+//    carries none of that code.
 #include <cuda_bf16.h>
 #include <cstddef>
 #include <cstdint>
@@ -76,6 +77,7 @@ struct Ctrl {
   uint64_t xsync;     // cluster rendezvous (8 arrivals)
   uint32_t tmem_slot;
   int abort;
+  uint32_t writers[kNumFlags];       // CTAs that signal each hand-off per round
   alignas(16) float rstd[kRows];
   alignas(16) float red[8][kRows];   // written with float4 stores
   GemmView views[4];                 // this CTA's share of each linear (fixed per launch)
@@ -87,7 +89,7 @@ static_assert(kSmemBytes <= (size_t)kSmemMax, "shared memory budget");
 
 // Error codes (bit flags in p.err).
 enum : uint32_t {
-  E_GRID = 1u << 0,
+  E_FLAG = 1u << 0,
   E_RING_PROD = 1u << 1,
   E_RING_MMA = 1u << 2,
   E_RECV = 1u << 3,
@@ -148,7 +150,8 @@ struct Ctx {
   int lane;
   uint32_t gemm_count;  // GEMM phases run (parity of act_full / mma_done)
   uint32_t recv_count, att_count, xs_count;
-  uint32_t epoch;       // grid barriers passed
+  uint32_t phase;       // phases passed (profiling marks)
+  uint32_t ep[kNumFlags];   // hand-off rounds signalled so far, per counter
   int P;                // prefix length (read from the device)
   bool ok;
 };
@@ -161,7 +164,7 @@ __device__ __forceinline__ void compute_sync() { named_bar_sync(1, kComputeWarps
 // synchronised, 8.. phase-specific points.
 __device__ __forceinline__ void tmark(const Ctx& c, int slot) {
   if (c.p->tlog != nullptr && c.tid == 0) {
-    const int idx = (int)c.epoch * 16 + slot;
+    const int idx = (int)c.phase * 16 + slot;
     if (idx < c.p->tlog_mma_off) c.p->tlog[(size_t)c.cta * c.p->tlog_stride + idx] = gtimer();
   }
 }
@@ -172,33 +175,59 @@ __device__ void fail(Ctx& c, uint32_t code) {
   c.ok = false;
 }
 
-// Grid barrier among the compute warps of every CTA: one release add per CTA
-// on a shared arrival counter (cumulative: the CTA barrier before it orders
-// every compute thread's writes), then one thread polls it with acquire loads
-// until all CTAs of this barrier generation have arrived.
-__device__ void grid_sync(Ctx& c) {
+// Bulk loads of `nch` 8 KB activation blocks (one thread), completing on act_full.
+__device__ __forceinline__ void issue_act(const Ctx& c, const uint16_t* src, int nch) {
+  const uint64_t pol = policy_evict_last();
+  const uint32_t bar = smem_u32(&c.ctl->act_full);
+  mbar_arrive_expect_tx(bar, (uint32_t)nch * 8192u);
+  const uint32_t dst = smem_u32(c.work);
+#pragma unroll 1
+  for (int i = 0; i < nch; ++i) bulk_g2s(dst + i * 8192, src + (size_t)i * (kRows * 64), 8192, bar, pol);
+}
+
+// Waits until hand-off counter f has seen every writer of every round
+// signalled so far (one thread polls, bounded), makes the data visible to
+// this CTA's bulk copies and releases the compute warps.  A GEMM phase passes
+// its K-slice of the activations (`act`, `nch` blocks), which the polling
+// thread requests at once, before the other threads are released.
+__device__ __noinline__ void wait_flag(Ctx& c, int f, const uint16_t* act = nullptr, int nch = 0) {
   if (!c.ok) return;
-  tmark(c, 4);
-  fence_proxy_async_global();
-  compute_sync();
+  const uint32_t target = c.ep[f] * c.ctl->writers[f];
   if (c.tid == 0) {
-    const uint32_t target = (c.epoch + 1) * (uint32_t)c.p->n_ctas;
-    uint32_t* count = c.p->bar_count;
-    red_release_add(count, 1u);
-    tmark(c, 5);
-    const long long t0 = clock64();
-    while (ld_acquire_u32(count) < target) {
-      if (*(volatile uint32_t*)c.p->err != 0u || clock64() - t0 > c.p->spin_budget) {
-        fail(c, E_GRID);
-        break;
+    if (target > 0u) {
+      const uint32_t* cnt = c.p->flags + f * kFlagStride;
+      const long long t0 = clock64();
+      uint32_t it = 0;
+      while (ld_acquire_u32(cnt) < target) {
+        if ((++it & 15u) == 0u &&
+            (*(volatile uint32_t*)c.p->err != 0u || clock64() - t0 > c.p->spin_budget)) {
+          fail(c, E_FLAG);
+          break;
+        }
       }
+      fence_proxy_async_global();
     }
-    fence_proxy_async_global();
+    if (act != nullptr && c.ok) issue_act(c, act, nch);
   }
   compute_sync();
   if (*(volatile int*)&c.ctl->abort) c.ok = false;
-  ++c.epoch;
   tmark(c, 0);
+}
+
+// Ends a phase: a writer CTA orders its stores (generic and async proxy)
+// before one release add on counter f; every CTA counts the round.
+__device__ __noinline__ void signal(Ctx& c, int f, bool wrote) {
+  if (c.ok && wrote) {
+    tmark(c, 4);
+    fence_proxy_async_global();
+    tmark(c, 13);
+    compute_sync();
+    tmark(c, 14);
+    if (c.tid == 0) red_release_add(c.p->flags + f * kFlagStride, 1u);
+    tmark(c, 5);
+  }
+  ++c.ep[f];
+  ++c.phase;
 }
 
 // ------------------------------------------------------------ producer warp
@@ -372,40 +401,46 @@ __device__ __noinline__ void converter(const StepParams& p, uint8_t* ring, Ctrl*
 // ------------------------------------------------------------ MMA warp
 __device__ __noinline__ void mma_issuer(const StepParams& p, uint8_t* ring, uint8_t* work, Ctrl* ctl,
                            uint32_t tmem, int cluster) {
-  uint32_t nch[4], bytes[4], idesc[4];
+  // per-linear values in registers: the linear loop below is unrolled
+  uint32_t nch[4], bytes[4], idesc[4], wide[4];
+#pragma unroll
   for (int g = 0; g < 4; ++g) {
     const int ng = p.g[g].ng[cluster];
     nch[g] = ng > 0 ? (uint32_t)p.g[g].nchunk : 0u;
     bytes[g] = (uint32_t)ng * 128u;
     idesc[g] = idesc_bf16(kRows, ng > 0 ? ng : 16);
+    wide[g] = p.wfmt[g] != 0 ? 1u : 0u;
   }
+  unsigned long long* const tlog = p.tlog;
+  const int tlog_row = p.tlog_stride * (int)blockIdx.x, tlog_mma = p.tlog_mma_off, tlog_chunk = p.tlog_chunk_off,
+            tlog_chunks = p.tlog_chunks, tlog_stride = p.tlog_stride;
+  const long long budget = p.spin_budget;
   uint32_t it = 0, pos = 0, gemm_count = 0;
   bool good = true;
   const uint32_t a_base = smem_u32(work);
   const uint32_t r_base = smem_u32(ring);
   for (int s = p.step0; s < p.step1 && good; ++s) {
     for (int l = p.layer0; l < p.layer1 && good; ++l) {
-      for (int g = 0; g < 4 && good; ++g) {
-        if (nch[g] == 0) continue;
-        if (!wait_ab(smem_u32(&ctl->act_full), gemm_count & 1, p.spin_budget, &ctl->abort)) {
+#pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        if (!good || nch[g] == 0) continue;
+        if (!wait_ab(smem_u32(&ctl->act_full), gemm_count & 1, budget, &ctl->abort)) {
           good = false;
-          break;
+          continue;
         }
         tc_fence_after();
-        if (p.tlog != nullptr) {
-          const int idx = p.tlog_mma_off + 2 * (int)gemm_count;
-          if (idx < p.tlog_stride) p.tlog[(size_t)blockIdx.x * p.tlog_stride + idx] = gtimer();
-        }
+        if (tlog != nullptr && tlog_mma + 2 * (int)gemm_count < tlog_stride)
+          tlog[tlog_row + tlog_mma + 2 * (int)gemm_count] = gtimer();
+#pragma unroll 1
         for (uint32_t c = 0; c < nch[g]; ++c, ++it) {
           const uint32_t at = ring_place(pos, bytes[g]);
           const uint32_t slot = it % kRingSlots;
-          if (!wait_ab(smem_u32(p.wfmt[g] ? &ctl->conv[slot] : &ctl->full[slot]), (it / kRingSlots) & 1,
-                       p.spin_budget, &ctl->abort)) {
+          if (!wait_ab(smem_u32(wide[g] ? &ctl->conv[slot] : &ctl->full[slot]), (it / kRingSlots) & 1, budget,
+                       &ctl->abort)) {
             good = false;
             break;
           }
-          if (p.tlog != nullptr && (int)it < p.tlog_chunks)
-            p.tlog[(size_t)blockIdx.x * p.tlog_stride + p.tlog_chunk_off + it] = gtimer();
+          if (tlog != nullptr && (int)it < tlog_chunks) tlog[tlog_row + tlog_chunk + it] = gtimer();
           tc_fence_after();
 #pragma unroll
           for (int k16 = 0; k16 < 4; ++k16)
@@ -413,11 +448,9 @@ __device__ __noinline__ void mma_issuer(const StepParams& p, uint8_t* ring, uint
                      desc_sw128(r_base + at + k16 * 32), idesc[g], (c | k16) != 0);
           mma_commit(smem_u32(&ctl->empty[slot]));
         }
-        if (!good) break;
-        if (p.tlog != nullptr) {
-          const int idx = p.tlog_mma_off + 2 * (int)gemm_count + 1;
-          if (idx < p.tlog_stride) p.tlog[(size_t)blockIdx.x * p.tlog_stride + idx] = gtimer();
-        }
+        if (!good) continue;
+        if (tlog != nullptr && tlog_mma + 2 * (int)gemm_count + 1 < tlog_stride)
+          tlog[tlog_row + tlog_mma + 2 * (int)gemm_count + 1] = gtimer();
         mma_commit(smem_u32(&ctl->mma_done));
         ++gemm_count;
       }
@@ -429,7 +462,7 @@ __device__ __noinline__ void mma_issuer(const StepParams& p, uint8_t* ring, uint
   }
   // Drain: all issued MMAs must finish before TMEM is released.
   mma_commit(smem_u32(&ctl->drain));
-  mbar_wait(smem_u32(&ctl->drain), 0, p.spin_budget);
+  mbar_wait(smem_u32(&ctl->drain), 0, budget);
 }
 
 // ------------------------------------------------------------ compute warps
@@ -472,103 +505,75 @@ __device__ __forceinline__ float2 wscale2(const Ctx& c, int g, int l, int idx) {
   return *reinterpret_cast<const float2*>(p.wscale + (size_t)l * p.sc_stride + p.sc_off[g] + idx);
 }
 
-// Starts GEMM g: arms the receive barrier for the partials the cluster will
-// push here and loads this CTA's K-slice of the activations.
-__device__ __noinline__ void gemm_begin(const Ctx& c, const GemmView& v, const uint16_t* act) {
-  if (c.tid == 0) {
-    Ctrl* ctl = c.ctl;
-    mbar_arrive_expect_tx(smem_u32(&ctl->recv), (uint32_t)(v.KS * kRecvRows * v.ownp * 4));
-    fence_proxy_async_smem();
-    const uint64_t pol = policy_evict_last();
-    const uint32_t bar = smem_u32(&ctl->act_full);
-    const int nch = v.nchunk;
-    mbar_arrive_expect_tx(bar, (uint32_t)nch * 8192u);
-    const uint16_t* src = act + (size_t)(v.ks * nch) * (kRows * 64);
-    const uint32_t dst = smem_u32(c.work);
-#pragma unroll 1
-    for (int i = 0; i < nch; ++i) bulk_g2s(dst + i * 8192, src + (size_t)i * (kRows * 64), 8192, bar, pol);
-  }
+// Arms the receive barrier for the split-K partials the cluster will push
+// here in GEMM g (safe before the input is ready: a peer pushes only after
+// its own input wait, which this CTA's previous phase has released).
+__device__ __forceinline__ void arm_recv(const Ctx& c, const GemmView& v) {
+  if (c.tid == 0)
+    mbar_arrive_expect_tx(smem_u32(&c.ctl->recv), (uint32_t)(v.KS * kRecvRows * v.own * 4));
 }
 
-// Waits for the MMAs, stages rows 0..50 of the fp32 partial sums as one
-// contiguous block per owner ([owner][row][ownp]) and sends block o to owner
-// o's receive slot `ks` with one bulk copy each.  push_wait then waits until
-// this CTA's own receive buffer is complete; work that does not need the
-// partials goes between the two.
+// Waits for the MMAs and sends rows 0..50 of the fp32 partial sums to the
+// owners of their columns.  With the M = 64 accumulator, rows 16 q .. 16 q +
+// 15 sit in TMEM lanes 32 q .. 32 q + 15 of warp quarter q; a 16x256b load
+// gives lane t rows 16 q + t/4 and + 8 and column pairs 2 (t % 4) + 8 j.  One
+// exchange between lanes t and t ^ 1 leaves every lane four consecutive
+// columns of one row (even lanes the low row, odd lanes the high row), which
+// go to the column's owner as one 16-byte st.async into its receive slot
+// `ks`, completing bytes on the owner's receive barrier.  Owners hold a
+// multiple of 4 columns, so a piece never straddles two owners.
 __device__ __noinline__ void push_send(Ctx& c, const GemmView& v) {
   if (!c.ok) return;
   Ctrl* const ctl = c.ctl;
-  const long long budget = c.p->spin_budget;
-  const int tid = c.tid;
   tmark(c, 12);
-  if (!wait_ab(smem_u32(&ctl->mma_done), c.gemm_count & 1, budget, &ctl->abort)) {
+  if (!wait_ab(smem_u32(&ctl->mma_done), c.gemm_count & 1, c.p->spin_budget, &ctl->abort)) {
     fail(c, E_MMA_DONE);
     return;
   }
   ++c.gemm_count;
   tc_fence_after();
   tmark(c, 1);
-  const int ng = v.ng, own = v.own, ownp = v.ownp;
-  // M = 64 accumulator: rows 16 sp .. 16 sp + 15 sit in TMEM lanes 32 sp ..
-  // 32 sp + 15 of this warp's quarter; 16x256b loads spread them over all 32
-  // threads (rows r_lo, r_lo + 8; column pairs 2 (lane % 4) + 8 j).
-  const int sp = c.warp & 3;
-  const int r_lo = 16 * sp + (c.lane >> 2), r_hi = r_lo + 8;
-  const bool ok_lo = r_lo < kRecvRows, ok_hi = r_hi < kRecvRows;
-  const int cq = 2 * (c.lane & 3);
-  const uint32_t tb = c.tmem + ((uint32_t)(32 * sp) << 16);
-  float* const stg = reinterpret_cast<float*>(c.work);
-  // this thread's columns are cq, cq + 8, ...: their owner block and column
-  // inside it advance incrementally (owners hold an even number of columns,
-  // so a column pair never straddles two owners)
-  float* blk = stg;
-  int lc = cq;
+  const int q = c.warp & 3, lane = c.lane;
+  const bool odd = (lane & 1) != 0;
+  const int r = 16 * q + (lane >> 2) + (odd ? 8 : 0);
+  const bool act = r < kRecvRows;
+  const uint32_t tb = c.tmem + ((uint32_t)(32 * q) << 16);
+  const int ng = v.ng, own = v.own;
+  const uint32_t recv_local = smem_u32(c.work + v.recv_off), bar_local = smem_u32(&ctl->recv);
+  const uint32_t row_bytes = (uint32_t)((v.ks * kRecvRows + r) * v.ownp) * 4u;
+  const int rank0 = v.grp * v.KS;
+  // owner and column inside it of this lane's first column (2 (lane & 2)),
+  // advanced by 8 columns per piece
+  int o = 0, lc = 2 * (lane & 2);
   while (lc >= own) {
     lc -= own;
-    blk += kRecvRows * ownp;
+    ++o;
   }
-  blk += lc;
-  // up to 128 columns are requested before one wait, so the TMEM read
-  // latency is paid once per 128 columns
-  constexpr int kBatch = 4;   // loads of 32 columns per wait
 #pragma unroll 1
-  for (int c0 = 0; c0 < ng; c0 += 32 * kBatch) {
-    float x[kBatch][16];
-#pragma unroll
-    for (int h = 0; h < kBatch; ++h)
-      if (c0 + 32 * h < ng) tmem_ld_16x256b_x4(tb + c0 + 32 * h, x[h]);
+  for (int c0 = 0; c0 < ng; c0 += 32) {
+    float x[16];
+    tmem_ld_16x256b_x4(tb + c0, x);
     tmem_ld_wait();
-    if (c0 == 0) tmark(c, 13);
 #pragma unroll
-    for (int h = 0; h < kBatch; ++h) {
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        if (c0 + 32 * h + 8 * j >= ng) break;
-        if (ok_lo) *reinterpret_cast<float2*>(blk + r_lo * ownp) = make_float2(x[h][4 * j], x[h][4 * j + 1]);
-        if (ok_hi) *reinterpret_cast<float2*>(blk + r_hi * ownp) = make_float2(x[h][4 * j + 2], x[h][4 * j + 3]);
-        lc += 8;
-        blk += 8;
-        while (lc >= own) {
-          lc -= own;
-          blk += kRecvRows * ownp - own;
-        }
+    for (int j = 0; j < 4; ++j) {
+      const float sa = odd ? x[4 * j] : x[4 * j + 2];
+      const float sb = odd ? x[4 * j + 1] : x[4 * j + 3];
+      const float ra = __shfl_xor_sync(0xffffffffu, sa, 1);
+      const float rb = __shfl_xor_sync(0xffffffffu, sb, 1);
+      if (act && c0 + 8 * j < ng) {
+        const uint32_t rk = (uint32_t)(rank0 + o);
+        const uint32_t dst = map_shared_rank(recv_local, rk) + row_bytes + 4u * lc;
+        if (odd) st_async_v4(dst, ra, rb, x[4 * j + 2], x[4 * j + 3], map_shared_rank(bar_local, rk));
+        else st_async_v4(dst, x[4 * j], x[4 * j + 1], ra, rb, map_shared_rank(bar_local, rk));
+      }
+      lc += 8;
+      while (lc >= own) {
+        lc -= own;
+        ++o;
       }
     }
   }
   tc_fence_before();
-  tmark(c, 6);
-  fence_proxy_async_smem();
-  compute_sync();
-  tmark(c, 7);
-  const uint32_t recv_local = smem_u32(c.work + v.recv_off);
-  const uint32_t bar_local = smem_u32(&ctl->recv);
-  if (tid < v.KS) {
-    // one thread per owner issues that owner's copy
-    const uint32_t blk = (uint32_t)(kRecvRows * ownp * 4);
-    const uint32_t dst = (uint32_t)(v.grp * v.KS + tid);
-    bulk_s2cluster(map_shared_rank(recv_local + (uint32_t)v.ks * blk, dst), smem_u32(stg) + (uint32_t)tid * blk,
-                   blk, map_shared_rank(bar_local, dst));
-  }
   tmark(c, 2);
 }
 
@@ -655,9 +660,7 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
   const StepParams& p = *c.p;
   const GemmView v = gemm_view(c, G_QKV);
   if (v.ng == 0) return;
-  gemm_begin(c, v, p.z_a);
-  tmark(c, 11);
-  load_rstd(c, p.sumsq_a);
+  arm_recv(c, v);
   const int T = p.T, hd = p.hd, half = hd / 2, G = p.Hq / p.Hkv;
   const int qn = p.Hq * hd, kn = p.Hkv * hd, N = p.g[G_QKV].N;
   const int P = c.P;
@@ -677,10 +680,8 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
     dst = (kind == 1 ? p.kcache : p.vcache) + (((size_t)l * p.B_cap + p.b) * p.Hkv + head) * p.S_max * hd;
     row_off = P;
   }
-  const float2 sc = act ? wscale2(c, G_QKV, l, v.pbase + 2 * pa.pr) : make_float2(1.f, 1.f);
-  push_send(c, v);
-  // stage the rotation of every row of this thread while the partials are in
-  // flight (all loads at once; the planner keeps the rows per thread within
+  // stage the rotation of every row of this thread before the input is
+  // ready (all loads at once; the planner keeps the rows per thread within
   // kAuxRows)
   float2* aux = reinterpret_cast<float2*>(c.work + kWorkBytes - kAuxBytes) + c.tid;
   if (act && kind < 2) {
@@ -695,6 +696,11 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
     for (int k = 0; k < kAuxRows; ++k)
       if (pa.t0 + k * pa.dt < T) aux[k * 128] = rv[k];
   }
+  wait_flag(c, F_Z, p.z_a + (size_t)(l & 1) * kRows * p.d + (size_t)(v.ks * v.nchunk) * (kRows * 64), v.nchunk);
+  tmark(c, 11);
+  load_rstd(c, p.sumsq_a);
+  const float2 sc = act ? wscale2(c, G_QKV, l, v.pbase + 2 * pa.pr) : make_float2(1.f, 1.f);
+  push_send(c, v);
   push_wait(c);
   if (!c.ok || !act) return;
   const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
@@ -940,7 +946,7 @@ __device__ __noinline__ void attention_unit(Ctx& c, int l, int grp, int blk) {
       uint32_t pk[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) pk[i] = pack_bf16(acc[2 * i] * inv, acc[2 * i + 1] * inv);
-      *reinterpret_cast<uint4*>(p.o_act + act64_off(t, head * HD + 8 * seg)) =
+      *reinterpret_cast<uint4*>(p.o_act + (size_t)(l & 1) * kRows * p.Hq * HD + act64_off(t, head * HD + 8 * seg)) =
           make_uint4(pk[0], pk[1], pk[2], pk[3]);
     }
   }
@@ -950,6 +956,8 @@ __device__ __noinline__ void phase_attn(Ctx& c, int l) {
   const StepParams& p = *c.p;
   if (!c.ok) return;
   const int units = p.Hkv * p.att_blocks;
+  if (c.cluster >= units) return;
+  wait_flag(c, F_QKV);
   bool more = false;
   for (int u = c.cluster; u < units; u += p.n_clusters) {
     if (more) {
@@ -977,14 +985,13 @@ __device__ __noinline__ void phase_attn(Ctx& c, int l) {
 // o_proj / down: gated residual on the owned columns, two threads per row t
 // (each half of the owned column pairs); z for the next linear, row sum of
 // squares.  Operands of the epilogue are fetched before the MMAs finish.
-__device__ __noinline__ void residual_phase(Ctx& c, int g, int l, const uint16_t* act, const float* h_old,
-                                            float* h_new, const float* gate, const float* sc,
-                                            const float* shift, uint16_t* z, float* sumsq) {
+__device__ __noinline__ void residual_phase(Ctx& c, int g, int f_in, int l, const uint16_t* act,
+                                            const float* h_old, float* h_new, const float* gate,
+                                            const float* sc, const float* shift, uint16_t* z, float* sumsq) {
   if (!c.ok) return;
   const GemmView v = gemm_view(c, g);
   if (v.ng == 0) return;
-  gemm_begin(c, v, act);
-  tmark(c, 11);
+  arm_recv(c, v);
   const int T = c.p->T, d = c.p->d;
   const int tid = c.tid;
   const int t = tid >> 1, hf = tid & 1;
@@ -1003,14 +1010,20 @@ __device__ __noinline__ void residual_phase(Ctx& c, int g, int l, const uint16_t
       const float2 ws = wscale2(c, g, l, v.pbase + 2 * (p0 + k));
       gt[k].x *= ws.x;
       gt[k].y *= ws.y;
-      if (t < T) ho[k] = *reinterpret_cast<const float2*>(h_old + (size_t)t * d + hc);
       if (z != nullptr) sv[k] = *reinterpret_cast<const float2*>((t == kBiasRow ? shift : sc) + hc);
     }
   }
+  wait_flag(c, f_in, act + (size_t)(v.ks * v.nchunk) * (kRows * 64), v.nchunk);
+  tmark(c, 11);
+  // the residual rows were stored two hand-offs ago: visible after the wait
+#pragma unroll
+  for (int k = 0; k < kMaxPairs; ++k)
+    if (k < np && t < T) ho[k] = *reinterpret_cast<const float2*>(h_old + (size_t)t * d + hc0 + 2 * k);
   push_send(c, v);
   push_wait(c);
   if (!c.ok) return;
   const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
+  tmark(c, 8);
   float sq = 0.f;
 #pragma unroll
   for (int k = 0; k < kMaxPairs; ++k) {
@@ -1038,7 +1051,8 @@ __device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
   const StepParams& p = *c.p;
   const GemmView v = gemm_view(c, G_GU);
   if (v.ng == 0) return;
-  gemm_begin(c, v, p.z_f);
+  arm_recv(c, v);
+  wait_flag(c, F_ZF, p.z_f + (size_t)(l & 1) * kRows * p.d + (size_t)(v.ks * v.nchunk) * (kRows * 64), v.nchunk);
   tmark(c, 11);
   load_rstd(c, p.sumsq_f);
   push_send(c, v);
@@ -1051,7 +1065,7 @@ __device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
   if (!pa.active || uc >= F) return;
   const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
   const float* rstd = c.ctl->rstd;
-  uint16_t* u_act = p.u_act;
+  uint16_t* u_act = p.u_act + (size_t)(l & 1) * kRows * F;
   const int lg = 2 * pa.pr, lu = uown + 2 * pa.pr;
   const float2 sg = wscale2(c, G_GU, l, v.pbase + lg), su = wscale2(c, G_GU, l, v.pbase + lu);
   const float2 bg = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lg);
@@ -1077,6 +1091,7 @@ __device__ __noinline__ void phase_inproj(Ctx& c, int step) {
   const StepParams& p = *c.p;
   const GemmView v = gemm_view(c, G_DOWN);
   if (v.ng == 0) return;
+  wait_flag(c, F_X);   // the previous step's Euler update of the whole chunk
   const int T = p.T, A = p.A, d = p.d, own = v.own, base = v.base;
   const int tid = c.tid;
   float* xs = reinterpret_cast<float*>(c.work);            // [T][A]
@@ -1116,7 +1131,7 @@ __device__ __noinline__ void phase_inproj(Ctx& c, int step) {
   const int hc = base + 2 * pa.pr;
   if (pa.active && hc < d) {
     float* h_a = p.h_a;
-    uint16_t* z_a = p.z_a;
+    uint16_t* z_a = p.z_a + (size_t)(p.layer0 & 1) * kRows * d;
     const float2 sa = *reinterpret_cast<const float2*>(s_a + hc);
     const float* w0 = ws + (2 * pa.pr) * A;
     const float* w1 = w0 + A;
@@ -1163,6 +1178,7 @@ __device__ __noinline__ void phase_inproj(Ctx& c, int step) {
 // up to 4 actions at a time.
 __device__ __noinline__ void phase_outproj(Ctx& c, int step) {
   if (!c.ok) return;
+  wait_flag(c, F_Z);   // every residual column and its row sums
   const StepParams& p = *c.p;
   const int T = p.T, A = p.A, d = p.d, n_ctas = p.n_ctas;
   const int lane = c.lane;
@@ -1232,40 +1248,48 @@ __device__ __noinline__ void phase_outproj(Ctx& c, int step) {
 
 __device__ void compute_main(Ctx& c) {
   const StepParams& p = *c.p;
-  tmark(c, 0);
+  const int L = p.L, d = p.d;
+  const size_t zs = (size_t)kRows * d;
+  const bool busy_qkv = gemm_view(c, G_QKV).ng > 0, busy_o = gemm_view(c, G_O).ng > 0,
+             busy_gu = gemm_view(c, G_GU).ng > 0, busy_down = gemm_view(c, G_DOWN).ng > 0;
+  const bool busy_att = c.cluster < p.Hkv * p.att_blocks;
   for (int s = p.step0; s < p.step1 && c.ok; ++s) {
     if (p.do_inproj) {
       phase_inproj(c, s);
-      grid_sync(c);
+      signal(c, F_Z, busy_down);
     }
     for (int l = p.layer0; l < p.layer1 && c.ok; ++l) {
+      const size_t par = (size_t)(l & 1);
       phase_qkv(c, s, l);
-      grid_sync(c);
+      signal(c, F_QKV, busy_qkv);
       phase_attn(c, l);
-      grid_sync(c);
-      residual_phase(c, G_O, l, p.o_act, p.h_a, p.h_b, mod_vec(p, s, l, 2), mod_vec(p, s, l, 3),
-                     mod_vec(p, s, l, 4), p.z_f, p.sumsq_f);
-      grid_sync(c);
+      signal(c, F_O, busy_att);
+      residual_phase(c, G_O, F_O, l, p.o_act + par * kRows * p.Hq * p.hd, p.h_a, p.h_b, mod_vec(p, s, l, 2),
+                     mod_vec(p, s, l, 3), mod_vec(p, s, l, 4), p.z_f + par * zs, p.sumsq_f);
+      signal(c, F_ZF, busy_o);
       phase_gu(c, s, l);
-      grid_sync(c);
+      signal(c, F_U, busy_gu);
       {
-        const bool next = l + 1 < p.L;
-        residual_phase(c, G_DOWN, l, p.u_act, p.h_b, p.h_a, mod_vec(p, s, l, 5),
+        const bool next = l + 1 < L;
+        residual_phase(c, G_DOWN, F_U, l, p.u_act + par * kRows * p.F, p.h_b, p.h_a, mod_vec(p, s, l, 5),
                        next ? mod_vec(p, s, l + 1, 0) : nullptr, next ? mod_vec(p, s, l + 1, 1) : nullptr,
-                       next ? p.z_a : nullptr, p.sumsq_a);
+                       next ? p.z_a + (1 - par) * zs : nullptr, p.sumsq_a);
       }
-      grid_sync(c);
+      signal(c, F_Z, busy_down);
     }
     if (p.do_outproj) {
       phase_outproj(c, s);
-      grid_sync(c);
+      signal(c, F_X, true);
     }
   }
 }
 
 }  // namespace
 
-__global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_constant__ StepParams p) {
+// kWide: quantised weights (two widening warps); otherwise bf16 weights only.
+template <bool kWide>
+__global__ void __launch_bounds__(kWide ? kStepThreads : kThreads, 1)
+    step_kernel(const __grid_constant__ StepParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* ring = smem;
@@ -1289,6 +1313,14 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_cons
     mbar_init(smem_u32(&ctl->xsync), kClusterSize);
     ctl->abort = 0;
     for (int g = 0; g < 4; ++g) ctl->views[g] = compute_view(p, g, cluster, (int)cluster_rank());
+    // writer CTAs of each hand-off: the busy clusters of the phase
+    const int units = p.Hkv * p.att_blocks;
+    ctl->writers[F_Z] = (uint32_t)(kClusterSize * p.g[G_DOWN].busy_clusters);
+    ctl->writers[F_ZF] = (uint32_t)(kClusterSize * p.g[G_O].busy_clusters);
+    ctl->writers[F_QKV] = (uint32_t)(kClusterSize * p.g[G_QKV].busy_clusters + (p.stall_test ? 1 : 0));
+    ctl->writers[F_U] = (uint32_t)(kClusterSize * p.g[G_GU].busy_clusters);
+    ctl->writers[F_O] = (uint32_t)(kClusterSize * min(units, p.n_clusters));
+    ctl->writers[F_X] = (uint32_t)p.n_ctas;
     fence_mbar_init();
   }
   if (warp == 1) {
@@ -1310,8 +1342,7 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_cons
     if (lane == 0) mma_issuer(p, ring, work, ctl, tmem, cluster);
     __syncwarp();
   } else if (warp >= 2 + kComputeWarps) {
-    if (p.wfmt[0] | p.wfmt[1] | p.wfmt[2] | p.wfmt[3])
-      converter(p, ring, ctl, cluster, threadIdx.x - 32 * (2 + kComputeWarps));
+    if constexpr (kWide) converter(p, ring, ctl, cluster, threadIdx.x - 32 * (2 + kComputeWarps));
   } else {
     Ctx c;
     c.p = &p;
@@ -1325,7 +1356,8 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_cons
     c.warp = warp;
     c.lane = lane;
     c.gemm_count = c.recv_count = c.att_count = c.xs_count = 0;
-    c.epoch = 0;
+    c.phase = 0;
+    for (int f = 0; f < kNumFlags; ++f) c.ep[f] = 0;
     c.P = p.P_dev[p.b];
     c.ok = true;
     compute_main(c);
@@ -1341,40 +1373,45 @@ __global__ void __launch_bounds__(kStepThreads, 1) step_kernel(const __grid_cons
   }
 }
 
+namespace {
+
+bool wide_weights(const StepParams& p) { return (p.wfmt[0] | p.wfmt[1] | p.wfmt[2] | p.wfmt[3]) != 0; }
+
+cudaLaunchConfig_t step_config(int n_ctas, bool wide, cudaLaunchAttribute* attr) {
+  cudaLaunchConfig_t cfg = {};
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kClusterSize;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.gridDim = dim3(n_ctas, 1, 1);
+  cfg.blockDim = dim3(wide ? kStepThreads : kThreads, 1, 1);
+  cfg.dynamicSmemBytes = kSmemBytes;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cfg;
+}
+
+}  // namespace
+
 size_t step_smem_bytes() { return kSmemBytes; }
 
 cudaError_t step_max_clusters(int* n_clusters) {
-  cudaError_t e = cudaFuncSetAttribute(step_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(step_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kSmemBytes);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(step_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
   if (e != cudaSuccess) return e;
-  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kClusterSize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(kClusterSize * 32, 1, 1);
-  cfg.blockDim = dim3(kStepThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaOccupancyMaxActiveClusters(n_clusters, step_kernel, &cfg);
+  const cudaLaunchConfig_t cfg = step_config(kClusterSize * 32, true, attr);
+  return cudaOccupancyMaxActiveClusters(n_clusters, step_kernel<true>, &cfg);
 }
 
 cudaError_t launch_step(const StepParams& p, cudaStream_t st) {
-  cudaLaunchConfig_t cfg = {};
   cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = kClusterSize;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.gridDim = dim3(p.n_ctas, 1, 1);
-  cfg.blockDim = dim3(kStepThreads, 1, 1);
-  cfg.dynamicSmemBytes = kSmemBytes;
+  const bool wide = wide_weights(p);
+  cudaLaunchConfig_t cfg = step_config(p.n_ctas, wide, attr);
   cfg.stream = st;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, step_kernel, p);
+  return wide ? cudaLaunchKernelEx(&cfg, step_kernel<true>, p) : cudaLaunchKernelEx(&cfg, step_kernel<false>, p);
 }
 
 }  // namespace fm
