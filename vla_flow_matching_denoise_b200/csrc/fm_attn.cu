@@ -3,32 +3,29 @@
 // attention over the cached prefix keys and the chunk's own keys, pack_gqa).
 //
 // One CTA per (request b, KV group g, block of 128 query rows of that group:
-// row (h % G) T + t for the group's G heads and the chunk's T tokens), four
-// warps; thread i owns query row i (TMEM lane i of the M = 128 accumulators).
+// row (h % G) T + t for the group's G heads and the chunk's T tokens), eight
+// warps; query row i (TMEM lane i of the M = 128 accumulators) belongs to lane
+// i % 32 of warps i / 32 and i / 32 + 4, which split its keys and columns.
+// Two CTAs share an SM (256 TMEM columns and ~99 KB of shared memory each), so
+// one CTA's loads and tensor-core work overlap the other's softmax.
 //   1. Thread 0 moves Q rows and, per 128-key chunk, K and V rows into shared
 //      memory with one TMA copy per 64-element half of 128 rows (4-D views
 //      (64 elements, half, row, segment) of the q buffer and the caches): both
 //      store each row's 16-byte pieces swizzled by (row & 7), so every 128-byte
 //      half row is already a row of the 128-byte-swizzled image tcgen05 reads,
-//      and the copy lands as [half][128 rows][128 B].  K and V are
-//      double-buffered and stream while the tensor cores work.
-//   2. S = Q K^T for every chunk (up to 3 x 128 keys) accumulates in TMEM
-//      columns [128 c, 128 c + 128) (K is the K-major B operand).
-//   3. Each thread reads its S row twice: the row maximum, then
-//      p = exp2(s log2(e) / sqrt(hd) - max) for valid keys (0 for the padding
-//      keys of the last chunk), summing l in fp32 and storing p as bf16 into
-//      the K-major image of P (over the Q and K buffers, which S has
-//      finished with).  Every key is in TMEM at once, so the softmax is exact
-//      in one pass and O is never rescaled.
-//   4. O = P V accumulates in TMEM columns [384, 384 + hd); V rows, hd
-//      contiguous, are the MN-major B operand as they arrive.
-//   5. o = O / l in bf16 goes to the ACT128 activation of o_proj.
-// Rows past the request's P_b + T (up to the cache's row count) hold finite
-// values the kernels wrote earlier, rows past the cache are filled with zeros
-// by the copy: their scores are masked and their probabilities are exactly 0.
-// Query rows beyond G T stay in their own rows, which are not stored.
-// Requests are independent and every sum runs in a fixed order
-// (bit-reproducible).
+//      and the copy lands as [half][128 rows][128 B].
+//   2. Pass 1, per chunk: S = Q K^T into TMEM columns [0, 128) (K is the
+//      K-major B operand); each thread reads its half of the chunk's S row
+//      and keeps the running row maximum.  The two halves meet in shared
+//      memory: m = the row maximum over every key.
+//   3. Pass 2, per chunk: S = Q K^T again (a 128-key MMA costs ~0.25 us), p =
+//      exp2(s log2(e) / sqrt(hd) - m) for valid keys (0 for the padding keys
+//      of the last chunk) in bf16 into the K-major image of P (over K, which
+//      the MMA has finished with), l += p in fp32, then O += P V in TMEM
+//      columns [128, 128 + hd); V rows, hd contiguous, are the MN-major B
+//      operand as they arrive.  The maximum is final before any p is formed,
+//      so the softmax is exact and O is never rescaled.
+//   4. o = O / l in bf16 goes to the ACT128 activation of o_proj.
 #include <cuda_bf16.h>
 #include <cstddef>
 #include <cstdint>
@@ -41,24 +38,24 @@ namespace fm {
 
 namespace {
 
-constexpr int kAtThreads = 128;
+constexpr int kAtThreads = 256;          // 8 warps: two per TMEM lane quarter
 constexpr int kAtRows = 128;            // query rows per CTA (MMA M)
 constexpr int kAtChunk = 128;           // keys per chunk (MMA N of S, K of O)
 constexpr int kAtMaxChunks = 3;
 constexpr int kAtTile = kAtRows * 128;  // bytes of one 128-row x 128-byte image
-constexpr int kOCol = kAtMaxChunks * kAtChunk;   // first TMEM column of O
+constexpr int kOCol = kAtChunk;         // first TMEM column of O (S takes [0, 128))
+constexpr int kAtTmem = 256;            // TMEM columns per CTA (two CTAs per SM)
 
-// Barriers: Q, K buffers (2), V buffers (2), S per chunk (3), O per chunk (3).
-enum { BQ = 0, BK = 1, BV = 3, BS = 5, BO = 8, kAtBars = 11 };
+// Barriers: Q loaded, K chunk loaded, V chunk loaded, S MMA done, PV MMA done
+// (each completes once per use; waits alternate parity).
+enum { BQ = 0, BK = 1, BV = 2, BS = 3, BO = 4, kAtBars = 5 };
 
 template <int HD>
 struct AtCfg {
-  static constexpr int kHalves = HD / 64;                   // 128-byte halves of a row
-  static constexpr int kImg = kHalves * kAtTile;            // Q / K / V image: [half][128 rows][128 B]
+  static constexpr int kImg = (HD / 64) * kAtTile;          // Q / K / V image: [half][128 rows][128 B]
   static constexpr int kPBytes = 2 * kAtTile;               // P chunk: [key half][128 rows][128 B]
-  // region A: Q, K0, K1 (later P of 3 chunks); region V: V0, V1
-  static constexpr int kRegA = 3 * kImg > kAtMaxChunks * kPBytes ? 3 * kImg : kAtMaxChunks * kPBytes;
-  static constexpr int kSmem = 1024 + kRegA + 2 * kImg + 256;
+  static constexpr int kKP = kImg > kPBytes ? kImg : kPBytes;   // K chunk, then P of that chunk
+  static constexpr int kSmem = 1024 + kImg + kKP + kImg + 256 + 2 * 2 * kAtRows * 4;
 };
 
 __device__ __forceinline__ uint32_t pk_bf16(float lo, float hi) {
@@ -79,17 +76,18 @@ __device__ __forceinline__ void tma_tile(uint8_t* dst, const CUtensorMap* tm, in
 }  // namespace
 
 template <int HD>
-__global__ void __launch_bounds__(kAtThreads, 1) battn_tc_kernel(const __grid_constant__ BAttnParams p) {
+__global__ void __launch_bounds__(kAtThreads, 2) battn_tc_kernel(const __grid_constant__ BAttnParams p) {
   using C = AtCfg<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* qs = sm;                                    // region A
-  uint8_t* kbuf[2] = {sm + C::kImg, sm + 2 * C::kImg};
-  uint8_t* ps = sm;                                    // region A again, once S is complete
-  uint8_t* vbuf[2] = {sm + C::kRegA, sm + C::kRegA + C::kImg};
-  uint64_t* bars = reinterpret_cast<uint64_t*>(sm + C::kRegA + 2 * C::kImg);
+  uint8_t* qs = sm;
+  uint8_t* kp = sm + C::kImg;                          // K chunk, then P of that chunk
+  uint8_t* vs = sm + C::kImg + C::kKP;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(vs + C::kImg);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(bars + kAtBars + 1);
+  float* red = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);   // [2 halves][128 rows]
   const int tid = threadIdx.x, warp = tid >> 5;
+  const int half = warp >> 2, row = 32 * (warp & 3) + (tid & 31);   // row = TMEM lane
   const int qb = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
   const int G = p.Hq / p.Hkv, T = p.T;
   const int nq = G * T;                                // query rows of the group
@@ -100,7 +98,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) battn_tc_kernel(const __grid_co
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(smem_u32(tslot), 512);
+    tmem_alloc(smem_u32(tslot), kAtTmem);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -111,133 +109,156 @@ __global__ void __launch_bounds__(kAtThreads, 1) battn_tc_kernel(const __grid_co
 
   const int S = p.P_dev[b] + T;                       // keys of this request
   const int nch = (S + kAtChunk - 1) / kAtChunk;
+  const int qseg = b * p.Hkv + g, kvseg = p.seg_base + qseg;
+  // K and V rows serve the group's other query blocks too: keep them in L2
+  const uint64_t pol_q = policy_evict_first(), pol_kv = policy_evict_last();
+  const uint32_t id_s = idesc_bf16(kAtRows, kAtChunk), id_o = idesc_bf16_bmn(kAtRows, HD);
+  const uint32_t trow = tmem + ((uint32_t)(32 * (warp & 3)) << 16);
+  const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
+  const int cb = half * (kAtChunk / 2);                // this thread's 64 columns of a chunk
   bool ok = true;
 
-  // 1: Q, the first two K chunks and the first two V chunks start streaming
-  const int qseg = b * p.Hkv + g, kvseg = p.seg_base + qseg;
   if (tid == 0) {
-    // K and V rows serve the group's other query blocks too: keep them in L2
-    const uint64_t pol = policy_evict_first(), pol_kv = policy_evict_last();
-    tma_tile<HD>(qs, &p.tm_q, qb * kAtRows, qseg, smem_u32(&bars[BQ]), pol);
-    for (int c = 0; c < nch && c < 2; ++c) {
-      tma_tile<HD>(kbuf[c], &p.tm_k, c * kAtChunk, kvseg, smem_u32(&bars[BK + c]), pol_kv);
-      tma_tile<HD>(vbuf[c], &p.tm_v, c * kAtChunk, kvseg, smem_u32(&bars[BV + c]), pol_kv);
-    }
+    tma_tile<HD>(qs, &p.tm_q, qb * kAtRows, qseg, smem_u32(&bars[BQ]), pol_q);
+    tma_tile<HD>(kp, &p.tm_k, 0, kvseg, smem_u32(&bars[BK]), pol_kv);
+    tma_tile<HD>(vs, &p.tm_v, 0, kvseg, smem_u32(&bars[BV]), pol_kv);
   }
   __syncwarp();
 
-  // 2: S = Q K^T per chunk (thread 32 issues); a third K chunk reuses buffer 0
-  const uint32_t id_s = idesc_bf16(kAtRows, kAtChunk);
-  if (tid == 32) {
-    ok &= mbar_wait(smem_u32(&bars[BQ]), 0, budget);
-    for (int c = 0; c < nch; ++c) {
-      ok &= mbar_wait(smem_u32(&bars[BK + (c & 1)]), (uint32_t)(c >> 1), budget);
+  float mx = -INFINITY, mb = 0.f, l = 0.f;
+  for (int i = 0; i < 2 * nch; ++i) {
+    const int c = i < nch ? i : i - nch;
+    const bool second = i >= nch;
+    // S = Q K_c^T
+    if (tid == 32) {
+      if (i == 0) ok &= mbar_wait(smem_u32(&bars[BQ]), 0, budget);
+      ok &= mbar_wait(smem_u32(&bars[BK]), (uint32_t)(i & 1), budget);
       tc_fence_after();
 #pragma unroll
       for (int k16 = 0; k16 < HD / 16; ++k16) {
         const uint32_t off = (uint32_t)((k16 >> 2) * kAtTile + (k16 & 3) * 32);
-        mma_bf16(tmem + c * kAtChunk, desc_sw128(smem_u32(qs) + off), desc_sw128(smem_u32(kbuf[c & 1]) + off),
-                 id_s, k16 > 0);
+        mma_bf16(tmem, desc_sw128(smem_u32(qs) + off), desc_sw128(smem_u32(kp) + off), id_s, k16 > 0);
       }
-      mma_commit(smem_u32(&bars[BS + c]));
+      mma_commit(smem_u32(&bars[BS]));
     }
-  }
-  __syncwarp();
-  if (tid == 0 && nch > 2) {
-    ok &= mbar_wait(smem_u32(&bars[BS + 0]), 0, budget);
-    tma_tile<HD>(kbuf[0], &p.tm_k, 2 * kAtChunk, kvseg, smem_u32(&bars[BK + 0]), policy_evict_last());
-  }
-  __syncwarp();
-  // every S chunk complete: the last commit covers all earlier MMAs
-  ok &= mbar_wait(smem_u32(&bars[BS + nch - 1]), 0, budget);
-  tc_fence_after();
-
-  // 3: softmax of row `tid` over the S keys; P over region A
-  const uint32_t trow = tmem + ((uint32_t)(32 * warp) << 16);
-  const float sl2 = 1.4426950408889634f / sqrtf((float)HD);
-  float mx = -INFINITY;
-  for (int c0 = 0; c0 < nch * kAtChunk; c0 += 32) {
-    float v[2][16];
-    tmem_ld16(trow + c0, v[0]);
-    tmem_ld16(trow + c0 + 16, v[1]);
-    tmem_ld_wait();
-#pragma unroll
-    for (int j = 0; j < 32; ++j)
-      if (c0 + j < S) mx = fmaxf(mx, v[j >> 4][j & 15]);
-  }
-  const float mb = mx * sl2;
-  float l = 0.f;
-  for (int c0 = 0; c0 < nch * kAtChunk; c0 += 32) {
-    float v[2][16];
-    tmem_ld16(trow + c0, v[0]);
-    tmem_ld16(trow + c0 + 16, v[1]);
-    tmem_ld_wait();
-    uint32_t pk[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) {
-      const float s0 = v[(2 * j) >> 4][(2 * j) & 15], s1 = v[(2 * j + 1) >> 4][(2 * j + 1) & 15];
-      const float e0 = c0 + 2 * j < S ? exp2f(fmaf(s0, sl2, -mb)) : 0.f;
-      const float e1 = c0 + 2 * j + 1 < S ? exp2f(fmaf(s1, sl2, -mb)) : 0.f;
-      l += e0;
-      l += e1;
-      pk[j] = pk_bf16(e0, e1);
-    }
-    // P chunk c0 / 128, key half (c0 % 128) / 64, pieces (c0 % 64) / 8 .. + 3
-    const int c = c0 >> 7, kh = (c0 >> 6) & 1, pc0 = (c0 & 63) >> 3;
-    uint8_t* row = ps + c * C::kPBytes + kh * kAtTile + tid * 128;
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-      *reinterpret_cast<uint4*>(row + (((pc0 + i) ^ (tid & 7)) << 4)) =
-          make_uint4(pk[4 * i], pk[4 * i + 1], pk[4 * i + 2], pk[4 * i + 3]);
-  }
-  fence_proxy_async_smem();
-  tc_fence_before();
-  __syncthreads();
-
-  // 4: O = P V per chunk (V: hd-contiguous rows = MN-major B); a third V
-  // chunk reuses buffer 0 once the first chunk's MMAs are done
-  const uint32_t id_o = idesc_bf16_bmn(kAtRows, HD);
-  if (tid == 32) {
+    __syncwarp();
+    ok &= mbar_wait(smem_u32(&bars[BS]), (uint32_t)(i & 1), budget);
     tc_fence_after();
-    for (int c = 0; c < nch; ++c) {
-      ok &= mbar_wait(smem_u32(&bars[BV + (c & 1)]), (uint32_t)(c >> 1), budget);
+    const int k0 = c * kAtChunk + cb;                  // key index of this thread's first column
+    if (!second) {
+      // pass 1: running maximum over valid keys
+#pragma unroll 1
+      for (int j0 = 0; j0 < kAtChunk / 2; j0 += 32) {
+        float v[2][16];
+        tmem_ld16(trow + cb + j0, v[0]);
+        tmem_ld16(trow + cb + j0 + 16, v[1]);
+        tmem_ld_wait();
+        if (k0 + j0 + 32 <= S) {
+#pragma unroll
+          for (int j = 0; j < 32; ++j) mx = fmaxf(mx, v[j >> 4][j & 15]);
+        } else {
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            if (k0 + j0 + j < S) mx = fmaxf(mx, v[j >> 4][j & 15]);
+        }
+      }
+      tc_fence_before();
+      __syncthreads();   // S read: the next S MMA may overwrite it, the K buffer is free
+      if (tid == 0) {
+        // the next K chunk (pass 2 starts again at chunk 0)
+        tma_tile<HD>(kp, &p.tm_k, (c + 1 < nch ? c + 1 : 0) * kAtChunk, kvseg, smem_u32(&bars[BK]), pol_kv);
+      }
+      if (c == nch - 1) {
+        red[half * kAtRows + row] = mx;
+        __syncthreads();
+        mb = fmaxf(red[row], red[kAtRows + row]) * sl2;
+      }
+      continue;
+    }
+    // pass 2: p = exp2(s sl2 - m) -> P (over the K buffer), l += p
+#pragma unroll 1
+    for (int j0 = 0; j0 < kAtChunk / 2; j0 += 32) {
+      float v[2][16];
+      tmem_ld16(trow + cb + j0, v[0]);
+      tmem_ld16(trow + cb + j0 + 16, v[1]);
+      tmem_ld_wait();
+      uint32_t pk[16];
+      if (k0 + j0 + 32 <= S) {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float e0 = exp2f(fmaf(v[(2 * j) >> 4][(2 * j) & 15], sl2, -mb));
+          const float e1 = exp2f(fmaf(v[(2 * j + 1) >> 4][(2 * j + 1) & 15], sl2, -mb));
+          l += e0;
+          l += e1;
+          pk[j] = pk_bf16(e0, e1);
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const float s0 = v[(2 * j) >> 4][(2 * j) & 15], s1 = v[(2 * j + 1) >> 4][(2 * j + 1) & 15];
+          const float e0 = k0 + j0 + 2 * j < S ? exp2f(fmaf(s0, sl2, -mb)) : 0.f;
+          const float e1 = k0 + j0 + 2 * j + 1 < S ? exp2f(fmaf(s1, sl2, -mb)) : 0.f;
+          l += e0;
+          l += e1;
+          pk[j] = pk_bf16(e0, e1);
+        }
+      }
+      // columns cb + j0 .. + 31 of the chunk: key half (cb + j0) / 64, pieces ((cb + j0) % 64) / 8 .. + 3
+      const int col = cb + j0, kh = col >> 6, pc0 = (col & 63) >> 3;
+      uint8_t* prow = kp + kh * kAtTile + row * 128;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(prow + (((pc0 + q) ^ (row & 7)) << 4)) =
+            make_uint4(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]);
+    }
+    fence_proxy_async_smem();
+    tc_fence_before();
+    __syncthreads();   // P complete, S read
+    if (tid == 32) {
+      ok &= mbar_wait(smem_u32(&bars[BV]), (uint32_t)(c & 1), budget);
       tc_fence_after();
 #pragma unroll
       for (int k16 = 0; k16 < kAtChunk / 16; ++k16) {
         const uint32_t aoff = (uint32_t)((k16 >> 2) * kAtTile + (k16 & 3) * 32);
-        mma_bf16(tmem + kOCol, desc_sw128(smem_u32(ps + c * C::kPBytes) + aoff),
-                 desc_sw128_mn(smem_u32(vbuf[c & 1]) + (uint32_t)k16 * 2048u, kAtTile), id_o, (c | k16) != 0);
+        mma_bf16(tmem + kOCol, desc_sw128(smem_u32(kp) + aoff),
+                 desc_sw128_mn(smem_u32(vs) + (uint32_t)k16 * 2048u, kAtTile), id_o, (c | k16) != 0);
       }
-      mma_commit(smem_u32(&bars[BO + c]));
+      mma_commit(smem_u32(&bars[BO]));
     }
+    __syncwarp();
+    if (tid == 0 && c + 1 < nch) {
+      // the P and V buffers are free once this chunk's PV MMAs are done
+      ok &= mbar_wait(smem_u32(&bars[BO]), (uint32_t)(c & 1), budget);
+      tma_tile<HD>(kp, &p.tm_k, (c + 1) * kAtChunk, kvseg, smem_u32(&bars[BK]), pol_kv);
+      tma_tile<HD>(vs, &p.tm_v, (c + 1) * kAtChunk, kvseg, smem_u32(&bars[BV]), pol_kv);
+    }
+    __syncwarp();
   }
-  __syncwarp();
-  if (tid == 0 && nch > 2) {
-    ok &= mbar_wait(smem_u32(&bars[BO + 0]), 0, budget);
-    tma_tile<HD>(vbuf[0], &p.tm_v, 2 * kAtChunk, kvseg, smem_u32(&bars[BV + 0]), policy_evict_last());
-  }
-  __syncwarp();
-  ok &= mbar_wait(smem_u32(&bars[BO + nch - 1]), 0, budget);
+  ok &= mbar_wait(smem_u32(&bars[BO]), (uint32_t)((nch - 1) & 1), budget);
   tc_fence_after();
+  red[half * kAtRows + row] = l;
+  __syncthreads();
+  l = red[row] + red[kAtRows + row];
 
-  // 5: o = O / l -> ACT128 [Mp/128][Hq*hd/64] rows b T + t, columns h hd + e
-  const int qr = qb * kAtRows + tid;
+  // 4: o = O / l -> ACT128 [Mp/128][Hq*hd/64] rows b T + t, columns h hd + e;
+  // each thread of the row takes half of the hd columns
+  const int qr = qb * kAtRows + row;
   const float inv = 1.0f / l;
   const int head = g * G + (qr < nq ? qr / T : 0), t = qr < nq ? qr % T : 0;
   const int m = b * T + t;
   const int K = p.Hq * HD;
-  for (int e0 = 0; e0 < HD; e0 += 32) {
+  for (int e0 = half * (HD / 2); e0 < (half + 1) * (HD / 2); e0 += 32) {
     float v[2][16];
     tmem_ld16(trow + kOCol + e0, v[0]);
     tmem_ld16(trow + kOCol + e0 + 16, v[1]);
     tmem_ld_wait();
     if (qr < nq) {
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const int col = head * HD + e0 + 8 * i;
+      for (int q = 0; q < 4; ++q) {
+        const int col = head * HD + e0 + 8 * q;
         uint16_t* blk = p.o_act + ((size_t)(m >> 7) * (K >> 6) + (col >> 6)) * (kBM * 64);
         const int r = m & 127;
-        const float* x = &v[i >> 1][(i & 1) * 8];
+        const float* x = &v[q >> 1][(q & 1) * 8];
         *reinterpret_cast<uint4*>(blk + r * 64 + ((((col & 63) >> 3) ^ (r & 7)) << 3)) =
             make_uint4(pk_bf16(x[0] * inv, x[1] * inv), pk_bf16(x[2] * inv, x[3] * inv),
                        pk_bf16(x[4] * inv, x[5] * inv), pk_bf16(x[6] * inv, x[7] * inv));
@@ -250,7 +271,7 @@ __global__ void __launch_bounds__(kAtThreads, 1) battn_tc_kernel(const __grid_co
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc(tmem, kAtTmem);
   }
 }
 

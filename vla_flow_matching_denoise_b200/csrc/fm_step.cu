@@ -622,17 +622,18 @@ __device__ __noinline__ void load_rstd(const Ctx& c, const float* sumsq) {
 
 // Sum over the KS senders of two adjacent received columns of row r.
 __device__ __forceinline__ float2 recv_sum2(const float* rb, int KS, int ownp, int r, int lc) {
-  float2 a = make_float2(0.f, 0.f);
+  // every slot's load in flight at once, then the sum in slot order
   const float* p0 = rb + r * ownp + lc;
-#pragma unroll 1
-  for (int s = 0; s < KS; s += 2) {
-    const float2 x = *reinterpret_cast<const float2*>(p0 + s * kRecvRows * ownp);
-    const float2 y = s + 1 < KS ? *reinterpret_cast<const float2*>(p0 + (s + 1) * kRecvRows * ownp)
-                                : make_float2(0.f, 0.f);
-    a.x += x.x;
-    a.y += x.y;
-    a.x += y.x;
-    a.y += y.y;
+  const int stride = kRecvRows * ownp;
+  float2 x[kClusterSize];
+#pragma unroll
+  for (int s = 0; s < kClusterSize; ++s)
+    x[s] = s < KS ? *reinterpret_cast<const float2*>(p0 + s * stride) : make_float2(0.f, 0.f);
+  float2 a = x[0];
+#pragma unroll
+  for (int s = 1; s < kClusterSize; ++s) {
+    a.x += x[s].x;
+    a.y += x[s].y;
   }
   return a;
 }
@@ -1024,13 +1025,18 @@ __device__ __noinline__ void residual_phase(Ctx& c, int g, int f_in, int l, cons
   if (!c.ok) return;
   const float* rb = reinterpret_cast<const float*>(c.work + v.recv_off);
   tmark(c, 8);
+  float2 acc[kMaxPairs];
+#pragma unroll
+  for (int k = 0; k < kMaxPairs; ++k)
+    acc[k] = (k < np && t < T) ? recv_sum2(rb, v.KS, v.ownp, t, 2 * (p0 + k)) : make_float2(0.f, 0.f);
+  tmark(c, 9);
   float sq = 0.f;
 #pragma unroll
   for (int k = 0; k < kMaxPairs; ++k) {
     if (k >= np) break;
     const int hc = hc0 + 2 * k;
     if (t < T) {
-      const float2 a = recv_sum2(rb, v.KS, v.ownp, t, 2 * (p0 + k));
+      const float2 a = acc[k];
       const float n0 = fmaf(gt[k].x, a.x, ho[k].x), n1 = fmaf(gt[k].y, a.y, ho[k].y);
       *reinterpret_cast<float2*>(h_new + (size_t)t * d + hc) = make_float2(n0, n1);
       sq = fmaf(n0, n0, fmaf(n1, n1, sq));
@@ -1042,6 +1048,7 @@ __device__ __noinline__ void residual_phase(Ctx& c, int g, int f_in, int l, cons
   }
   sq += __shfl_xor_sync(0xffffffffu, sq, 1);
   if (hf == 0 && t < T) sumsq[c.cta * kRows + t] = sq;
+  tmark(c, 10);
 }
 
 // gate_up: reduce, rstd + shift row, SwiGLU -> u (bf16, ACT64).  The owned
