@@ -190,7 +190,7 @@ __device__ __forceinline__ void issue_act(const Ctx& c, const uint16_t* src, int
 // this CTA's bulk copies and releases the compute warps.  A GEMM phase passes
 // its K-slice of the activations (`act`, `nch` blocks), which the polling
 // thread requests at once, before the other threads are released.
-__device__ __noinline__ void wait_flag(Ctx& c, int f, const uint16_t* act = nullptr, int nch = 0) {
+__device__ __forceinline__ void wait_flag(Ctx& c, int f, const uint16_t* act = nullptr, int nch = 0) {
   if (!c.ok) return;
   const uint32_t target = c.ep[f] * c.ctl->writers[f];
   if (c.tid == 0) {
@@ -216,7 +216,7 @@ __device__ __noinline__ void wait_flag(Ctx& c, int f, const uint16_t* act = null
 
 // Ends a phase: a writer CTA orders its stores (generic and async proxy)
 // before one release add on counter f; every CTA counts the round.
-__device__ __noinline__ void signal(Ctx& c, int f, bool wrote) {
+__device__ __forceinline__ void signal(Ctx& c, int f, bool wrote) {
   if (c.ok && wrote) {
     tmark(c, 4);
     fence_proxy_async_global();
@@ -522,7 +522,7 @@ __device__ __forceinline__ void arm_recv(const Ctx& c, const GemmView& v) {
 // go to the column's owner as one 16-byte st.async into its receive slot
 // `ks`, completing bytes on the owner's receive barrier.  Owners hold a
 // multiple of 4 columns, so a piece never straddles two owners.
-__device__ __noinline__ void push_send(Ctx& c, const GemmView& v) {
+__device__ __forceinline__ void push_send(Ctx& c, const GemmView& v) {
   if (!c.ok) return;
   Ctrl* const ctl = c.ctl;
   tmark(c, 12);
@@ -577,7 +577,7 @@ __device__ __noinline__ void push_send(Ctx& c, const GemmView& v) {
   tmark(c, 2);
 }
 
-__device__ __noinline__ void push_wait(Ctx& c) {
+__device__ __forceinline__ void push_wait(Ctx& c) {
   if (!c.ok) return;
   if (!wait_ab(smem_u32(&c.ctl->recv), c.recv_count & 1, c.p->spin_budget, &c.ctl->abort)) {
     fail(c, E_RECV);
@@ -590,7 +590,7 @@ __device__ __noinline__ void push_wait(Ctx& c) {
 // rstd[t] = (sum over CTAs of the partial sums of h^2 / d + eps)^-1/2.
 // Thread tid adds rows 4*(tid%16)..+3 of CTAs tid/16 + 8k (independent float4
 // loads, four per round); the eight groups are then added in a fixed order.
-__device__ __noinline__ void load_rstd(const Ctx& c, const float* sumsq) {
+__device__ __forceinline__ void load_rstd(const Ctx& c, const float* sumsq) {
   const int T = c.p->T, n = c.p->n_ctas, d = c.p->d;
   const float eps = c.p->eps;
   const int tid = c.tid;
