@@ -169,7 +169,7 @@ __device__ __forceinline__ void tmark(const Ctx& c, int slot) {
   }
 }
 
-__device__ void fail(Ctx& c, uint32_t code) {
+__device__ __forceinline__ void fail(Ctx& c, uint32_t code) {
   atomicOr(c.p->err, code);
   c.ctl->abort = 1;
   c.ok = false;
@@ -656,7 +656,7 @@ __device__ __forceinline__ PairRows pair_rows(int tid, int npair) {
 
 // QKV: reduce, rstd + shift row, RoPE -> q buffer and the chunk rows of the
 // KV cache.
-__device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
+__device__ __forceinline__ void phase_qkv(Ctx& c, int step, int l) {
   if (!c.ok) return;
   const StepParams& p = *c.p;
   const GemmView v = gemm_view(c, G_QKV);
@@ -728,7 +728,7 @@ __device__ __noinline__ void phase_qkv(Ctx& c, int step, int l) {
 // Attention for one (KV group, 64-row block of the group's G*T query rows);
 // this CTA takes one key range of [prefix ; chunk].
 template <int HD>
-__device__ __noinline__ void attention_unit(Ctx& c, int l, int grp, int blk) {
+__device__ __forceinline__ void attention_unit(Ctx& c, int l, int grp, int blk) {
   const StepParams& p = *c.p;
   constexpr int KSTEPS = HD / 16;
   constexpr int DT = HD / 8;         // n-tiles of the output
@@ -953,7 +953,7 @@ __device__ __noinline__ void attention_unit(Ctx& c, int l, int grp, int blk) {
   }
 }
 
-__device__ __noinline__ void phase_attn(Ctx& c, int l) {
+__device__ __forceinline__ void phase_attn(Ctx& c, int l) {
   const StepParams& p = *c.p;
   if (!c.ok) return;
   const int units = p.Hkv * p.att_blocks;
@@ -986,7 +986,7 @@ __device__ __noinline__ void phase_attn(Ctx& c, int l) {
 // o_proj / down: gated residual on the owned columns, two threads per row t
 // (each half of the owned column pairs); z for the next linear, row sum of
 // squares.  Operands of the epilogue are fetched before the MMAs finish.
-__device__ __noinline__ void residual_phase(Ctx& c, int g, int f_in, int l, const uint16_t* act,
+__device__ __forceinline__ void residual_phase(Ctx& c, int g, int f_in, int l, const uint16_t* act,
                                             const float* h_old, float* h_new, const float* gate,
                                             const float* sc, const float* shift, uint16_t* z, float* sumsq) {
   if (!c.ok) return;
@@ -1053,7 +1053,7 @@ __device__ __noinline__ void residual_phase(Ctx& c, int g, int f_in, int l, cons
 
 // gate_up: reduce, rstd + shift row, SwiGLU -> u (bf16, ACT64).  The owned
 // columns hold own/2 gate rows then own/2 matching up rows.
-__device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
+__device__ __forceinline__ void phase_gu(Ctx& c, int step, int l) {
   if (!c.ok) return;
   const StepParams& p = *c.p;
   const GemmView v = gemm_view(c, G_GU);
@@ -1093,7 +1093,7 @@ __device__ __noinline__ void phase_gu(Ctx& c, int step, int l) {
 
 // In-proj: h = x W_in^T for the residual columns this CTA owns in the down
 // projection (same owners as sumsq_a); z_a for layer0.
-__device__ __noinline__ void phase_inproj(Ctx& c, int step) {
+__device__ __forceinline__ void phase_inproj(Ctx& c, int step) {
   if (!c.ok) return;
   const StepParams& p = *c.p;
   const GemmView v = gemm_view(c, G_DOWN);
@@ -1183,7 +1183,7 @@ __device__ __noinline__ void phase_inproj(Ctx& c, int step) {
 // Final AdaRMSNorm (s_o, b_o) + out-proj + Euler: items (t, a) in order, a
 // contiguous range per warp; the warp keeps y(t) in registers and evaluates
 // up to 4 actions at a time.
-__device__ __noinline__ void phase_outproj(Ctx& c, int step) {
+__device__ __forceinline__ void phase_outproj(Ctx& c, int step) {
   if (!c.ok) return;
   wait_flag(c, F_Z);   // every residual column and its row sums
   const StepParams& p = *c.p;
@@ -1253,7 +1253,7 @@ __device__ __noinline__ void phase_outproj(Ctx& c, int step) {
   }
 }
 
-__device__ void compute_main(Ctx& c) {
+__device__ __forceinline__ void compute_main(Ctx& c) {
   const StepParams& p = *c.p;
   const int L = p.L, d = p.d;
   const size_t zs = (size_t)kRows * d;
