@@ -783,6 +783,13 @@ StepParams base_params(const fm_expert* h) {
   p.step1 = 0;
   p.layer0 = 0;
   p.layer1 = c.n_layers;
+  {
+    const GemmPlan &go = h->plan[G_O], &gd = h->plan[G_DOWN];
+    bool same = go.KS == gd.KS;
+    for (int i = 0; i < kMaxClusters && same; ++i) same = go.ng[i] == gd.ng[i] && go.ch_off[i] == gd.ch_off[i];
+    p.h_regs = same ? 1 : 0;
+  }
+  p.store_mid = 0;
   p.do_inproj = 1;
   p.do_outproj = 1;
   p.update_x = 1;
@@ -1399,6 +1406,7 @@ fm_status fm_trace_velocity(fm_expert* h, const float* x, int step_index, int st
     p.do_inproj = inproj;
     p.do_outproj = outproj;
     p.update_x = 0;
+    p.store_mid = 1;
     CK(cudaMemsetAsync(h->flags, 0, kFlagBytes, st));
     CK(launch_step(p, st));
     CK(cudaStreamSynchronize(st));

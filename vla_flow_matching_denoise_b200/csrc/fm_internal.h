@@ -124,6 +124,8 @@ struct StepParams {
   int step0, step1;          // modulation rows used
   int layer0, layer1;        // layers run per step
   int do_inproj, do_outproj, update_x;
+  int store_mid;             // also store h after the attention residual (h_b; per-layer trace only)
+  int h_regs;                // o_proj and down have the same owners: h stays in registers
   float dt;
   long long spin_budget;     // cycles before a wait gives up
   int stall_test;            // test hook: one writer too many at the QKV hand-off (that wait

@@ -107,6 +107,11 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void* src, uint32_t
       "l"(src), "r"(bytes), "r"(bar), "l"(policy)
       : "memory");
 }
+// Hint: bring [src, src + bytes) into L2 (no completion, no shared memory);
+// src 16-byte aligned, bytes a multiple of 16.
+__device__ __forceinline__ void bulk_prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
 // 4-D tiled TMA load global -> this CTA's shared memory (no multicast),
 // completing tx bytes on `bar`.  `tmap`: generic address of a CUtensorMap
 // kernel parameter (__grid_constant__); the innermost coordinate c0 times the

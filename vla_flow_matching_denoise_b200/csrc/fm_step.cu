@@ -152,6 +152,7 @@ struct Ctx {
   uint32_t recv_count, att_count, xs_count;
   uint32_t phase;       // phases passed (profiling marks)
   uint32_t ep[kNumFlags];   // hand-off rounds signalled so far, per counter
+  float2 hres[4];           // this thread's owned residual values (o_proj and down share owners)
   int P;                // prefix length (read from the device)
   bool ok;
 };
@@ -198,13 +199,15 @@ __device__ __forceinline__ void wait_flag(Ctx& c, int f, const uint16_t* act = n
       const uint32_t* cnt = c.p->flags + f * kFlagStride;
       const long long t0 = clock64();
       uint32_t it = 0;
-      while (ld_acquire_u32(cnt) < target) {
+      // relaxed polls, then one acquire fence (the acquire pattern)
+      while (ld_relaxed_u32(cnt) < target) {
         if ((++it & 15u) == 0u &&
             (*(volatile uint32_t*)c.p->err != 0u || clock64() - t0 > c.p->spin_budget)) {
           fail(c, E_FLAG);
           break;
         }
       }
+      asm volatile("fence.acq_rel.gpu;" ::: "memory");
       fence_proxy_async_global();
     }
     if (act != nullptr && c.ok) issue_act(c, act, nch);
@@ -246,9 +249,22 @@ __device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* 
   uint32_t st[kRingSlots], en[kRingSlots];
   uint32_t head = 0, tail = 0, pos = 0;
   const uint32_t span0 = p.span_off[cta];
+  // this CTA's bytes of one layer (one contiguous span per layer)
+  uint32_t span = 0;
+  for (int g = 0; g < 4; ++g) span += nch[g] * (bytes[g] >> 7) * rowb[g];
+  // The ring holds less than one layer of this CTA's weights (gate_up alone
+  // can exceed it), so the span of the layer after the one being streamed is
+  // requested into L2 ahead of time: ring refills inside a phase then come
+  // from L2 instead of waiting on HBM.
+  auto prefetch_layer = [&](int l) {
+    const uint8_t* a = p.arena + (size_t)l * p.layer_bytes + span0;
+    for (uint32_t o = 0; o < span; o += 65536u) bulk_prefetch_l2(a + o, min(65536u, span - o));
+  };
+  if (span > 0) prefetch_layer(p.layer0);
   bool good = true;
   for (int s = p.step0; s < p.step1 && good; ++s) {
     for (int l = p.layer0; l < p.layer1 && good; ++l) {
+      if (span > 0 && (l + 1 < p.layer1 || s + 1 < p.step1)) prefetch_layer(l + 1 < p.layer1 ? l + 1 : p.layer0);
       const uint8_t* src = p.arena + (size_t)l * p.layer_bytes + span0;
       for (int g = 0; g < 4 && good; ++g) {
         for (uint32_t i = 0; i < nch[g]; ++i) {
@@ -989,6 +1005,9 @@ __device__ __forceinline__ void phase_attn(Ctx& c, int l) {
 __device__ __forceinline__ void residual_phase(Ctx& c, int g, int f_in, int l, const uint16_t* act,
                                             const float* h_old, float* h_new, const float* gate,
                                             const float* sc, const float* shift, uint16_t* z, float* sumsq) {
+  // h_old == nullptr: the residual rows are this thread's registers (the
+  // previous residual phase ran on the same owners and thread mapping);
+  // h_new == nullptr: the new rows stay in registers only
   if (!c.ok) return;
   const GemmView v = gemm_view(c, g);
   if (v.ng == 0) return;
@@ -1016,10 +1035,12 @@ __device__ __forceinline__ void residual_phase(Ctx& c, int g, int f_in, int l, c
   }
   wait_flag(c, f_in, act + (size_t)(v.ks * v.nchunk) * (kRows * 64), v.nchunk);
   tmark(c, 11);
-  // the residual rows were stored two hand-offs ago: visible after the wait
+  // global residual rows (first layer of a launch) were stored before an
+  // earlier hand-off: visible after the wait
 #pragma unroll
   for (int k = 0; k < kMaxPairs; ++k)
-    if (k < np && t < T) ho[k] = *reinterpret_cast<const float2*>(h_old + (size_t)t * d + hc0 + 2 * k);
+    if (k < np && t < T)
+      ho[k] = h_old != nullptr ? *reinterpret_cast<const float2*>(h_old + (size_t)t * d + hc0 + 2 * k) : c.hres[k];
   push_send(c, v);
   push_wait(c);
   if (!c.ok) return;
@@ -1038,7 +1059,8 @@ __device__ __forceinline__ void residual_phase(Ctx& c, int g, int f_in, int l, c
     if (t < T) {
       const float2 a = acc[k];
       const float n0 = fmaf(gt[k].x, a.x, ho[k].x), n1 = fmaf(gt[k].y, a.y, ho[k].y);
-      *reinterpret_cast<float2*>(h_new + (size_t)t * d + hc) = make_float2(n0, n1);
+      c.hres[k] = make_float2(n0, n1);
+      if (h_new != nullptr) *reinterpret_cast<float2*>(h_new + (size_t)t * d + hc) = make_float2(n0, n1);
       sq = fmaf(n0, n0, fmaf(n1, n1, sq));
       if (z != nullptr)
         *reinterpret_cast<uint32_t*>(z + act64_off(t, hc)) = pack_bf16(n0 * (1.0f + sv[k].x), n1 * (1.0f + sv[k].y));
@@ -1271,14 +1293,22 @@ __device__ __forceinline__ void compute_main(Ctx& c) {
       signal(c, F_QKV, busy_qkv);
       phase_attn(c, l);
       signal(c, F_O, busy_att);
-      residual_phase(c, G_O, F_O, l, p.o_act + par * kRows * p.Hq * p.hd, p.h_a, p.h_b, mod_vec(p, s, l, 2),
+      // h lives in the owners' registers between the two residual phases
+      // and across layers; it is read from memory at the first layer of a
+      // launch and stored after the last (the out-projection and the next
+      // launch read it there)
+      residual_phase(c, G_O, F_O, l, p.o_act + par * kRows * p.Hq * p.hd,
+                     (l == p.layer0 || !p.h_regs) ? p.h_a : nullptr,
+                     (p.store_mid || !p.h_regs) ? p.h_b : nullptr, mod_vec(p, s, l, 2),
                      mod_vec(p, s, l, 3), mod_vec(p, s, l, 4), p.z_f + par * zs, p.sumsq_f);
       signal(c, F_ZF, busy_o);
       phase_gu(c, s, l);
       signal(c, F_U, busy_gu);
       {
         const bool next = l + 1 < L;
-        residual_phase(c, G_DOWN, F_U, l, p.u_act + par * kRows * p.F, p.h_b, p.h_a, mod_vec(p, s, l, 5),
+        residual_phase(c, G_DOWN, F_U, l, p.u_act + par * kRows * p.F, p.h_regs ? nullptr : p.h_b,
+                       (l + 1 == p.layer1 || !p.h_regs) ? p.h_a : nullptr,
+                       mod_vec(p, s, l, 5),
                        next ? mod_vec(p, s, l + 1, 0) : nullptr, next ? mod_vec(p, s, l + 1, 1) : nullptr,
                        next ? p.z_a + (1 - par) * zs : nullptr, p.sumsq_a);
       }
