@@ -199,15 +199,13 @@ __device__ __forceinline__ void wait_flag(Ctx& c, int f, const uint16_t* act = n
       const uint32_t* cnt = c.p->flags + f * kFlagStride;
       const long long t0 = clock64();
       uint32_t it = 0;
-      // relaxed polls, then one acquire fence (the acquire pattern)
-      while (ld_relaxed_u32(cnt) < target) {
+      while (ld_acquire_u32(cnt) < target) {
         if ((++it & 15u) == 0u &&
             (*(volatile uint32_t*)c.p->err != 0u || clock64() - t0 > c.p->spin_budget)) {
           fail(c, E_FLAG);
           break;
         }
       }
-      asm volatile("fence.acq_rel.gpu;" ::: "memory");
       fence_proxy_async_global();
     }
     if (act != nullptr && c.ok) issue_act(c, act, nch);
@@ -525,8 +523,9 @@ __device__ __forceinline__ float2 wscale2(const Ctx& c, int g, int l, int idx) {
 // here in GEMM g (safe before the input is ready: a peer pushes only after
 // its own input wait, which this CTA's previous phase has released).
 __device__ __forceinline__ void arm_recv(const Ctx& c, const GemmView& v) {
+  // this CTA's own slot is written with plain shared-memory stores
   if (c.tid == 0)
-    mbar_arrive_expect_tx(smem_u32(&c.ctl->recv), (uint32_t)(v.KS * kRecvRows * v.own * 4));
+    mbar_arrive_expect_tx(smem_u32(&c.ctl->recv), (uint32_t)((v.KS - 1) * kRecvRows * v.own * 4));
 }
 
 // Waits for the MMAs and sends rows 0..50 of the fp32 partial sums to the
@@ -578,9 +577,14 @@ __device__ __forceinline__ void push_send(Ctx& c, const GemmView& v) {
       const float rb = __shfl_xor_sync(0xffffffffu, sb, 1);
       if (act && c0 + 8 * j < ng) {
         const uint32_t rk = (uint32_t)(rank0 + o);
-        const uint32_t dst = map_shared_rank(recv_local, rk) + row_bytes + 4u * lc;
-        if (odd) st_async_v4(dst, ra, rb, x[4 * j + 2], x[4 * j + 3], map_shared_rank(bar_local, rk));
-        else st_async_v4(dst, x[4 * j], x[4 * j + 1], ra, rb, map_shared_rank(bar_local, rk));
+        const float e0 = odd ? ra : x[4 * j], e1 = odd ? rb : x[4 * j + 1];
+        const float e2 = odd ? x[4 * j + 2] : ra, e3 = odd ? x[4 * j + 3] : rb;
+        if (rk == (uint32_t)c.rank) {
+          st_shared_v4(recv_local + row_bytes + 4u * lc, e0, e1, e2, e3);
+        } else {
+          const uint32_t dst = map_shared_rank(recv_local, rk) + row_bytes + 4u * lc;
+          st_async_v4(dst, e0, e1, e2, e3, map_shared_rank(bar_local, rk));
+        }
       }
       lc += 8;
       while (lc >= own) {
@@ -593,10 +597,15 @@ __device__ __forceinline__ void push_send(Ctx& c, const GemmView& v) {
   tmark(c, 2);
 }
 
+// Every compute thread waits for the peers' partials, then all meet (this
+// CTA's own slot was stored by all of them) and agree on the outcome, so a
+// wait that gives up sends every thread the same way.
 __device__ __forceinline__ void push_wait(Ctx& c) {
-  if (!c.ok) return;
-  if (!wait_ab(smem_u32(&c.ctl->recv), c.recv_count & 1, c.p->spin_budget, &c.ctl->abort)) {
-    fail(c, E_RECV);
+  bool w = c.ok && wait_ab(smem_u32(&c.ctl->recv), c.recv_count & 1, c.p->spin_budget, &c.ctl->abort);
+  w = named_bar_and(1, kComputeWarps * 32, w);
+  if (!w) {
+    if (c.ok) fail(c, E_RECV);
+    c.ok = false;
     return;
   }
   ++c.recv_count;
