@@ -44,6 +44,7 @@
 #include <cuda_bf16.h>
 #include <cstddef>
 #include <cstdint>
+#include <type_traits>
 
 #include "fm_internal.h"
 #include "fm_launch.h"
@@ -75,6 +76,7 @@ struct Ctrl {
   uint64_t att;       // attention tile loads
   uint64_t drain;
   uint64_t xsync;     // cluster rendezvous (8 arrivals)
+  uint32_t ring_st[kRingSlots], ring_en[kRingSlots];   // producer only: chunk ranges in flight
   uint32_t tmem_slot;
   int abort;
   uint32_t writers[kNumFlags];       // CTAs that signal each hand-off per round
@@ -244,7 +246,12 @@ __device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* 
   // widened in place; copy bytes per chunk row: 128 (bf16), 64, 36
   uint32_t rowb[4];
   for (int g = 0; g < 4; ++g) rowb[g] = p.wfmt[g] == 0 ? 128u : p.wfmt[g] == 1 ? 64u : 36u;
-  uint32_t st[kRingSlots], en[kRingSlots];
+  // byte range of every chunk in flight, by barrier slot: in shared memory
+  // (a local array indexed at run time lives in local memory, whose L1
+  // share is small next to 227 KB of shared memory: every scan of the ring
+  // then waited on L2)
+  uint32_t* const st = ctl->ring_st;
+  uint32_t* const en = ctl->ring_en;
   uint32_t head = 0, tail = 0, pos = 0;
   const uint32_t span0 = p.span_off[cta];
   // this CTA's bytes of one layer (one contiguous span per layer)
@@ -663,6 +670,24 @@ __device__ __forceinline__ float2 recv_sum2(const float* rb, int KS, int ownp, i
   return a;
 }
 
+// As recv_sum2 for exactly N senders: no predicated slots (the epilogues call
+// it when the plan's KS equals N; same slot order, same sum).
+template <int N>
+__device__ __forceinline__ float2 recv_sum2n(const float* rb, int ownp, int r, int lc) {
+  const float* p0 = rb + r * ownp + lc;
+  const int stride = kRecvRows * ownp;
+  float2 x[N];
+#pragma unroll
+  for (int s = 0; s < N; ++s) x[s] = *reinterpret_cast<const float2*>(p0 + s * stride);
+  float2 a = x[0];
+#pragma unroll
+  for (int s = 1; s < N; ++s) {
+    a.x += x[s].x;
+    a.y += x[s].y;
+  }
+  return a;
+}
+
 // Fixed item assignment of the epilogues: thread tid takes column pair
 // tid % npair for rows tid / npair + k * (128 / npair).
 struct PairRows {
@@ -733,21 +758,29 @@ __device__ __forceinline__ void phase_qkv(Ctx& c, int step, int l) {
   const float* rstd = c.ctl->rstd;
   const float2 bsh = recv_sum2(rb, v.KS, v.ownp, kBiasRow, 2 * pa.pr);
   tmark(c, 8);
+  // the row loop is instruction-bound (one compute warp per scheduler): the
+  // plan's split (four ways) gets a copy without predicated receive slots
+  auto rows = [&](auto ksn) {
+    constexpr int N = decltype(ksn)::value;
 #pragma unroll 1
-  for (int t = pa.t0, k = 0; t < T; t += pa.dt, ++k) {
-    const float2 a = recv_sum2(rb, v.KS, v.ownp, t, 2 * pa.pr);
-    const float rs = rstd[t];
-    const float y0 = fmaf(rs, a.x, bsh.x) * sc.x, y1 = fmaf(rs, a.y, bsh.y) * sc.y;
-    const int rr = row_off + t;
-    uint16_t* rowp = dst + (size_t)rr * hd;
-    if (kind < 2) {
-      const float2 r = aux[k * 128];
-      rowp[swz(rr, ri)] = bf16_bits(y0 * r.x - y1 * r.y);
-      rowp[swz(rr, ri + half)] = bf16_bits(y1 * r.x + y0 * r.y);
-    } else {
-      *reinterpret_cast<uint32_t*>(rowp + swz(rr, w)) = pack_bf16(y0, y1);
+    for (int t = pa.t0, k = 0; t < T; t += pa.dt, ++k) {
+      const float2 a = N > 0 ? recv_sum2n<(N > 0 ? N : 1)>(rb, v.ownp, t, 2 * pa.pr)
+                             : recv_sum2(rb, v.KS, v.ownp, t, 2 * pa.pr);
+      const float rs = rstd[t];
+      const float y0 = fmaf(rs, a.x, bsh.x) * sc.x, y1 = fmaf(rs, a.y, bsh.y) * sc.y;
+      const int rr = row_off + t;
+      uint16_t* rowp = dst + (size_t)rr * hd;
+      if (kind < 2) {
+        const float2 r = aux[k * 128];
+        rowp[swz(rr, ri)] = bf16_bits(y0 * r.x - y1 * r.y);
+        rowp[swz(rr, ri + half)] = bf16_bits(y1 * r.x + y0 * r.y);
+      } else {
+        *reinterpret_cast<uint32_t*>(rowp + swz(rr, w)) = pack_bf16(y0, y1);
+      }
     }
-  }
+  };
+  if (v.KS == 4) rows(std::integral_constant<int, 4>{});
+  else rows(std::integral_constant<int, 0>{});
 }
 
 // Attention for one (KV group, 64-row block of the group's G*T query rows);
@@ -1109,17 +1142,24 @@ __device__ __forceinline__ void phase_gu(Ctx& c, int step, int l) {
   const float2 bg = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lg);
   const float2 bu = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lu);
   tmark(c, 8);
+  // instruction-bound row loop: the plan's split (two ways) gets a copy
+  // without predicated receive slots
+  auto rows = [&](auto ksn) {
+    constexpr int N = decltype(ksn)::value;
 #pragma unroll 1
-  for (int t = pa.t0; t < T; t += pa.dt) {
-    const float2 ag = recv_sum2(rb, v.KS, v.ownp, t, lg);
-    const float2 au = recv_sum2(rb, v.KS, v.ownp, t, lu);
-    const float rs = rstd[t];
-    const float g0 = fmaf(rs, ag.x, bg.x) * sg.x, g1 = fmaf(rs, ag.y, bg.y) * sg.y;
-    const float u0 = fmaf(rs, au.x, bu.x) * su.x, u1 = fmaf(rs, au.y, bu.y) * su.y;
-    const float v0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
-    const float v1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
-    *reinterpret_cast<uint32_t*>(u_act + act64_off(t, uc)) = pack_bf16(v0, v1);
-  }
+    for (int t = pa.t0; t < T; t += pa.dt) {
+      const float2 ag = N > 0 ? recv_sum2n<(N > 0 ? N : 1)>(rb, v.ownp, t, lg) : recv_sum2(rb, v.KS, v.ownp, t, lg);
+      const float2 au = N > 0 ? recv_sum2n<(N > 0 ? N : 1)>(rb, v.ownp, t, lu) : recv_sum2(rb, v.KS, v.ownp, t, lu);
+      const float rs = rstd[t];
+      const float g0 = fmaf(rs, ag.x, bg.x) * sg.x, g1 = fmaf(rs, ag.y, bg.y) * sg.y;
+      const float u0 = fmaf(rs, au.x, bu.x) * su.x, u1 = fmaf(rs, au.y, bu.y) * su.y;
+      const float v0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+      const float v1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
+      *reinterpret_cast<uint32_t*>(u_act + act64_off(t, uc)) = pack_bf16(v0, v1);
+    }
+  };
+  if (v.KS == 2) rows(std::integral_constant<int, 2>{});
+  else rows(std::integral_constant<int, 0>{});
 }
 
 // In-proj: h = x W_in^T for the residual columns this CTA owns in the down
