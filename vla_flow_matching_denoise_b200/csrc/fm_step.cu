@@ -182,10 +182,10 @@ __device__ __forceinline__ void fail(Ctx& c, uint32_t code) {
 __device__ __forceinline__ void issue_act(const Ctx& c, const uint16_t* src, int nch) {
   const uint64_t pol = policy_evict_last();
   const uint32_t bar = smem_u32(&c.ctl->act_full);
+  // the K-slice's blocks are consecutive in the ACT64 layout and in the work
+  // region: one copy (fewer requests queued behind the weight stream's)
   mbar_arrive_expect_tx(bar, (uint32_t)nch * 8192u);
-  const uint32_t dst = smem_u32(c.work);
-#pragma unroll 1
-  for (int i = 0; i < nch; ++i) bulk_g2s(dst + i * 8192, src + (size_t)i * (kRows * 64), 8192, bar, pol);
+  bulk_g2s(smem_u32(c.work), src, (uint32_t)nch * 8192u, bar, pol);
 }
 
 // Waits until hand-off counter f has seen every writer of every round
@@ -1139,13 +1139,15 @@ __device__ __forceinline__ void phase_gu(Ctx& c, int step, int l) {
   uint16_t* u_act = p.u_act + (size_t)(l & 1) * kRows * F;
   const int lg = 2 * pa.pr, lu = uown + 2 * pa.pr;
   const float2 sg = wscale2(c, G_GU, l, v.pbase + lg), su = wscale2(c, G_GU, l, v.pbase + lu);
-  const float2 bg = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lg);
-  const float2 bu = recv_sum2(rb, v.KS, v.ownp, kBiasRow, lu);
   tmark(c, 8);
   // instruction-bound row loop: the plan's split (two ways) gets a copy
   // without predicated receive slots
   auto rows = [&](auto ksn) {
     constexpr int N = decltype(ksn)::value;
+    const float2 bg = N > 0 ? recv_sum2n<(N > 0 ? N : 1)>(rb, v.ownp, kBiasRow, lg)
+                            : recv_sum2(rb, v.KS, v.ownp, kBiasRow, lg);
+    const float2 bu = N > 0 ? recv_sum2n<(N > 0 ? N : 1)>(rb, v.ownp, kBiasRow, lu)
+                            : recv_sum2(rb, v.KS, v.ownp, kBiasRow, lu);
 #pragma unroll 1
     for (int t = pa.t0; t < T; t += pa.dt) {
       const float2 ag = N > 0 ? recv_sum2n<(N > 0 ? N : 1)>(rb, v.ownp, t, lg) : recv_sum2(rb, v.KS, v.ownp, t, lg);
