@@ -298,6 +298,15 @@ __device__ __noinline__ void producer(const StepParams& p, uint8_t* ring, Ctrl* 
           if (p.tlog != nullptr && (int)head < p.tlog_chunks)
             p.tlog[(size_t)cta * p.tlog_stride + p.tlog_chunk_off + p.tlog_chunks + head] = gtimer();
           const uint32_t csz = (sz >> 7) * rowb[g];
+          // at most 2 weight copies in flight: a phase's activation copy shares
+          // this SM's bulk-copy engine and must not queue behind a deep stream
+          if (head >= 2u) {
+            const uint32_t q = head - 2u;
+            if (!wait_ab(smem_u32(&ctl->full[q % kRingSlots]), (q / kRingSlots) & 1, p.spin_budget, &ctl->abort)) {
+              good = false;
+              break;
+            }
+          }
           mbar_arrive_expect_tx(smem_u32(&ctl->full[slot]), csz);
           bulk_g2s(smem_u32(ring + at + (sz - csz)), src, csz, smem_u32(&ctl->full[slot]), pol);
           src += csz;
@@ -982,15 +991,19 @@ __device__ __forceinline__ void attention_unit(Ctx& c, int l, int grp, int blk) 
     const int rblk = 8 * rank + rloc;
     if (seg < SEGS && rblk < nrows) {
       const float* src = rb + rloc * RWP;
+      // every sender's (m, l) first (eight loads in flight), then its o terms
+      float2 ml[kClusterSize];
+#pragma unroll
+      for (int s = 0; s < kClusterSize; ++s) ml[s] = *reinterpret_cast<const float2*>(src + s * 8 * RWP + HD);
       float M = -INFINITY;
-#pragma unroll 1
-      for (int s = 0; s < kClusterSize; ++s) M = fmaxf(M, src[s * 8 * RWP + HD]);
+#pragma unroll
+      for (int s = 0; s < kClusterSize; ++s) M = fmaxf(M, ml[s].x);
       float L = 0.f, acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll 1
+#pragma unroll
       for (int s = 0; s < kClusterSize; ++s) {
         const float* sr = src + s * 8 * RWP;
-        const float ls = sr[HD + 1];
-        const float wgt = ls == 0.f ? 0.f : exp2f(sr[HD] - M);
+        const float ls = ml[s].y;
+        const float wgt = ls == 0.f ? 0.f : exp2f(ml[s].x - M);
         L = fmaf(ls, wgt, L);
         const float4 x0 = *reinterpret_cast<const float4*>(sr + 8 * seg);
         const float4 x1 = *reinterpret_cast<const float4*>(sr + 8 * seg + 4);
