@@ -1104,7 +1104,9 @@ __device__ __forceinline__ void residual_phase(Ctx& c, int g, int f_in, int l, c
   float2 acc[kMaxPairs];
 #pragma unroll
   for (int k = 0; k < kMaxPairs; ++k)
-    acc[k] = (k < np && t < T) ? recv_sum2(rb, v.KS, v.ownp, t, 2 * (p0 + k)) : make_float2(0.f, 0.f);
+    acc[k] = (k < np && t < T) ? (v.KS == kClusterSize ? recv_sum2n<kClusterSize>(rb, v.ownp, t, 2 * (p0 + k))
+                                                        : recv_sum2(rb, v.KS, v.ownp, t, 2 * (p0 + k)))
+                               : make_float2(0.f, 0.f);
   tmark(c, 9);
   float sq = 0.f;
 #pragma unroll
