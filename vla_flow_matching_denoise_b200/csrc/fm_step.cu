@@ -161,6 +161,15 @@ struct Ctx {
 
 __device__ __forceinline__ void compute_sync() { named_bar_sync(1, kComputeWarps * 32); }
 
+// Every compute thread passes its view of the phase's health (its own waits
+// and the CTA's abort flag); all leave with the same answer, so a wait that
+// gave up on one thread sends every thread the same way and none is left
+// waiting at a later barrier.
+__device__ __forceinline__ bool compute_vote(const Ctx& c, bool ok) {
+  ok = ok && *(volatile int*)&c.ctl->abort == 0;
+  return named_bar_and(1, kComputeWarps * 32, ok);
+}
+
 // Phase timeline (profiling only): mark `slot` of the current phase: 0 start,
 // 1 MMA / attention compute done, 2 partials pushed, 3 partials received,
 // 4 epilogue done, 5 barrier arrival issued, 6 partials staged, 7 staging
@@ -212,8 +221,7 @@ __device__ __forceinline__ void wait_flag(Ctx& c, int f, const uint16_t* act = n
     }
     if (act != nullptr && c.ok) issue_act(c, act, nch);
   }
-  compute_sync();
-  if (*(volatile int*)&c.ctl->abort) c.ok = false;
+  c.ok = compute_vote(c, c.ok);
   tmark(c, 0);
 }
 
@@ -618,7 +626,7 @@ __device__ __forceinline__ void push_send(Ctx& c, const GemmView& v) {
 // wait that gives up sends every thread the same way.
 __device__ __forceinline__ void push_wait(Ctx& c) {
   bool w = c.ok && wait_ab(smem_u32(&c.ctl->recv), c.recv_count & 1, c.p->spin_budget, &c.ctl->abort);
-  w = named_bar_and(1, kComputeWarps * 32, w);
+  w = compute_vote(c, w);
   if (!w) {
     if (c.ok) fail(c, E_RECV);
     c.ok = false;
@@ -859,9 +867,13 @@ __device__ __forceinline__ void attention_unit(Ctx& c, int l, int grp, int blk) 
         bulk_g2s(va, vg + (size_t)kb * HD, (uint32_t)nk * HD * 2, att_bar, pol);
       }
     }
-    if (!wait_ab(att_bar, c.att_count & 1, budget, &ctl->abort)) {
-      fail(c, E_ATT);
-      return;
+    {
+      const bool w = wait_ab(att_bar, c.att_count & 1, budget, &ctl->abort);
+      if (!w) fail(c, E_ATT);
+      if (!compute_vote(c, w)) {
+        c.ok = false;
+        return;
+      }
     }
     ++c.att_count;
     {
@@ -978,9 +990,13 @@ __device__ __forceinline__ void attention_unit(Ctx& c, int l, int grp, int blk) 
                    blk8, map_shared_rank(bar_local, tid));
   }
   tmark(c, 2);
-  if (!wait_ab(smem_u32(&ctl->recv), c.recv_count & 1, budget, &ctl->abort)) {
-    fail(c, E_RECV);
-    return;
+  {
+    const bool w = wait_ab(smem_u32(&ctl->recv), c.recv_count & 1, budget, &ctl->abort);
+    if (!w) fail(c, E_RECV);
+    if (!compute_vote(c, w)) {
+      c.ok = false;
+      return;
+    }
   }
   ++c.recv_count;
   tmark(c, 3);
@@ -1041,9 +1057,13 @@ __device__ __forceinline__ void phase_attn(Ctx& c, int l) {
         asm volatile("fence.acq_rel.cluster;" ::: "memory");
         for (int r = 0; r < kClusterSize; ++r) mbar_arrive_cluster(smem_u32(&c.ctl->xsync), r);
       }
-      if (!wait_ab(smem_u32(&c.ctl->xsync), c.xs_count & 1, p.spin_budget, &c.ctl->abort)) {
-        fail(c, E_RECV);
-        return;
+      {
+        const bool w = wait_ab(smem_u32(&c.ctl->xsync), c.xs_count & 1, p.spin_budget, &c.ctl->abort);
+        if (!w) fail(c, E_RECV);
+        if (!compute_vote(c, w)) {
+          c.ok = false;
+          return;
+        }
       }
       ++c.xs_count;
     }
