@@ -177,56 +177,80 @@ __device__ __forceinline__ void epi_qkv(const BGemmParams& p, uint32_t ta, int m
   const int b = valid ? m / p.T : 0, t = valid ? m % p.T : 0;
   // chunk: rows and RoPE positions follow this request's prefix length
   const int P = p.P_dev != nullptr ? p.P_dev[b] : 0;
-  const float2* rope = reinterpret_cast<const float2*>(p.rope) + ((size_t)b * p.rope_stride_b + t) * half;
-#pragma unroll 1
-  for (int ho = 0; ho < BN; ho += hd) {
-    const int col0 = nt * BN + ho;
+  const float4* rope4 = reinterpret_cast<const float4*>(reinterpret_cast<const float2*>(p.rope) +
+                                                        ((size_t)b * p.rope_stride_b + t) * half);
+  const int nh = BN / hd;
+  auto dst = [&](int h, int& row) -> uint16_t* {
+    const int col0 = nt * BN + h * hd;
     const int kind = col0 < qn ? 0 : col0 < qn + kn ? 1 : 2;
     const int head = (kind == 0 ? col0 : kind == 1 ? col0 - qn : col0 - qn - kn) / hd;
-    uint16_t* rowp;
-    int row;
     if (kind == 0) {   // (only when Hq > 0)
       row = (head % G) * p.T + t;
-      rowp = p.qbuf + (((size_t)b * p.Hkv + head / G) * p.q_rows + row) * hd;
-    } else {
-      row = P + t;
-      rowp = (kind == 1 ? p.kc : p.vc) + (((size_t)b * p.Hkv + head) * p.S_max + row) * hd;
+      return p.qbuf + (((size_t)b * p.Hkv + head / G) * p.q_rows + row) * hd;
     }
-    if (kind < 2) {
-#pragma unroll 1
-      for (int c = 0; c < half; c += 16) {
-        float lo[16], hi[16];
-        tmem_ld16(ta + ho + c, lo);
-        tmem_ld16(ta + ho + half + c, hi);
-        tmem_ld_wait();
-        if (!valid) continue;
-        if (F8) {
-          dequant16(lo, sa, cs + ho + c);
-          dequant16(hi, sa, cs + ho + half + c);
-        }
-        float ol[16], oh[16];
-        const float4* r4 = reinterpret_cast<const float4*>(rope + c);   // (cos, sin) pairs, 128 B
+    row = P + t;
+    return (kind == 1 ? p.kc : p.vc) + (((size_t)b * p.Hkv + head) * p.S_max + row) * hd;
+  };
+  auto rotated = [&](int h) { return nt * BN + h * hd < qn + kn; };   // q and k heads take RoPE
+  // The tile's q/k heads share this row's (cos, sin) table: each 16-frequency
+  // group is loaded once for all of them, one group ahead of its use, so no
+  // L2 round trip sits between a TMEM read and its stores.
+  float4 rc[8], rn[8];
+  if (valid) {
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float4 r = r4[i];
-          ol[2 * i] = lo[2 * i] * r.x - hi[2 * i] * r.y;
-          oh[2 * i] = hi[2 * i] * r.x + lo[2 * i] * r.y;
-          ol[2 * i + 1] = lo[2 * i + 1] * r.z - hi[2 * i + 1] * r.w;
-          oh[2 * i + 1] = hi[2 * i + 1] * r.z + lo[2 * i + 1] * r.w;
-        }
-        store_row16(rowp, row, c, ol);
-        store_row16(rowp, row, half + c, oh);
-      }
-    } else {
+    for (int i = 0; i < 8; ++i) rc[i] = rope4[i];
+  }
 #pragma unroll 1
-      for (int c = 0; c < hd; c += 16) {
-        float v[16];
-        tmem_ld16(ta + ho + c, v);
-        tmem_ld_wait();
-        if (!valid) continue;
-        if (F8) dequant16(v, sa, cs + ho + c);
-        store_row16(rowp, row, c, v);
+  for (int c = 0; c < half; c += 16) {
+    if (valid && c + 16 < half) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) rn[i] = rope4[(c + 16) / 2 + i];
+    }
+#pragma unroll 1
+    for (int h = 0; h < nh; ++h) {
+      if (!rotated(h)) continue;
+      const int ho = h * hd;
+      float lo[16], hi[16];
+      tmem_ld16(ta + ho + c, lo);
+      tmem_ld16(ta + ho + half + c, hi);
+      tmem_ld_wait();
+      if (!valid) continue;
+      if (F8) {
+        dequant16(lo, sa, cs + ho + c);
+        dequant16(hi, sa, cs + ho + half + c);
       }
+      float ol[16], oh[16];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float4 r = rc[i];
+        ol[2 * i] = lo[2 * i] * r.x - hi[2 * i] * r.y;
+        oh[2 * i] = hi[2 * i] * r.x + lo[2 * i] * r.y;
+        ol[2 * i + 1] = lo[2 * i + 1] * r.z - hi[2 * i + 1] * r.w;
+        oh[2 * i + 1] = hi[2 * i + 1] * r.z + lo[2 * i + 1] * r.w;
+      }
+      int row;
+      uint16_t* rowp = dst(h, row);
+      store_row16(rowp, row, c, ol);
+      store_row16(rowp, row, half + c, oh);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) rc[i] = rn[i];
+  }
+  // v heads: no rotation
+#pragma unroll 1
+  for (int h = 0; h < nh; ++h) {
+    if (rotated(h)) continue;
+    const int ho = h * hd;
+    int row;
+    uint16_t* rowp = dst(h, row);
+#pragma unroll 1
+    for (int c = 0; c < hd; c += 16) {
+      float v[16];
+      tmem_ld16(ta + ho + c, v);
+      tmem_ld_wait();
+      if (!valid) continue;
+      if (F8) dequant16(v, sa, cs + ho + c);
+      store_row16(rowp, row, c, v);
     }
   }
 }
