@@ -1312,37 +1312,76 @@ __device__ __forceinline__ void phase_outproj(Ctx& c, int step) {
   const int total = T * A;
   const int per = (total + nw - 1) / nw;
   const int i0 = gw * per, i1 = min(total, i0 + per);
-  constexpr int MAXV = 32;   // d <= 1024
-  float y[MAXV];
+  // Lane l takes inputs 256 c + 8 l .. + 7 (c < 4, d <= 1024): one 16-byte
+  // load per 8 weights, and every load of a row or a weight pair is in flight
+  // at once (the per-element loop had one L2 round trip per few loads).
+  constexpr int kC = 4;
+  float y[8 * kC];
   int it = i0;
 #pragma unroll 1
   while (it < i1) {
     const int t = it / A;
     const int iend = min(i1, (t + 1) * A);
     {
+      float q6[kMaxClusters * kClusterSize / 32];
+#pragma unroll
+      for (int j = 0; j < kMaxClusters * kClusterSize / 32; ++j) {
+        const int q = lane + 32 * j;
+        q6[j] = q < n_ctas ? sumsq[q * kRows + t] : 0.f;
+      }
       float s = 0.f;
-#pragma unroll 1
-      for (int q = lane; q < n_ctas; q += 32) s += sumsq[q * kRows + t];
+#pragma unroll
+      for (int j = 0; j < kMaxClusters * kClusterSize / 32; ++j) s += q6[j];
       for (int o = 16; o; o >>= 1) s += __shfl_xor_sync(0xffffffffu, s, o);
       const float rs = 1.0f / sqrtf(s / (float)d + eps);
+      // one chunk per wave (its six loads in flight together)
 #pragma unroll
-      for (int i = 0; i < MAXV; ++i) {
-        const int k = lane + 32 * i;
-        y[i] = k < d ? fmaf(h_a[(size_t)t * d + k] * rs, 1.0f + s_o[k], b_o[k]) : 0.f;
+      for (int c = 0; c < kC; ++c) {
+        const int k0 = 256 * c + 8 * lane;
+        float4 hv[2], sv[2], bv[2];
+        if (k0 < d) {
+#pragma unroll
+          for (int j = 0; j < 2; ++j) {
+            hv[j] = *reinterpret_cast<const float4*>(h_a + (size_t)t * d + k0 + 4 * j);
+            sv[j] = *reinterpret_cast<const float4*>(s_o + k0 + 4 * j);
+            bv[j] = *reinterpret_cast<const float4*>(b_o + k0 + 4 * j);
+          }
+        }
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+          const float4 h4 = hv[j], s4 = sv[j], b4 = bv[j];
+          float* yy = y + 8 * c + 4 * j;
+          const bool in = k0 < d;
+          yy[0] = in ? fmaf(h4.x * rs, 1.0f + s4.x, b4.x) : 0.f;
+          yy[1] = in ? fmaf(h4.y * rs, 1.0f + s4.y, b4.y) : 0.f;
+          yy[2] = in ? fmaf(h4.z * rs, 1.0f + s4.z, b4.z) : 0.f;
+          yy[3] = in ? fmaf(h4.w * rs, 1.0f + s4.w, b4.w) : 0.f;
+        }
       }
     }
     if (it == i0) tmark(c, 8);
 #pragma unroll 1
     for (; it < iend; it += 2) {
-      float dot0 = 0.f, dot1 = 0.f;
       const bool two = it + 1 < iend;
       const uint16_t* w = w_out + (size_t)(it - t * A) * d;
+      uint4 w0[kC], w1[kC];
 #pragma unroll
-      for (int i = 0; i < MAXV; ++i) {
-        const int k = lane + 32 * i;
-        if (k < d) {
-          dot0 = fmaf(y[i], __uint_as_float((uint32_t)w[k] << 16), dot0);
-          if (two) dot1 = fmaf(y[i], __uint_as_float((uint32_t)w[k + d] << 16), dot1);
+      for (int c = 0; c < kC; ++c) {
+        const int k0 = 256 * c + 8 * lane;
+        w0[c] = k0 < d ? *reinterpret_cast<const uint4*>(w + k0) : make_uint4(0u, 0u, 0u, 0u);
+        w1[c] = (two && k0 < d) ? *reinterpret_cast<const uint4*>(w + d + k0) : make_uint4(0u, 0u, 0u, 0u);
+      }
+      float dot0 = 0.f, dot1 = 0.f;
+#pragma unroll
+      for (int c = 0; c < kC; ++c) {
+        const uint32_t a[4] = {w0[c].x, w0[c].y, w0[c].z, w0[c].w};
+        const uint32_t b[4] = {w1[c].x, w1[c].y, w1[c].z, w1[c].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          dot0 = fmaf(y[8 * c + 2 * e], __uint_as_float(a[e] << 16), dot0);
+          dot0 = fmaf(y[8 * c + 2 * e + 1], __uint_as_float(a[e] & 0xFFFF0000u), dot0);
+          dot1 = fmaf(y[8 * c + 2 * e], __uint_as_float(b[e] << 16), dot1);
+          dot1 = fmaf(y[8 * c + 2 * e + 1], __uint_as_float(b[e] & 0xFFFF0000u), dot1);
         }
       }
       for (int o = 16; o; o >>= 1) {
