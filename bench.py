@@ -47,9 +47,9 @@ UNIT = "denoise steps/s"
 NCU_TRAFFIC = {
     # step_kernel, bench workload: dram__bytes_read.sum + dram__bytes_write.sum of one
     # `python bench.py --workload lingbot_l4_p256_n10 --once` launch (4 layers x 1 Euler
-    # step: 140.575 + 3.129 MB), scaled by the 90x layer-steps of a 36-layer, 10-step
+    # step: 140.582 + 3.483 MB), scaled by the 90x layer-steps of a 36-layer, 10-step
     # launch (weight and KV traffic grow in proportion).
-    "lingbot_p256_n10": {"source_hash": "76fddef9a1c58ac5", "dram_bytes": 143.704e6 * 90},
+    "lingbot_p256_n10": {"source_hash": "27f9fee91c0e1644", "dram_bytes": 144.066e6 * 90},
 }
 
 

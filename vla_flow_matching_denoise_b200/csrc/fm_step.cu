@@ -1215,7 +1215,8 @@ __device__ __forceinline__ void phase_inproj(Ctx& c, int step) {
   {
     const float2* x2 = reinterpret_cast<const float2*>(p.x);
     const int n2 = T * A / 2;
-#pragma unroll 1
+    // unrolled: several batches of loads in flight (same stores)
+#pragma unroll 4
     for (int i = tid; i < n2; i += 4 * 128) {
       float2 xv[4];
 #pragma unroll
@@ -1226,7 +1227,7 @@ __device__ __forceinline__ void phase_inproj(Ctx& c, int step) {
     }
     const uint16_t* w = p.w_in + (size_t)base * A;
     const int nw = min(own, d - base) * A;
-#pragma unroll 1
+#pragma unroll 4
     for (int i = tid; i < own * A; i += 4 * 128) {
       uint16_t wv[4];
 #pragma unroll
@@ -1257,7 +1258,8 @@ __device__ __forceinline__ void phase_inproj(Ctx& c, int step) {
       const float* xr = xs + t * A;
       float a0 = 0.f, a1 = 0.f, c0 = 0.f, c1 = 0.f;
       int k = 0;
-#pragma unroll 1
+      // unrolled for independent loads; each accumulator's order is unchanged
+#pragma unroll 4
       for (; k + 2 <= A; k += 2) {
         a0 = fmaf(xr[k], w0[k], a0);
         a1 = fmaf(xr[k], w1[k], a1);
