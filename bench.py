@@ -23,6 +23,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -49,15 +50,20 @@ NCU_TRAFFIC = {
     # `python bench.py --workload lingbot_l4_p256_n10 --once` launch (4 layers x 1 Euler
     # step: 140.582 + 3.483 MB), scaled by the 90x layer-steps of a 36-layer, 10-step
     # launch (weight and KV traffic grow in proportion).
-    "lingbot_p256_n10": {"source_hash": "27f9fee91c0e1644", "dram_bytes": 144.066e6 * 90},
+    "lingbot_p256_n10": {"source_hash": "4c8f763fcfd0d301", "dram_bytes": 144.066e6 * 90},
 }
 
 
 def kernel_source_hash() -> str:
+    """Hash of the loop kernel's sources with comments and blank space removed
+    (a comment edit does not change the kernel the counters were taken on)."""
     h = hashlib.sha256()
     for f in ("fm_step.cu", "fm_ptx.cuh", "fm_internal.h"):
-        with open(os.path.join(ROOT, "vla_flow_matching_denoise_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+        with open(os.path.join(ROOT, "vla_flow_matching_denoise_b200", "csrc", f), encoding="utf-8") as fh:
+            text = fh.read()
+        text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+        text = re.sub(r"//[^\n]*", "", text)
+        h.update(re.sub(r"\s+", " ", text).strip().encode())
     return h.hexdigest()[:16]
 
 

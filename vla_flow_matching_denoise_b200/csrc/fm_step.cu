@@ -12,20 +12,26 @@
 //    is no grid barrier: each phase's writers add 1 to that phase's counter
 //    in global memory (release) once their outputs are stored, and a phase
 //    waits (acquire, bounded spin) only for the counter of the outputs it
-//    reads, right before it reads them.  Activations alternate between two
-//    copies by layer parity.
+//    reads, right before it reads them; the polling thread then requests the
+//    CTA's K-slice of the activations with one bulk copy.  Activations
+//    alternate between two copies by layer parity.  Every wait of the compute
+//    warps ends in a vote, so a wait that gives up sends them all the same way.
 //  * Weights dominate the bytes (34.6 MB per layer at d = 1024), so warp 0 of
 //    every CTA streams its share of every layer, in consumption order, through
-//    a 126 KB shared-memory ring with 1-D bulk (TMA) copies.  The stream runs
-//    ahead across phases; only ring space throttles it.
+//    a 126 KB shared-memory ring with 1-D bulk (TMA) copies, and requests the
+//    next layer's span into L2 ahead of time.  The stream runs ahead across
+//    phases, throttled by ring space and by at most two copies in flight (the
+//    activation copies share the SM's bulk-copy engine).
 //  * Each linear is split over clusters by output channels and, inside a
 //    cluster, over its 8 CTAs by K and n-groups.  Warp 1 issues tcgen05.mma
 //    with M = 64 token rows (50 valid + the shift row + padding), N = the
 //    CTA's channels, accumulating fp32 in TMEM.
 //  * Split-K partials leave TMEM through tcgen05.ld straight into registers
 //    and go to the owner of each column with st.async into the owner's shared
-//    memory, completing bytes on its mbarrier; the owner reduces its KS slots
-//    in a fixed order (results are bit-reproducible).
+//    memory, completing bytes on its mbarrier (a CTA's own slot with plain
+//    shared stores); the owner reduces its KS slots in a fixed order (results
+//    are bit-reproducible).  o_proj and down have the same owners, which keep
+//    the residual stream h in registers across phases and layers.
 //  * AdaRMSNorm is folded into the linears: the owner of a residual column
 //    writes z = bf16(h (1 + s)) and, in row 50, the shift b; the consumer
 //    linear's epilogue applies rstd(row) to rows 0..49 and adds row 50
