@@ -51,3 +51,19 @@ def test_batched_flops_per_call(name):
     want = 10 * (lin + att)
     assert bench.loop_flops(synth.WORKLOADS[name], 10, 64) == pytest.approx(want, rel=1e-12)
     assert want == pytest.approx(42.76e12, rel=1e-3)
+
+
+def test_kernel_hash_ignores_comments_but_not_code(tmp_path, monkeypatch):
+    # the traffic figure stays attached to an unchanged kernel across comment
+    # edits, and is dropped when the code changes
+    src = tmp_path / "vla_flow_matching_denoise_b200" / "csrc"
+    src.mkdir(parents=True)
+    names = ("fm_step.cu", "fm_ptx.cuh", "fm_internal.h")
+    for n in names:
+        (src / n).write_text("int f(int x) {\n  return x + 1;  // add one\n}\n/* block */\n")
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    h0 = bench.kernel_source_hash()
+    (src / "fm_step.cu").write_text("// a new header\nint f(int x) {\n    return x + 1;  // plus one\n}\n")
+    assert bench.kernel_source_hash() == h0
+    (src / "fm_step.cu").write_text("int f(int x) {\n  return x + 2;\n}\n")
+    assert bench.kernel_source_hash() != h0
